@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of one hybrid block (1 full layer + N sparse layers) on B200.
+
+Workload (default): HySparse block-level prefill, 1 x 32768 tokens, 32 query
+heads / 8 KV heads, d = 128, 64-token blocks, top-16, separate SWA window 128
++ sigmoid gate, 1 full layer feeding 3 sparse layers; seeded synthetic bf16
+N(0,1) inputs with 1 % planted keys. A "step" is one pass of the whole block:
+hs_full_attn_select -> hs_topk_select -> 3 x (hs_sparse_attn_prefill ->
+hs_swa_gated). The per-step working set (~2 GB) is larger than the 126 MB L2.
+
+Multi-GPU (torchrun): every rank runs its own independent block (its own
+sequences); no data-path collective. value = tokens of all ranks / max-over-
+ranks time ("weak" scaling).
+
+--impl reference: the fp64 CPU oracle on host cores, timed on a bounded
+sample of the same workload (one selection tile of 64 queries per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "hybrid-block attn tokens/s; TFLOP/s & HBM GB/s as % of roofline (1×B200)"
+KERNEL_SOURCES = ["hybrid_sparse_attention_tma_b200/csrc/attn_fwd.cuh",
+                  "hybrid_sparse_attention_tma_b200/csrc/hs_common.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="hys_block", choices=list(W.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def causal_pairs(w: W.Workload) -> int:
+    tot = 0
+    for c, n in zip(w.ctx, w.new):
+        # queries at positions c..c+n-1 see pos+1 keys
+        tot += n * (c + 1) + n * (n - 1) // 2
+    return tot
+
+
+def full_flops(w: W.Workload) -> float:
+    return 4.0 * w.head_dim * w.n_q_heads * causal_pairs(w)
+
+
+def src_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel}:{workload}")
+    if not e or e.get("src_hash") != src_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu),
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_runner(w, device, seed):
+    import hybrid_sparse_attention_tma_b200 as hs
+    from hybrid_sparse_attention_tma_b200.block import HybridBlock, SparseLayerIn
+    inp = W.make_block_inputs(w, device=device, seed=seed)
+    vl = hs.Varlen(w.cu_q(), w.cu_kv(), w.n_q_heads, w.n_kv_heads, w.head_dim, device=device)
+    blk = HybridBlock(vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device)
+    layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
+    return inp, vl, blk, layers
+
+
+def bench_ours(args, world, rank, local):
+    import torch.distributed as dist
+    device = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    w = W.WORKLOADS[args.workload]
+    inp, vl, blk, layers = make_runner(w, device, seed=1000 + w.config_index + 7919 * rank)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return blk.forward(inp.q, inp.k, inp.v, layers, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    import hybrid_sparse_attention_tma_b200 as hs
+    hs.check_error(blk.ws)
+
+    # per-kernel events for the dominant kernel (full attention + select)
+    full_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    from hybrid_sparse_attention_tma_b200 import full_attn_select, topk_select, sparse_attn_prefill, swa_gated
+
+    def step_instrumented(i):
+        sel = blk.sel
+        bufs = blk._bufs
+        full_ev[i][0].record(stream)
+        full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"], bufs["scores"],
+                         ws=blk.ws, stream=stream)
+        full_ev[i][1].record(stream)
+        topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws, stream=stream)
+        for j, L in enumerate(layers):
+            tag = str(j % 2)
+            sparse_attn_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["o_sp" + tag],
+                                bufs["lse_sp" + tag], ws=blk.ws, stream=stream)
+            if blk.swa_window > 0:
+                swa_gated(vl, blk.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, bufs["o_sp" + tag],
+                          bufs["o_l" + tag], ws=blk.ws, stream=stream)
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        step_instrumented(i)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    hs.check_error(blk.ws)
+    ms_total = t0.elapsed_time(t1)
+    full_ms = statistics.mean(a.elapsed_time(b) for a, b in full_ev)
+    vals = torch.tensor([ms_total, full_ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    ms_total, full_ms = vals.tolist()
+    ms_step = ms_total / args.steps
+    tokens = w.total_q
+    value = world * tokens / (ms_step / 1e3)
+
+    # ---- e2e through the public API with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_e2e(args, w, inp, vl, blk, layers, device, world)
+
+    hbm, tf_burst, tf_sust, src = peaks()
+    flops = full_flops(w)
+    achieved = flops / (full_ms / 1e3) / 1e12
+    roof = {"bound": "tensor", "kernel": "attn_fwd_kernel<128,full,64>", "achieved": round(achieved, 1),
+            "peak": tf_burst, "unit": "TFLOP/s", "frac": round(achieved / tf_burst, 4),
+            "traffic": traffic_for("attn_fwd_full", args.workload),
+            "peak_kind": f"{src} bf16 burst", "algorithmic_flop_per_launch": flops,
+            "ms_per_launch": round(full_ms, 4)}
+    out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (seeded N(0,1) bf16, 1% planted keys)",
+           "config": {"workload": f"{w.name}: HySparse block-level prefill, 1x{w.total_q} tokens, "
+                                  f"{w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim}, B={w.block}, "
+                                  f"k={w.topk}, SWA {w.swa_window}+gate, 1 full + {w.n_sparse} sparse",
+                      "tokens_per_step_per_gpu": tokens, "l2": "inputs larger than L2 (~2 GB/step)",
+                      "parallelism": f"independent blocks x{world}"},
+           "roofline": roof, "gpu_launches": blk.launches_per_forward(len(layers)) * args.steps,
+           "clocks": clk, "e2e": e2e}
+    return out
+
+
+def bench_e2e(args, w, inp, vl, blk, layers, device, world):
+    """Same metric through HybridBlock.forward with the step's inputs copied
+    from pinned host memory each step and the last layer's output read back."""
+    from hybrid_sparse_attention_tma_b200.block import SparseLayerIn
+    host = {"q": inp.q.cpu().pin_memory(), "k": inp.k.cpu().pin_memory(), "v": inp.v.cpu().pin_memory()}
+    hl = []
+    for L in inp.layers:
+        d = {"q": L.q.cpu().pin_memory()}
+        if L.k_swa is not None:
+            d.update(k_swa=L.k_swa.cpu().pin_memory(), v_swa=L.v_swa.cpu().pin_memory(),
+                     gamma=L.gamma.cpu().pin_memory())
+        hl.append(d)
+    dev_q, dev_k, dev_v = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
+    dev_layers = [SparseLayerIn(torch.empty_like(L.q),
+                                torch.empty_like(L.k_swa) if L.k_swa is not None else None,
+                                torch.empty_like(L.v_swa) if L.v_swa is not None else None,
+                                torch.empty_like(L.gamma) if L.gamma is not None else None) for L in inp.layers]
+    out_host = torch.empty(inp.q.shape, dtype=torch.bfloat16).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d += sum(t.numel() * t.element_size() for d in hl for t in d.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def step():
+        dev_q.copy_(host["q"], non_blocking=True)
+        dev_k.copy_(host["k"], non_blocking=True)
+        dev_v.copy_(host["v"], non_blocking=True)
+        for dl, d in zip(dev_layers, hl):
+            dl.q.copy_(d["q"], non_blocking=True)
+            if dl.k_swa is not None:
+                dl.k_swa.copy_(d["k_swa"], non_blocking=True)
+                dl.v_swa.copy_(d["v_swa"], non_blocking=True)
+                dl.gamma.copy_(d["gamma"], non_blocking=True)
+        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream)
+        out_host.copy_(res["layers"][-1]["o"], non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, args.steps // 4)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = t.item()
+    return {"value": round(world * w.total_q / (ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
+
+
+# ---------------------------------------------------------------- oracle side
+
+def oracle_sample(w, tile_id, inp_cpu):
+    """Run the oracle's whole block on one selection tile; returns tokens."""
+    import numpy as np
+    import oracle as O
+    from oracle.block import run_block
+    q = O.bf16_to_f64(W.bf16_bits(inp_cpu.q))
+    k = O.bf16_to_f64(W.bf16_bits(inp_cpu.k))
+    v = O.bf16_to_f64(W.bf16_bits(inp_cpu.v))
+    layers = []
+    for L in inp_cpu.layers:
+        d = {"q": O.bf16_to_f64(W.bf16_bits(L.q))}
+        if L.k_swa is not None:
+            d.update(k_swa=O.bf16_to_f64(W.bf16_bits(L.k_swa)), v_swa=O.bf16_to_f64(W.bf16_bits(L.v_swa)),
+                     gamma=L.gamma.double().numpy())
+        layers.append(d)
+    return q, k, v, layers
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(w, n_tiles_sample=1, repeats=1):
+    """Time the oracle's block on `n_tiles_sample` middle tiles; tokens/s."""
+    import oracle as O
+    from oracle.block import run_block
+    inp = W.make_block_inputs(w, device="cpu")
+    q, k, v, layers = oracle_sample(w, 0, inp)
+    n_t = w.n_tiles()
+    mids = [n_t // 2 + i for i in range(n_tiles_sample)]
+    tiles = O.make_tiles(w.cu_q(), w.cu_kv(), w.q_tile)
+    toks = sum(tiles[i].n for i in mids)
+    times = []
+    for _ in range(repeats):
+        t = time.perf_counter()
+        run_block(q, k, v, layers, w.cu_q(), w.cu_kv(), w.n_kv_heads, w.q_tile, w.block, w.topk, w.window,
+                  w.swa_window, tile_ids=mids)
+        times.append(time.perf_counter() - t)
+    return toks, times
+
+
+def bench_reference(args, world, rank):
+    if rank != 0:
+        return None
+    w = W.WORKLOADS[args.workload]
+    import oracle as O  # noqa: F401
+    toks, times = time_oracle(w, 1, repeats=args.warmup + args.steps)
+    timed = times[args.warmup:]
+    s = sum(timed) / len(timed)
+    value = toks / s
+    cores = oracle_threads()
+    sample = f"selection tile {w.n_tiles() // 2} ({toks} queries, all layers of the block) per step"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16, 1% planted keys)",
+            "config": {"workload": w.name, "tokens_per_step": toks},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        out = bench_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out))
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    out = bench_ours(args, world, rank, local)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        w = W.WORKLOADS[args.workload]
+        toks, times = time_oracle(w, 1, repeats=1)
+        out["cpu_baseline"] = {"value": round(toks / sum(times), 3), "unit": "tokens/s", "cores": oracle_threads(),
+                               "kind": "oracle",
+                               "sample": f"1 middle selection tile ({toks} queries), whole block, {sum(times):.1f} s"}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

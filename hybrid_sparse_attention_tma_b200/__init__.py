@@ -1,0 +1,189 @@
+"""libhs: hybrid-block sparse attention (HySparse / HySparse2) on B200.
+
+Thin Python binding over the C ABI in include/hs.h. Every step of the path runs
+in libhs's CUDA kernels; this module only allocates outputs/workspaces with
+torch, builds the argument structs and checks status codes. There is no
+fallback: if libhs.so is missing the import of the library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import List, Optional, Sequence
+
+import torch
+
+from . import _lib as L
+from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
+
+__all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
+           "sparse_attn_decode", "swa_gated", "workspace_size", "check_error", "HsError"]
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class Varlen:
+    """Packed variable-length batch: prefix sums of new queries and of keys."""
+
+    def __init__(self, cu_q: Sequence[int], cu_kv: Sequence[int], n_q_heads: int, n_kv_heads: int,
+                 head_dim: int, device="cuda", softmax_scale: float = 0.0):
+        self.cu_q_list: List[int] = [int(x) for x in cu_q]
+        self.cu_kv_list: List[int] = [int(x) for x in cu_kv]
+        self.batch = len(self.cu_q_list) - 1
+        self.n_q_heads, self.n_kv_heads, self.head_dim = n_q_heads, n_kv_heads, head_dim
+        self.cu_q = torch.tensor(self.cu_q_list, dtype=torch.int32, device=device)
+        self.cu_kv = torch.tensor(self.cu_kv_list, dtype=torch.int32, device=device)
+        self._hq = (ctypes.c_int32 * len(self.cu_q_list))(*self.cu_q_list)
+        self._hkv = (ctypes.c_int32 * len(self.cu_kv_list))(*self.cu_kv_list)
+        self.c = L.HsVarlen(self.batch, n_q_heads, n_kv_heads, head_dim,
+                            self.cu_q.data_ptr(), self.cu_kv.data_ptr(), self._hq, self._hkv,
+                            float(softmax_scale))
+
+    @property
+    def total_q(self) -> int:
+        return self.cu_q_list[-1]
+
+    @property
+    def total_kv(self) -> int:
+        return self.cu_kv_list[-1]
+
+    @property
+    def max_kv(self) -> int:
+        return max(b - a for a, b in zip(self.cu_kv_list, self.cu_kv_list[1:]))
+
+    def n_tiles(self, T: int) -> int:
+        return sum((b - a + T - 1) // T for a, b in zip(self.cu_q_list, self.cu_q_list[1:]))
+
+
+def Sel(q_tile: int, block: int, topk: int, window: int) -> L.HsSel:
+    return L.HsSel(q_tile, block, topk, window)
+
+
+def workspace_size(op: int, vl: Varlen, sel: Optional[L.HsSel] = None) -> int:
+    lib = L.load()
+    n = lib.hs_workspace_size(op, ctypes.byref(vl.c), ctypes.byref(sel) if sel is not None else None)
+    if n == 0:
+        raise HsError("hs_workspace_size", L.HS_ERR_INVALID_ARG, "invalid shapes")
+    return n
+
+
+class Workspace:
+    """Caller-owned device scratch; grows on demand; header zeroed once."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int, stream=None) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+            L.check("hs_workspace_init", L.load().hs_workspace_init(_ptr(self.buf), self.buf.numel(), _stream(stream)))
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws: Optional[Workspace], device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def check_error(ws: Workspace, stream=None):
+    """Synchronise and raise if a device-side bounded wait gave up."""
+    L.check("hs_check_error", L.load().hs_check_error(_ptr(ws.buf), _stream(stream)))
+
+
+def full_attn_select(vl: Varlen, sel: L.HsSel, q, k, v, o=None, lse=None, scores=None,
+                     ws: Optional[Workspace] = None, stream=None):
+    """Full causal attention + importance scores. Returns (o, lse, scores)."""
+    lib = L.load()
+    dev = q.device
+    Tq, Hq, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((Hq, Tq), dtype=torch.float32, device=dev) if lse is None else lse
+    nblk = (vl.max_kv + sel.block - 1) // sel.block
+    if scores is None:
+        scores = torch.empty((vl.n_tiles(sel.q_tile), vl.n_kv_heads, nblk), dtype=torch.float32, device=dev)
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_FULL_ATTN_SELECT, vl, sel), stream)
+    L.check("hs_full_attn_select", lib.hs_full_attn_select(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(scores),
+        _ptr(buf), buf.numel(), _stream(stream)))
+    return o, lse, scores
+
+
+def topk_select(vl: Varlen, sel: L.HsSel, scores, idx=None, cnt=None, ws: Optional[Workspace] = None,
+                stream=None):
+    """Top-k candidate blocks per (tile, KV head). Returns (idx, cnt)."""
+    lib = L.load()
+    dev = scores.device
+    nt = vl.n_tiles(sel.q_tile)
+    idx = torch.empty((nt, vl.n_kv_heads, max(sel.topk, 1)), dtype=torch.int32, device=dev) if idx is None else idx
+    cnt = torch.empty((nt, vl.n_kv_heads), dtype=torch.int32, device=dev) if cnt is None else cnt
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_TOPK_SELECT, vl, sel), stream)
+    L.check("hs_topk_select", lib.hs_topk_select(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(scores), _ptr(idx), _ptr(cnt), _ptr(buf), buf.numel(),
+        _stream(stream)))
+    return idx, cnt
+
+
+def sparse_attn_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, o=None, lse=None,
+                        ws: Optional[Workspace] = None, stream=None, want_lse: bool = True):
+    """Sparse layer over the reused KV cache and indices. Returns (o, lse)."""
+    lib = L.load()
+    dev = q.device
+    Tq, Hq, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty((Hq, Tq), dtype=torch.float32, device=dev)
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_SPARSE_ATTN_PREFILL, vl, sel), stream)
+    L.check("hs_sparse_attn_prefill", lib.hs_sparse_attn_prefill(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), _ptr(o),
+        _ptr(lse), _ptr(buf), buf.numel(), _stream(stream)))
+    return o, lse
+
+
+def sparse_attn_decode(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, k_scale=None, v_scale=None,
+                       kv_dtype: int = HS_KV_BF16, split_k: int = 0, o=None, lse=None,
+                       ws: Optional[Workspace] = None, stream=None):
+    """Sparse decode (one query per sequence), bf16 or FP8-e4m3 KV. Returns (o, lse)."""
+    lib = L.load()
+    dev = q.device
+    Tq, Hq, d = q.shape
+    o = torch.empty((Tq, Hq, d), dtype=torch.bfloat16, device=dev) if o is None else o
+    lse = torch.empty((Hq, Tq), dtype=torch.float32, device=dev) if lse is None else lse
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_SPARSE_ATTN_DECODE, vl, sel), stream)
+    L.check("hs_sparse_attn_decode", lib.hs_sparse_attn_decode(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), kv_dtype, _ptr(k), _ptr(v), _ptr(k_scale),
+        _ptr(v_scale), _ptr(idx), _ptr(cnt), split_k, _ptr(o), _ptr(lse), _ptr(buf), buf.numel(),
+        _stream(stream)))
+    return o, lse
+
+
+def swa_gated(vl: Varlen, window: int, q, k_swa, v_swa, gamma, o_sparse, o=None,
+              ws: Optional[Workspace] = None, stream=None):
+    """Own-cache sliding-window branch fused with the sigmoid gate. Returns o."""
+    lib = L.load()
+    dev = q.device
+    o = torch.empty_like(q) if o is None else o
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_SWA_GATED, vl, None), stream)
+    L.check("hs_swa_gated", lib.hs_swa_gated(
+        ctypes.byref(vl.c), window, _ptr(q), _ptr(k_swa), _ptr(v_swa), _ptr(gamma), _ptr(o_sparse), _ptr(o),
+        _ptr(buf), buf.numel(), _stream(stream)))
+    return o

@@ -1,0 +1,77 @@
+"""One hybrid block: a full attention layer feeding N sparse layers that reuse
+its KV cache and its top-k indices (QbitAI repost of HySparse, "hybrid block";
+HySparse2 release note, "KV Reuse"). HySparse sparse layers also run the
+own-cache sliding-window branch and the sigmoid gate.
+
+Only sequencing of library calls lives here; all arithmetic is in libhs.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import List, Optional
+
+import torch
+
+from . import Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, swa_gated
+
+
+@dataclass
+class SparseLayerIn:
+    q: torch.Tensor                       # [T_q, H_q, d] bf16, this layer's queries
+    k_swa: Optional[torch.Tensor] = None  # [T_kv, H_kv, d] bf16, own SWA cache (HySparse)
+    v_swa: Optional[torch.Tensor] = None
+    gamma: Optional[torch.Tensor] = None  # [T_q, H_q] fp32 gate logits
+
+
+class HybridBlock:
+    def __init__(self, vl: Varlen, q_tile: int, block: int, topk: int, window: int, swa_window: int = 0,
+                 device="cuda"):
+        self.vl = vl
+        self.sel = Sel(q_tile, block, topk, window)
+        self.swa_window = swa_window
+        self.ws = Workspace(device)
+        self.device = device
+        self._bufs = {}
+
+    def _buf(self, name, shape, dtype):
+        t = self._bufs.get(name)
+        if t is None or t.shape != torch.Size(shape) or t.dtype != dtype:
+            t = torch.empty(shape, dtype=dtype, device=self.device)
+            self._bufs[name] = t
+        return t
+
+    def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False):
+        """Returns dict(o_full, lse_full, scores, idx, cnt, layers=[{o_sparse, lse_sparse, o}]).
+
+        With keep_all=False, output buffers are reused across calls (no
+        allocation in steady state) and only the last layer's tensors are
+        guaranteed distinct."""
+        vl, sel = self.vl, self.sel
+        Tq, Hq, d = q.shape
+        nblk = (vl.max_kv + sel.block - 1) // sel.block
+        nt = vl.n_tiles(sel.q_tile)
+        o = self._buf("o_full", (Tq, Hq, d), torch.bfloat16)
+        lse = self._buf("lse_full", (Hq, Tq), torch.float32)
+        scores = self._buf("scores", (nt, vl.n_kv_heads, nblk), torch.float32)
+        idx = self._buf("idx", (nt, vl.n_kv_heads, max(sel.topk, 1)), torch.int32)
+        cnt = self._buf("cnt", (nt, vl.n_kv_heads), torch.int32)
+        full_attn_select(vl, sel, q, k, v, o, lse, scores, ws=self.ws, stream=stream)
+        topk_select(vl, sel, scores, idx, cnt, ws=self.ws, stream=stream)
+        outs = []
+        for i, L in enumerate(layers):
+            tag = str(i) if keep_all else str(i % 2)
+            o_sp = self._buf("o_sp" + tag, (Tq, Hq, d), torch.bfloat16)
+            lse_sp = self._buf("lse_sp" + tag, (Hq, Tq), torch.float32)
+            sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream)
+            if self.swa_window > 0:
+                o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
+                swa_gated(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, ws=self.ws,
+                          stream=stream)
+            else:
+                o_l = o_sp
+            outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
+        return {"o_full": o, "lse_full": lse, "scores": scores, "idx": idx, "cnt": cnt, "layers": outs}
+
+    def launches_per_forward(self, n_layers: int) -> int:
+        """Kernels of this library launched by one forward (memsets excluded)."""
+        return 2 + n_layers * (2 if self.swa_window > 0 else 1)

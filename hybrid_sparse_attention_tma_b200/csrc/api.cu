@@ -1,0 +1,484 @@
+// api.cu -- the libhs C ABI: argument validation, workspace sizing, tensor
+// maps, schedules and kernel launches. No call allocates device memory.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <numeric>
+#include <vector>
+
+#include "../../include/hs.h"
+#include "attn_fwd.cuh"
+#include "hs_common.cuh"
+#include "seqtable.cuh"
+#include "topk.cuh"
+
+using namespace hs;
+
+namespace {
+
+constexpr size_t kHeaderBytes = 256;
+constexpr unsigned long long kDefaultTimeoutNs = 4000000000ull;  // 4 s
+unsigned long long g_timeout_ns = kDefaultTimeoutNs;
+
+inline cudaStream_t S(hs_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor [outer][mid][d] viewed as dims {d, mid, outer}; box {64, box_mid, box_outer};
+// 128-byte swizzle; out-of-range rows read as zero.
+bool make_map_3d(CUtensorMap* m, const void* base, int d, int mid, long long outer, int box_mid, int box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(mid), cuuint64_t(outer)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * 2, cuuint64_t(d) * 2 * cuuint64_t(mid)};
+  cuuint32_t box[3] = {64, cuuint32_t(box_mid), cuuint32_t(box_outer)};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------- validation ----------------
+struct Shape {
+  int batch, Hq, Hkv, G, d;
+  long long Tq, Tkv;
+  int max_q, max_kv;
+  float scale;
+};
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+hs_status check_varlen(const hs_varlen* vl, Shape* sh, bool need_device_cu = true) {
+  if (!vl) return HS_ERR_INVALID_ARG;
+  if (vl->batch < 1 || vl->n_q_heads < 1 || vl->n_kv_heads < 1) return HS_ERR_INVALID_ARG;
+  if (vl->n_q_heads % vl->n_kv_heads) return HS_ERR_INVALID_ARG;
+  if (!vl->cu_q_host || !vl->cu_kv_host) return HS_ERR_INVALID_ARG;
+  if (need_device_cu && (!vl->cu_q || !vl->cu_kv)) return HS_ERR_INVALID_ARG;
+  if (vl->cu_q_host[0] != 0 || vl->cu_kv_host[0] != 0) return HS_ERR_INVALID_ARG;
+  sh->batch = vl->batch;
+  sh->Hq = vl->n_q_heads;
+  sh->Hkv = vl->n_kv_heads;
+  sh->G = sh->Hq / sh->Hkv;
+  sh->d = vl->head_dim;
+  sh->max_q = 0;
+  sh->max_kv = 0;
+  for (int b = 0; b < vl->batch; ++b) {
+    const int nq = vl->cu_q_host[b + 1] - vl->cu_q_host[b];
+    const int nkv = vl->cu_kv_host[b + 1] - vl->cu_kv_host[b];
+    if (nq < 0 || nkv < nq) return HS_ERR_INVALID_ARG;
+    sh->max_q = std::max(sh->max_q, nq);
+    sh->max_kv = std::max(sh->max_kv, nkv);
+  }
+  sh->Tq = vl->cu_q_host[vl->batch];
+  sh->Tkv = vl->cu_kv_host[vl->batch];
+  if (sh->Tkv > (1LL << 31) - 1 || sh->Tq > (1LL << 31) - 1) return HS_ERR_UNSUPPORTED;
+  if (!(vl->softmax_scale >= 0.f) || std::isinf(vl->softmax_scale)) return HS_ERR_INVALID_ARG;
+  sh->scale = vl->softmax_scale > 0.f ? vl->softmax_scale : 1.f / std::sqrt(float(sh->d));
+  if (sh->d != 64 && sh->d != 128) return HS_ERR_UNSUPPORTED;
+  return HS_OK;
+}
+
+hs_status check_sel(const hs_sel* sel) {
+  if (!sel) return HS_ERR_INVALID_ARG;
+  if (sel->q_tile < 1 || sel->block < 1 || sel->topk < 0 || sel->window < 0) return HS_ERR_INVALID_ARG;
+  if (sel->topk > 4096) return HS_ERR_UNSUPPORTED;
+  if (!is_pow2(sel->block) || sel->block > 128 || (sel->block > 1 && sel->block < 8)) return HS_ERR_UNSUPPORTED;
+  return HS_OK;
+}
+
+int n_tiles_of(const hs_varlen* vl, int T) {
+  long long n = 0;
+  for (int b = 0; b < vl->batch; ++b) n += (vl->cu_q_host[b + 1] - vl->cu_q_host[b] + T - 1) / T;
+  return int(n);
+}
+
+bool fill_seqtable(const hs_varlen* vl, int T, SeqTable* st) {
+  if (vl->batch > kMaxSeq) return false;
+  st->batch = vl->batch;
+  st->T = T;
+  st->tile_base[0] = 0;
+  for (int b = 0; b <= vl->batch; ++b) {
+    st->cu_q[b] = vl->cu_q_host[b];
+    st->cu_kv[b] = vl->cu_kv_host[b];
+  }
+  for (int b = 0; b < vl->batch; ++b)
+    st->tile_base[b + 1] = st->tile_base[b] + (vl->cu_q_host[b + 1] - vl->cu_q_host[b] + T - 1) / T;
+  st->n_tiles = st->tile_base[vl->batch];
+  return true;
+}
+
+// Schedule of the tcgen05 attention kernel (see attn::Sched).
+bool fill_sched(const hs_varlen* vl, const Shape& sh, int mode, int T, int chunks_per_tile, attn::Sched* sc) {
+  if (vl->batch > attn::kMaxSched) return false;
+  const int B = vl->batch;
+  std::vector<int> order(B);
+  std::iota(order.begin(), order.end(), 0);
+  if (mode == attn::kFull) {
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+      return (vl->cu_kv_host[a + 1] - vl->cu_kv_host[a]) > (vl->cu_kv_host[b + 1] - vl->cu_kv_host[b]);
+    });
+  }
+  const int qpc = attn::kMaxItemRows / sh.G;
+  sc->n_seq = B;
+  sc->first_item[0] = 0;
+  int tb = 0;
+  for (int b = 0; b < B; ++b) {
+    sc->cu_q[b] = vl->cu_q_host[b];
+    sc->cu_kv[b] = vl->cu_kv_host[b];
+    sc->tile_base[b] = tb;
+    tb += (vl->cu_q_host[b + 1] - vl->cu_q_host[b] + T - 1) / T;
+  }
+  sc->cu_q[B] = vl->cu_q_host[B];
+  sc->cu_kv[B] = vl->cu_kv_host[B];
+  long long acc = 0;
+  for (int e = 0; e < B; ++e) {
+    const int b = order[e];
+    sc->seq[e] = b;
+    const int n_b = vl->cu_q_host[b + 1] - vl->cu_q_host[b];
+    long long items;
+    if (mode == attn::kFull)
+      items = (long long)((n_b + qpc - 1) / qpc) * sh.Hkv;
+    else
+      items = (long long)((n_b + T - 1) / T) * chunks_per_tile * sh.Hkv;
+    acc += items;
+    if (acc > (1LL << 30)) return false;
+    sc->first_item[e + 1] = int(acc);
+  }
+  sc->n_items = int(acc);
+  return true;
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+struct Maps {
+  CUtensorMap q, k, v, kb, vb;
+};
+
+// Launch the tcgen05 attention kernel.
+template <int D, int MODE, int SB>
+hs_status launch_attn(const Maps& m, const attn::Params& p, const attn::Sched& sc, int grid, cudaStream_t st) {
+  auto kern = attn::attn_fwd_kernel<D, MODE, SB>;
+  constexpr int smem = attn::smem_bytes<D>() > 116 * 1024 ? attn::smem_bytes<D>() : 116 * 1024;
+  static bool configured = false;
+  if (!configured) {
+    if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
+    configured = true;
+  }
+  kern<<<grid, attn::kThreads, smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, p, sc);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+template <int MODE, int SB>
+hs_status dispatch_attn_d(int d, const Maps& m, const attn::Params& p, const attn::Sched& sc, int grid,
+                          cudaStream_t st) {
+  if (d == 64) return launch_attn<64, MODE, SB>(m, p, sc, grid, st);
+  return launch_attn<128, MODE, SB>(m, p, sc, grid, st);
+}
+
+hs_status dispatch_full(int d, int B, const Maps& m, const attn::Params& p, const attn::Sched& sc, int grid,
+                        cudaStream_t st) {
+  switch (B) {
+    case 8: return dispatch_attn_d<attn::kFull, 8>(d, m, p, sc, grid, st);
+    case 16: return dispatch_attn_d<attn::kFull, 16>(d, m, p, sc, grid, st);
+    case 32: return dispatch_attn_d<attn::kFull, 32>(d, m, p, sc, grid, st);
+    case 64: return dispatch_attn_d<attn::kFull, 64>(d, m, p, sc, grid, st);
+    case 128: return dispatch_attn_d<attn::kFull, 128>(d, m, p, sc, grid, st);
+    default: return dispatch_attn_d<attn::kFull, 0>(d, m, p, sc, grid, st);
+  }
+}
+
+WaitCtl wait_ctl(void* ws) { return WaitCtl{reinterpret_cast<ErrWord*>(ws), g_timeout_ns}; }
+
+size_t full_ws_bytes(const Shape& sh, const hs_sel* sel) {
+  size_t b = kHeaderBytes;
+  if (sel->block > 1) {
+    const size_t nblk = (size_t(sh.max_kv) + sel->block - 1) / sel->block;
+    b += size_t(num_sms()) * nblk * attn::kMaxItemRows * sizeof(float);
+  }
+  return align_up(b, 256);
+}
+
+// Waits on an mbarrier that nothing ever arrives at; the bounded wait gives up
+// after wc.timeout_ns, records the failure in the error word and returns.
+__global__ void debug_wait_kernel(WaitCtl wc) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, wc, 99);
+}
+
+}  // namespace
+
+// ============================================================================
+extern "C" {
+
+const char* hs_status_string(hs_status s) {
+  switch (s) {
+    case HS_OK: return "ok";
+    case HS_ERR_INVALID_ARG: return "invalid argument";
+    case HS_ERR_UNSUPPORTED: return "unsupported configuration";
+    case HS_ERR_WORKSPACE: return "workspace missing or too small";
+    case HS_ERR_CUDA: return "CUDA error";
+    case HS_ERR_TIMEOUT: return "device-side bounded wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t hs_workspace_size(int op, const hs_varlen* vl, const hs_sel* sel) {
+  Shape sh;
+  if (check_varlen(vl, &sh, false) != HS_OK) return 0;
+  switch (op) {
+    case HS_OP_FULL_ATTN_SELECT:
+      if (!sel || check_sel(sel) != HS_OK) return 0;
+      return full_ws_bytes(sh, sel);
+    case HS_OP_TOPK_SELECT:
+    case HS_OP_SPARSE_ATTN_PREFILL:
+    case HS_OP_SWA_GATED:
+      return kHeaderBytes;
+    case HS_OP_SPARSE_ATTN_DECODE:
+      return kHeaderBytes;
+    default:
+      return 0;
+  }
+}
+
+hs_status hs_workspace_init(void* ws, size_t ws_bytes, hs_stream_t stream) {
+  if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
+  return cudaMemsetAsync(ws, 0, kHeaderBytes, S(stream)) == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_check_error(void* ws, hs_stream_t stream) {
+  if (!ws) return HS_ERR_WORKSPACE;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return HS_ERR_CUDA;
+  ErrWord e{};
+  if (cudaMemcpy(&e, ws, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return HS_ERR_CUDA;
+  if (e.flag != 0) {
+    if (cudaMemset(ws, 0, sizeof(ErrWord)) != cudaSuccess) return HS_ERR_CUDA;
+    return HS_ERR_TIMEOUT;
+  }
+  return HS_OK;
+}
+
+hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                              const void* v, void* o, float* lse, float* scores, void* ws, size_t ws_bytes,
+                              hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (!q || !k || !v || !o || !scores) return HS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < full_ws_bytes(sh, sel)) return HS_ERR_WORKSPACE;
+  if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
+  if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
+  if (sel->block == 1) return HS_ERR_UNSUPPORTED;  // token-level scores: second QK pass (not built yet)
+  if (sh.Tq == 0) return HS_OK;
+  const int T = sel->q_tile, B = sel->block;
+  const int n_tiles = n_tiles_of(vl, T);
+  const int nblk = (sh.max_kv + B - 1) / B;
+  cudaStream_t s = S(stream);
+  if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
+    return HS_ERR_CUDA;
+
+  Maps m;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
+      !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128))
+    return HS_ERR_CUDA;
+  m.kb = m.k;
+  m.vb = m.v;
+  static attn::Sched sc;  // large; filled per call under the host lock below
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!fill_sched(vl, sh, attn::kFull, T, 1, &sc)) return HS_ERR_UNSUPPORTED;
+  attn::Params p{};
+  p.G = sh.G;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.Tq = int(sh.Tq);
+  p.scale_log2 = sh.scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scores = scores;
+  p.spill = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kHeaderBytes);
+  p.nblk = nblk;
+  p.T = T;
+  p.B = B;
+  p.chunks_per_tile = 1;
+  p.wc = wait_ctl(ws);
+  const int grid = std::min(num_sms(), std::max(1, sc.n_items));
+  return dispatch_full(sh.d, B, m, p, sc, grid, s);
+}
+
+hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* scores, int32_t* idx, int32_t* cnt,
+                         void* ws, size_t ws_bytes, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh, false);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (!scores || !idx || !cnt) return HS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
+  if (vl->batch > kMaxSeq) return HS_ERR_UNSUPPORTED;
+  if (sh.Tq == 0) return HS_OK;
+  SeqTable table;
+  fill_seqtable(vl, sel->q_tile, &table);
+  topk::Params p{};
+  p.scores = scores;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.Hkv = sh.Hkv;
+  p.nblk = (sh.max_kv + sel->block - 1) / sel->block;
+  p.B = sel->block;
+  p.k = sel->topk;
+  const long long rows = (long long)table.n_tiles * sh.Hkv;
+  if (rows > (1LL << 31) - 1) return HS_ERR_UNSUPPORTED;
+  topk::topk_kernel<<<unsigned(rows), topk::kThreads, 0, S(stream)>>>(p, table);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                                 void* ws, size_t ws_bytes, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (!q || !k || !v || !o || (sel->topk > 0 && (!idx || !cnt))) return HS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
+  if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
+  if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
+  if (sel->block == 1 && sel->topk > 0) return HS_ERR_UNSUPPORTED;  // token gather: not built yet
+  if (sh.Tq == 0) return HS_OK;
+  const int T = sel->q_tile, B = sel->block;
+  Maps m;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
+      !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
+      !make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B))
+    return HS_ERR_CUDA;
+  static attn::Sched sc;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  const int cpt = (T * sh.G + attn::kMaxItemRows - 1) / attn::kMaxItemRows;
+  if (!fill_sched(vl, sh, attn::kSparse, T, cpt, &sc)) return HS_ERR_UNSUPPORTED;
+  attn::Params p{};
+  p.G = sh.G;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.Tq = int(sh.Tq);
+  p.scale_log2 = sh.scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.T = T;
+  p.B = B;
+  p.chunks_per_tile = cpt;
+  p.idx = idx;
+  p.cnt = cnt;
+  p.topk = sel->topk;
+  p.w = sel->window;
+  p.wc = wait_ctl(ws);
+  const int grid = std::min(num_sms(), std::max(1, sc.n_items));
+  switch (B) {
+    case 8: return dispatch_attn_d<attn::kSparse, 8>(sh.d, m, p, sc, grid, S(stream));
+    case 16: return dispatch_attn_d<attn::kSparse, 16>(sh.d, m, p, sc, grid, S(stream));
+    case 32: return dispatch_attn_d<attn::kSparse, 32>(sh.d, m, p, sc, grid, S(stream));
+    case 64: return dispatch_attn_d<attn::kSparse, 64>(sh.d, m, p, sc, grid, S(stream));
+    case 128: return dispatch_attn_d<attn::kSparse, 128>(sh.d, m, p, sc, grid, S(stream));
+    default: return HS_ERR_UNSUPPORTED;
+  }
+}
+
+hs_status hs_sparse_attn_decode(const hs_varlen*, const hs_sel*, const void*, hs_kv_dtype, const void*, const void*,
+                                const float*, const float*, const int32_t*, const int32_t*, int32_t, void*, float*,
+                                void*, size_t, hs_stream_t) {
+  return HS_ERR_UNSUPPORTED;
+}
+
+hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const void* k_swa, const void* v_swa,
+                       const float* gamma, const void* o_sparse, void* o, void* ws, size_t ws_bytes,
+                       hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if (window < 1) return HS_ERR_INVALID_ARG;
+  if (!q || !k_swa || !v_swa || !gamma || !o_sparse || !o) return HS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_swa) || !aligned16(v_swa) || !aligned16(o) || !aligned16(o_sparse))
+    return HS_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
+  if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
+  if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
+  if (sh.Tq == 0) return HS_OK;
+  Maps m;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
+      !make_map_3d(&m.k, k_swa, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
+      !make_map_3d(&m.v, v_swa, sh.d, sh.Hkv, sh.Tkv, 1, 128))
+    return HS_ERR_CUDA;
+  m.kb = m.k;
+  m.vb = m.v;
+  static attn::Sched sc;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  const int T = attn::kMaxItemRows / sh.G;  // one 256-row chunk per schedule tile
+  if (!fill_sched(vl, sh, attn::kSparse, T, 1, &sc)) return HS_ERR_UNSUPPORTED;
+  attn::Params p{};
+  p.G = sh.G;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.Tq = int(sh.Tq);
+  p.scale_log2 = sh.scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = nullptr;
+  p.T = T;
+  p.B = 1;
+  p.chunks_per_tile = 1;
+  p.idx = nullptr;
+  p.cnt = nullptr;
+  p.topk = 0;
+  p.w = window;
+  p.gamma = gamma;
+  p.o_other = reinterpret_cast<const __nv_bfloat16*>(o_sparse);
+  p.wc = wait_ctl(ws);
+  const int grid = std::min(num_sms(), std::max(1, sc.n_items));
+  return dispatch_attn_d<attn::kSparse, 0>(sh.d, m, p, sc, grid, S(stream));
+}
+
+hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, hs_stream_t stream) {
+  if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
+  if (timeout_ns == 0 || timeout_ns > 2000000000ull) return HS_ERR_INVALID_ARG;
+  WaitCtl wc{reinterpret_cast<ErrWord*>(ws), timeout_ns};
+  debug_wait_kernel<<<1, 32, 0, S(stream)>>>(wc);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,621 @@
+// attn_fwd.cuh -- tcgen05 attention forward shared by the full layer (causal
+// attention + block-score by-product) and the sparse layers (attention over
+// the reused KV cache at the selected blocks plus the forced recent window).
+//
+// Full layer: "standard scaled dot-product attention" whose FlashAttention
+// kernel is lightly modified to emit block-level maximum scores from the
+// online-softmax row maximum (HySparse explainer, techwalker.com, paragraphs
+// on the master layer and on the implementation). Sparse layer: attention over
+// the selected KV blocks of the shared cache (QbitAI repost, block-sparse
+// branch) with the most recent tokens forced into the set (HySparse2 release
+// note, airebao.com).
+//
+// CTA organisation (one CTA per SM, persistent over a host-ordered schedule):
+//   warps 0-3  softmax warpgroup for Q-tile 0 (128 rows = TMEM lanes)
+//   warps 4-7  softmax warpgroup for Q-tile 1
+//   warp  8    TMA producer (Q tiles, K/V tiles or gathered blocks)
+//   warp  9    UMMA issuer (one thread) + TMEM owner
+// A work item is up to 256 "rows" of one sequence and one KV head g; row
+// r = query * G + head-in-group, so every Q-tile holds whole queries and the
+// group's heads share each K/V tile (GQA/MQA packing into the MMA M dim).
+// TMEM (512 columns): S_t at t*256, O_t at t*256+128 (fp32, 128 lanes).
+// SMEM: Q[2] | K/V ring[3] | P[2] | control. All operand tiles use the
+// 128-byte swizzle (8-row x 128-byte atoms), K-major except V (MN-major).
+#pragma once
+
+#include "hs_common.cuh"
+
+namespace hs {
+namespace attn {
+
+constexpr int kThreads = 320;
+constexpr int kStages = 3;
+constexpr int kSlabBytes = 128 * 128;  // 128 rows x 64 bf16
+constexpr int kMaxItemRows = 256;
+
+enum Mode : int { kFull = 0, kSparse = 1 };
+
+// One work item: up to 256 rows (whole queries x the KV head's group) of one
+// sequence and one KV head.
+struct Item {
+  int qrow0;   // packed query row of the item's first query
+  int nq;      // queries in the item (rows = nq * G <= 256); <= 0 means empty
+  int pos0;    // position of the first query in its sequence
+  int kv0;     // packed key row of the sequence's first key
+  int kv_len;  // keys of the sequence
+  int g;       // KV head
+  int tile0;   // global selection tile of the first query
+  int qoff;    // index of the first query inside tile0
+};
+
+// Host-computed schedule, passed by value in the kernel parameters.
+// Items are enumerated sequence by sequence in `seq` order; the full layer
+// lists sequences longest first and each sequence's chunks last-to-first
+// (decreasing causal cost), so the round-robin over persistent CTAs starts
+// with the heaviest work.
+constexpr int kMaxSched = 256;
+struct Sched {
+  int n_seq;
+  int n_items;
+  int seq[kMaxSched];             // processing order -> sequence id
+  int first_item[kMaxSched + 1];  // prefix of item counts in processing order
+  int cu_q[kMaxSched + 1];        // natural order
+  int cu_kv[kMaxSched + 1];
+  int tile_base[kMaxSched];       // first global selection tile of each sequence
+};
+
+struct Params {
+  int G, Hq, Hkv, Tq;
+  float scale_log2;  // softmax scale * log2(e)
+  __nv_bfloat16* o;
+  float* lse;  // [Hq, Tq] natural log, may be null
+  // block-score by-product (full mode with SB = B > 1)
+  float* scores;  // [n_tiles, Hkv, nblk]
+  float* spill;   // [gridDim.x][nblk][256]
+  int nblk;
+  int T, B;
+  int chunks_per_tile;  // sparse mode: ceil(T*G / 256)
+  // sparse mode
+  const int* idx;  // [n_tiles, Hkv, topk]
+  const int* cnt;  // [n_tiles, Hkv]
+  int topk;
+  int w;
+  // gate epilogue (sliding-window branch): o = sig(gamma) * o_other + (1 - sig(gamma)) * o_this
+  const float* gamma;                // [Tq, Hq] or null
+  const __nv_bfloat16* o_other;      // [Tq, Hq, D] sparse-branch output
+  WaitCtl wc;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kSlabs = D / 64;
+  static constexpr int kTileBytes = kSlabs * kSlabBytes;  // Q tile / K tile / V tile
+  static constexpr int kPBytes = 2 * kSlabBytes;          // 128 rows x 128 keys bf16
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffP = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffCtl = kOffP + 2 * kPBytes;
+};
+
+struct Ctl {
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_ready[2], o_free[2];
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort;
+  float lse2[kMaxItemRows];
+};
+
+template <int D>
+constexpr int smem_bytes() {
+  // + 1024 for manual 1024-byte alignment of the dynamic smem base
+  return Layout<D>::kOffCtl + int(sizeof(Ctl)) + 1024;
+}
+
+
+template <int MODE>
+__device__ __forceinline__ Item get_item(const Params& p, const Sched& sc, int w) {
+  int lo = 0, hi = sc.n_seq - 1;  // entry e with first_item[e] <= w < first_item[e+1]
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (sc.first_item[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  const int b = sc.seq[lo];
+  const int local = w - sc.first_item[lo];
+  const int n_b = sc.cu_q[b + 1] - sc.cu_q[b];
+  const int kv_b = sc.cu_kv[b + 1] - sc.cu_kv[b];
+  const int c_b = kv_b - n_b;
+  const int qpc = kMaxItemRows / p.G;  // queries per 256-row chunk
+  Item it;
+  it.g = local % p.Hkv;
+  int qloc0, nq;
+  if (MODE == kFull) {
+    const int n_chunks = (n_b + qpc - 1) / qpc;
+    const int chunk = n_chunks - 1 - local / p.Hkv;
+    qloc0 = chunk * qpc;
+    nq = min(qpc, n_b - qloc0);
+  } else {
+    const int per_tile = p.chunks_per_tile * p.Hkv;
+    const int ti = local / per_tile;
+    const int chunk = (local / p.Hkv) % p.chunks_per_tile;
+    const int tile_nq = min(p.T, n_b - ti * p.T);
+    qloc0 = ti * p.T + chunk * qpc;
+    nq = min(qpc, tile_nq - chunk * qpc);
+  }
+  it.qrow0 = sc.cu_q[b] + qloc0;
+  it.nq = nq;
+  it.pos0 = c_b + qloc0;
+  it.kv0 = sc.cu_kv[b];
+  it.kv_len = kv_b;
+  it.tile0 = sc.tile_base[b] + qloc0 / p.T;
+  it.qoff = qloc0 % p.T;
+  return it;
+}
+
+// Number of 128-key tiles an item iterates over, and the sparse-mode split.
+struct KvPlan {
+  int n_sel;  // tiles of selected keys (sparse) or causal tiles (full)
+  int n_win;  // window tiles (sparse, w > 0)
+  int win_lo; // first window key (position)
+  int cnt;    // selected blocks
+};
+
+__device__ __forceinline__ KvPlan kv_plan(const Params& p, const Item& it, int mode) {
+  KvPlan k{};
+  const int last_pos = it.pos0 + it.nq - 1;
+  if (mode == kFull) {
+    k.n_sel = last_pos / 128 + 1;
+    k.n_win = 0;
+  } else {
+    const int c = p.cnt ? __ldg(p.cnt + it.tile0 * p.Hkv + it.g) : 0;
+    k.cnt = c;
+    k.n_sel = (c * p.B + 127) / 128;
+    if (p.w > 0) {
+      k.win_lo = max(0, it.pos0 - p.w + 1);
+      k.n_win = (last_pos - k.win_lo + 1 + 127) / 128;
+    }
+  }
+  return k;
+}
+
+// ------------------------------------------------------------------------
+// The kernel
+// ------------------------------------------------------------------------
+template <int D, int MODE, int SB>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kb,
+                    const __grid_constant__ CUtensorMap map_vb, const Params p,
+                    const __grid_constant__ Sched sc) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kOffCtl);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&c.q_full, 1);
+    mbar_init(&c.q_empty, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&c.kv_full[s], 1);
+      mbar_init(&c.kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&c.s_full[t], 1);
+      mbar_init(&c.p_full[t], 4);
+      mbar_init(&c.o_ready[t], 1);
+      mbar_init(&c.o_free[t], 4);
+    }
+    mbar_init(&c.teardown, 1);
+    c.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&c.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    prefetch_tensormap(&map_q);
+    prefetch_tensormap(&map_k);
+    prefetch_tensormap(&map_v);
+    if (MODE == kSparse) {
+      prefetch_tensormap(&map_kb);
+      prefetch_tensormap(&map_vb);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  volatile int* abort_flag = &c.abort;
+
+  if (warp == 8) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      int ctr = 0;        // K/V ring uses
+      int q_uses = 0;     // Q loads issued
+      int last_use[kStages] = {-1, -1, -1};
+      bool ok = true;
+      for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
+        const Item it = get_item<MODE>(p, sc, wi);
+        if (it.nq <= 0) continue;
+        const KvPlan kp = kv_plan(p, it, MODE);
+        const int n = kp.n_sel + kp.n_win;
+        if (n == 0) continue;
+        const int rows = it.nq * p.G;
+        const int n_qt = rows > 128 ? 2 : 1;
+        if (q_uses > 0 && !mbar_wait(&c.q_empty, (q_uses - 1) & 1, abort_flag, p.wc, 1)) { ok = false; break; }
+        mbar_expect_tx(&c.q_full, n_qt * L::kTileBytes);
+        for (int t = 0; t < n_qt; ++t)
+          for (int s = 0; s < L::kSlabs; ++s)
+            tma_load_3d(smem + L::kOffQ + t * L::kTileBytes + s * kSlabBytes, &map_q, &c.q_full, s * 64,
+                        it.g * p.G, it.qrow0 + t * (128 / p.G));
+        ++q_uses;
+        const int* idx_row = (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
+        for (int i = 0; i < n && ok; ++i) {
+          for (int kind = 0; kind < 2; ++kind) {
+            const int s = ctr % kStages;
+            if (!mbar_wait(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, abort_flag, p.wc, 2)) { ok = false; break; }
+            mbar_expect_tx(&c.kv_full[s], L::kTileBytes);
+            uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
+            const CUtensorMap* mt = kind == 0 ? &map_k : &map_v;
+            if (MODE == kFull || i >= kp.n_sel) {
+              const int key0 = (MODE == kFull) ? i * 128 : kp.win_lo + (i - kp.n_sel) * 128;
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                tma_load_3d(dst + sl * kSlabBytes, mt, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
+            } else {
+              const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
+              constexpr int sbk = SB > 0 ? SB : 128;
+              constexpr int nb = 128 / sbk;
+              for (int bi = 0; bi < nb; ++bi) {
+                const int slot = i * nb + bi;
+                const int blk = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
+                for (int sl = 0; sl < L::kSlabs; ++sl)
+                  tma_load_3d(dst + sl * kSlabBytes + bi * sbk * 128, mb, &c.kv_full[s], sl * 64, it.g,
+                              it.kv0 + blk * sbk);
+              }
+            }
+            last_use[s] = ctr;
+            ++ctr;
+          }
+        }
+      }
+      // drain: never leave the CTA with TMA writes in flight
+      if (*abort_flag) {
+        for (int s = 0; s < kStages; ++s)
+          if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kStages) & 1, p.wc, 90);
+        if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 91);
+      }
+    }
+  } else if (warp == 9) {
+    // ===================== UMMA issuer =====================
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
+      int ctr = 0, q_uses = 0;
+      int uses[2] = {0, 0};        // S/P/O phases per Q-tile
+      int items_t[2] = {0, 0};     // items in which tile t took part (o_free phase)
+      bool ok = true;
+      const uint32_t q_base = smem_u32(smem + L::kOffQ);
+      const uint32_t kv_base = smem_u32(smem + L::kOffKV);
+      const uint32_t p_base = smem_u32(smem + L::kOffP);
+      for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
+        const Item it = get_item<MODE>(p, sc, wi);
+        if (it.nq <= 0) continue;
+        const KvPlan kp = kv_plan(p, it, MODE);
+        const int n = kp.n_sel + kp.n_win;
+        if (n == 0) continue;
+        const int n_qt = it.nq * p.G > 128 ? 2 : 1;
+        if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10)) { ok = false; break; }
+        ++q_uses;
+        tc_fence_after();
+        auto issue_qk = [&](int t, int stage) {
+          const uint32_t d_tmem = tmem + t * 256;
+          const uint32_t qa = q_base + t * L::kTileBytes;
+          const uint32_t kb = kv_base + stage * L::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+            umma_bf16(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdQK,
+                      kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&c.s_full[t]);
+        };
+        auto issue_pv = [&](int t, int stage, bool acc) {
+          const uint32_t d_tmem = tmem + t * 256 + 128;
+          const uint32_t pa = p_base + t * L::kPBytes;
+          const uint32_t vb = kv_base + stage * L::kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t aoff = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+            umma_bf16(d_tmem, sdesc_sw128(pa + aoff, 16, 1024), sdesc_sw128(vb + kk * 2048, kSlabBytes, 1024),
+                      kIdPV, (acc || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&c.o_ready[t]);
+        };
+        // prologue: S_t(0)
+        int sk = ctr % kStages;
+        if (!mbar_wait(&c.kv_full[sk], (ctr / kStages) & 1, abort_flag, p.wc, 11)) { ok = false; break; }
+        ++ctr;
+        tc_fence_after();
+        for (int t = 0; t < n_qt; ++t) issue_qk(t, sk);
+        umma_commit(&c.kv_empty[sk]);
+        for (int i = 0; i < n && ok; ++i) {
+          const int sv = ctr % kStages;
+          if (!mbar_wait(&c.kv_full[sv], (ctr / kStages) & 1, abort_flag, p.wc, 12)) { ok = false; break; }
+          ++ctr;
+          int sk_next = -1;
+          for (int t = 0; t < n_qt; ++t) {
+            if (!mbar_wait(&c.p_full[t], (uses[t] + i) & 1, abort_flag, p.wc, 13)) { ok = false; break; }
+            if (i == 0 && items_t[t] > 0 &&
+                !mbar_wait(&c.o_free[t], (items_t[t] - 1) & 1, abort_flag, p.wc, 14)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, sv, i > 0);
+            if (i + 1 < n) {
+              if (sk_next < 0) {
+                sk_next = ctr % kStages;
+                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kStages) & 1, abort_flag, p.wc, 15)) { ok = false; break; }
+                ++ctr;
+                tc_fence_after();
+              }
+              issue_qk(t, sk_next);
+            }
+          }
+          if (!ok) break;
+          umma_commit(&c.kv_empty[sv]);
+          if (sk_next >= 0) umma_commit(&c.kv_empty[sk_next]);
+        }
+        if (!ok) break;
+        umma_commit(&c.q_empty);
+        for (int t = 0; t < n_qt; ++t) {
+          uses[t] += n;
+          items_t[t] += 1;
+        }
+      }
+      // make sure no tensor-core op is still writing TMEM before teardown
+      umma_commit(&c.teardown);
+      mbar_wait_drain(&c.teardown, 0, p.wc, 92);
+    }
+  } else {
+    // ===================== softmax warpgroups =====================
+    const int t = warp >> 2;       // Q-tile
+    const int quad = warp & 3;     // TMEM lane quadrant
+    const int r = quad * 32 + lane;  // row inside the Q-tile
+    const int vr = t * 128 + r;      // row inside the item
+    const uint32_t t_s = tmem + t * 256 + (uint32_t(quad * 32) << 16);
+    const uint32_t t_o = t_s + 128;
+    uint8_t* p_tile = smem + L::kOffP + t * L::kPBytes;
+    int uses = 0, items_t = 0;
+    bool ok = true;
+    for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
+      const Item it = get_item<MODE>(p, sc, wi);
+      if (it.nq <= 0) continue;
+      const KvPlan kp = kv_plan(p, it, MODE);
+      const int n = kp.n_sel + kp.n_win;
+      const int rows = it.nq * p.G;
+      const bool active = (t == 0) || rows > 128;
+      const bool valid = vr < rows;
+      const int ql = vr / p.G;
+      const int h = it.g * p.G + (vr % p.G);
+      const int pos = it.pos0 + ql;
+      const int qrow = it.qrow0 + ql;
+      float m_used = -INFINITY, l = 0.f;
+      if (active && n > 0 && ok) {
+        const int* idx_row =
+            (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
+        for (int i = 0; i < n; ++i) {
+          if (!mbar_wait_warp(&c.s_full[t], (uses + i) & 1, abort_flag, p.wc, 20)) { ok = false; break; }
+          tc_fence_after();
+          uint32_t u[128];
+          tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
+          tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
+          tmem_ld_wait();
+          float x[128];
+#pragma unroll
+          for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(u[j]) * p.scale_log2;
+          // ---- masks ----
+          if (MODE == kFull) {
+            const int key0 = i * 128;
+            if (key0 + 127 > pos) {
+#pragma unroll
+              for (int j = 0; j < 128; ++j)
+                if (key0 + j > pos) x[j] = -INFINITY;
+            }
+          } else if (i < kp.n_sel) {
+            if constexpr (SB > 0) {
+              // selected keys must satisfy key <= pos - w; keys of a block are
+              // consecutive, so each block gives one threshold on j % SB
+              constexpr int nb = 128 / SB;
+              const int lim = pos - p.w;
+              const int slot_last = min(kp.cnt, (i + 1) * nb) - 1;
+              const int maxkey = __ldg(idx_row + slot_last) * SB + SB - 1;
+              if (maxkey > lim || (i + 1) * nb > kp.cnt) {
+                int thr[nb];
+#pragma unroll
+                for (int b = 0; b < nb; ++b) {
+                  const int slot = i * nb + b;
+                  thr[b] = slot < kp.cnt ? lim - __ldg(idx_row + slot) * SB : -1;
+                }
+#pragma unroll
+                for (int j = 0; j < 128; ++j)
+                  if ((j % SB) > thr[j / SB]) x[j] = -INFINITY;
+              }
+            }
+          } else {
+            const int key0 = kp.win_lo + (i - kp.n_sel) * 128;
+            const int lo = pos - p.w + 1;
+#pragma unroll
+            for (int j = 0; j < 128; ++j) {
+              const int key = key0 + j;
+              if (key < lo || key > pos) x[j] = -INFINITY;
+            }
+          }
+          // ---- block maxima for the score by-product (full mode) ----
+          float mt = -INFINITY;
+          if constexpr (MODE == kFull && SB > 0) {
+            constexpr int nb = 128 / SB;
+            float* sp = p.spill + (size_t(blockIdx.x) * p.nblk) * kMaxItemRows + vr;
+#pragma unroll
+            for (int b = 0; b < nb; ++b) {
+              float mb = -INFINITY;
+#pragma unroll
+              for (int j = b * SB; j < (b + 1) * SB; ++j) mb = fmaxf(mb, x[j]);
+              const int gb = i * nb + b;
+              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = mb;
+              mt = fmaxf(mt, mb);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 128; ++j) mt = fmaxf(mt, x[j]);
+          }
+          // ---- online softmax with lazy rescaling (exact: O and l share m_used) ----
+          float factor = 1.f;
+          bool rescale = false;
+          if (mt > m_used + 8.f) {
+            const float m_new = mt;
+            factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
+            m_used = m_new;
+            rescale = true;
+          }
+          const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+          float rs = 0.f;
+          uint32_t pk[64];
+#pragma unroll
+          for (int j = 0; j < 128; j += 2) {
+            const float a = ex2(x[j] - mu), b2 = ex2(x[j + 1] - mu);
+            rs += a + b2;
+            pk[j >> 1] = pack_bf16(a, b2);
+          }
+          l = l * factor + rs;
+          // P buffer and O are free once the previous PV of this tile is done
+          if (i > 0 && !mbar_wait_warp(&c.o_ready[t], (uses + i - 1) & 1, abort_flag, p.wc, 21)) { ok = false; break; }
+          if (rescale && i > 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t ov[32];
+              tmem_ld32(t_o + ch * 32, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * factor);
+              tmem_st32(t_o + ch * 32, ov);
+            }
+            tmem_st_wait();
+          }
+#pragma unroll
+          for (int cc = 0; cc < 16; ++cc) {
+            const int slab = cc >> 3;
+            const int chunk = (cc & 7) ^ (r & 7);
+            *reinterpret_cast<uint4*>(p_tile + slab * kSlabBytes + r * 128 + chunk * 16) =
+                make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+          }
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.p_full[t]);
+        }
+        // ---- epilogue: O / l, lse ----
+        if (ok && mbar_wait_warp(&c.o_ready[t], (uses + n - 1) & 1, abort_flag, p.wc, 22)) {
+          tc_fence_after();
+          const float inv = l > 0.f ? 1.f / l : 0.f;
+          __nv_bfloat16* orow = p.o + (size_t(qrow) * p.Hq + h) * D;
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t ov[32];
+            tmem_ld32(t_o + ch * 32, ov);
+            tmem_ld_wait();
+            if (valid) {
+              float of[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) of[j] = __uint_as_float(ov[j]) * inv;
+              if (p.gamma) {
+                const float sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
+                const uint4* src = reinterpret_cast<const uint4*>(p.o_other + (size_t(qrow) * p.Hq + h) * D + ch * 32);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint4 u4 = __ldg(src + j);
+                  const uint32_t w4[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
+                    const float2 f2 = __bfloat1622float2(b2);
+                    of[8 * j + 2 * e] = sg * f2.x + (1.f - sg) * of[8 * j + 2 * e];
+                    of[8 * j + 2 * e + 1] = sg * f2.y + (1.f - sg) * of[8 * j + 2 * e + 1];
+                  }
+                }
+              }
+              uint32_t pk2[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pk2[j] = pack_bf16(of[2 * j], of[2 * j + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk2[4 * j], pk2[4 * j + 1], pk2[4 * j + 2], pk2[4 * j + 3]);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.o_free[t]);
+        } else {
+          ok = false;
+        }
+        uses += n;
+        items_t += 1;
+      } else if (valid && (n == 0 || !active)) {
+        // no visible key at all (sparse, k = 0 and w = 0): o = 0, lse = -inf
+        if (n == 0) {
+          uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(qrow) * p.Hq + h) * D);
+          for (int j = 0; j < D / 8; ++j) dst[j] = make_uint4(0, 0, 0, 0);
+        }
+      }
+      const float lse2 = (l > 0.f) ? m_used + __log2f(l) : -INFINITY;
+      if (valid && active && p.lse) p.lse[size_t(h) * p.Tq + qrow] = lse2 * 0.69314718055994531f;
+      if (valid && n == 0 && p.lse) p.lse[size_t(h) * p.Tq + qrow] = -INFINITY;
+      // ---- score epilogue (full mode, B > 1): max over the tile's rows ----
+      if constexpr (MODE == kFull && SB > 0) {
+        c.lse2[vr] = lse2;
+        __threadfence_block();
+        named_bar_sync(1, 256);
+        if (ok && !*abort_flag) {
+          const int nblk_item = min(p.nblk, (n * 128) / SB);
+          const float* sp = p.spill + size_t(blockIdx.x) * p.nblk * kMaxItemRows;
+          const int sw = warp;  // 0..7
+          for (int b = sw; b < nblk_item; b += 8) {
+            int qa = 0;
+            while (qa < it.nq) {
+              const int in_tile = (it.qoff + qa) % p.T;
+              const int tid = it.tile0 + (it.qoff + qa) / p.T;
+              const int qb = min(it.nq, qa + (p.T - in_tile));
+              const int tile_last = min(it.pos0 + qa - in_tile + p.T - 1, it.kv_len - 1);
+              if (b * SB <= tile_last) {
+                float v = -INFINITY;
+                for (int rr = qa * p.G + lane; rr < qb * p.G; rr += 32)
+                  v = fmaxf(v, sp[size_t(b) * kMaxItemRows + rr] - c.lse2[rr]);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                if (lane == 0 && v > -INFINITY)
+                  atomicMax(reinterpret_cast<unsigned int*>(p.scores + (size_t(tid) * p.Hkv + it.g) * p.nblk + b),
+                            __float_as_uint(ex2(v)));
+              }
+              qa = qb;
+            }
+          }
+        }
+        named_bar_sync(1, 256);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace attn
+}  // namespace hs

@@ -1,0 +1,145 @@
+// topk.cuh -- per-(tile, KV head) top-k selection over importance scores.
+//
+// TopK over the full layer's block scores (HySparse explainer, techwalker.com)
+// or token scores with k = 1024 (HySparse2 release note; demingchina
+// commentary section 03). Candidates of a tile are the blocks b with
+// b*B <= last query position of the tile. Rule: score descending, ties to the
+// lower index; the kept set is written in ascending index order, padded -1.
+//
+// Method: scores are >= 0, so their fp32 bit patterns order like the values.
+// A 4-pass MSB-first radix select (8 bits per pass, per-warp histograms in
+// shared memory) finds the k-th largest bit pattern tau and how many of the
+// k slots go to entries equal to tau. A final pass walks the row in index
+// order with a block-wide prefix scan and keeps every entry > tau plus the
+// first (k - #greater) entries == tau. Walking in index order both breaks
+// ties toward the lower index and emits the result already sorted.
+#pragma once
+
+#include "hs_common.cuh"
+#include "seqtable.cuh"
+
+namespace hs {
+namespace topk {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+
+struct Params {
+  const float* scores;  // [n_tiles, Hkv, nblk]
+  int* idx;             // [n_tiles, Hkv, k]
+  int* cnt;             // [n_tiles, Hkv]
+  int Hkv, nblk, B, k;
+};
+
+// Block-wide exclusive scan of one int per thread; returns the total.
+__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, off);
+    if (lane >= off) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int s = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += y;
+    }
+    warp_sums[lane] = s;  // inclusive
+  }
+  __syncthreads();
+  total = warp_sums[kWarps - 1];
+  const int base = warp > 0 ? warp_sums[warp - 1] : 0;
+  __syncthreads();
+  return base + x - v;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    topk_kernel(const Params p, const __grid_constant__ SeqTable st) {
+  __shared__ int hist[kWarps][256];
+  __shared__ int total_hist[256];
+  __shared__ int warp_sums[kWarps];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_krem;
+
+  const int row = blockIdx.x;  // tile * Hkv + g
+  const int tile = row / p.Hkv;
+  const TileInfo ti = tile_info(st, tile);
+  const int last_pos = ti.pos0 + ti.n - 1;
+  const int n = min(p.nblk, last_pos / p.B + 1);
+  const uint32_t* keys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
+  int* out = p.idx + size_t(row) * p.k;
+  const int k = p.k;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  if (n <= k) {
+    // every candidate is kept
+    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
+    if (threadIdx.x == 0) p.cnt[row] = n;
+    return;
+  }
+  if (k == 0) {
+    if (threadIdx.x == 0) p.cnt[row] = 0;
+    return;
+  }
+
+  // ---- radix select of the k-th largest bit pattern ----
+  uint32_t prefix = 0;  // fixed high bits of tau
+  int krem = k;         // how many of the k still to place at/below the prefix
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int b = lane; b < 256; b += 32) hist[warp][b] = 0;
+    __syncwarp();
+    for (int j = threadIdx.x; j < n; j += kThreads) {
+      const uint32_t key = __ldg(keys + j);
+      if ((key & hi_mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 0xFF], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 256) {
+      int s = 0;
+      for (int w = 0; w < kWarps; ++w) s += hist[w][threadIdx.x];
+      total_hist[threadIdx.x] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int acc = 0, b = 255;
+      for (; b > 0; --b) {
+        if (acc + total_hist[b] >= krem) break;
+        acc += total_hist[b];
+      }
+      s_prefix = prefix | (uint32_t(b) << shift);
+      s_krem = krem - acc;
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    krem = s_krem;
+  }
+  const uint32_t tau = prefix;
+  const int take_eq = krem;  // entries equal to tau to keep (lowest indices)
+
+  // ---- ordered compaction ----
+  int out_base = 0, eq_base = 0;
+  for (int j0 = 0; j0 < n; j0 += kThreads) {
+    const int j = j0 + threadIdx.x;
+    const uint32_t key = j < n ? __ldg(keys + j) : 0u;
+    const int is_eq = (j < n && key == tau) ? 1 : 0;
+    int eq_total;
+    const int eq_rank = eq_base + block_excl_scan(is_eq, warp_sums, eq_total);
+    const int sel = (j < n) && (key > tau || (is_eq && eq_rank < take_eq));
+    int sel_total;
+    const int pos = out_base + block_excl_scan(sel, warp_sums, sel_total);
+    if (sel) out[pos] = j;
+    out_base += sel_total;
+    eq_base += eq_total;
+  }
+  for (int j = out_base + threadIdx.x; j < k; j += kThreads) out[j] = -1;
+  if (threadIdx.x == 0) p.cnt[row] = out_base;
+}
+
+}  // namespace topk
+}  // namespace hs

@@ -1,0 +1,222 @@
+/*
+ * hs.h -- C ABI of libhs, the hybrid-block sparse attention hot path
+ * (HySparse / HySparse2) for NVIDIA B200 (sm_100a).
+ *
+ * A hybrid block is one full causal attention layer followed by N sparse
+ * attention layers that reuse the full layer's KV cache and its per-tile
+ * top-k key selection (QbitAI repost of HySparse, "hybrid block" paragraphs;
+ * HySparse2 release note on airebao.com, "KV Reuse").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * Pointers: every tensor argument is a DEVICE pointer owned by the caller,
+ *   except hs_varlen.cu_q_host / cu_kv_host, which are HOST pointers.
+ *   The library never allocates or frees memory. Calls that need scratch take
+ *   a caller-owned device workspace `ws` of at least hs_workspace_size(op, ...)
+ *   bytes; call hs_workspace_init() once on a new workspace.
+ * Streams: every call only enqueues work on `stream` and returns; nothing
+ *   synchronises except hs_check_error().
+ * Varlen packing: sequence b has n_b new queries and kv_b = c_b + n_b keys
+ *   (c_b cached tokens; the new tokens' K/V are already appended). Query rows
+ *   of all sequences are packed along one token axis with prefix sums cu_q;
+ *   keys likewise with cu_kv. Query i of sequence b sits at position
+ *   c_b + i of that sequence.
+ * Layouts (row-major, token-major, contiguous):
+ *   Q, O      [T_q,  H_q,  d]   bf16
+ *   K, V      [T_kv, H_kv, d]   bf16 (or e4m3 bytes for FP8 decode)
+ *   lse       [H_q, T_q]        fp32, natural log
+ *   gamma     [T_q, H_q]        fp32
+ *   scores    [n_tiles, H_kv, n_blk]  fp32, n_blk = ceil(max_kv / B)
+ *   idx       [n_tiles, H_kv, k] int32 ascending, padded with -1
+ *   cnt       [n_tiles, H_kv]   int32
+ *   Query head h reads KV head h / (H_q / H_kv). Selection tile i of sequence
+ *   b covers its new queries [i*T, min((i+1)*T, n_b)); tiles are numbered
+ *   sequence after sequence; n_tiles = sum_b ceil(n_b / T).
+ * Errors: each call validates its arguments on the host before launching
+ *   anything and returns a status. Device-side failures (a bounded wait that
+ *   gave up) are recorded in the workspace and reported by hs_check_error().
+ */
+#ifndef HS_H_
+#define HS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HS_API __attribute__((visibility("default")))
+#else
+#define HS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* hs_stream_t; /* same object as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  HS_OK = 0,
+  HS_ERR_INVALID_ARG = 1,  /* null pointer, bad size, inconsistent prefix sums */
+  HS_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. head_dim not 64/128) */
+  HS_ERR_WORKSPACE = 3,    /* workspace missing or smaller than hs_workspace_size() */
+  HS_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  HS_ERR_TIMEOUT = 5       /* a device-side bounded wait gave up (see hs_check_error) */
+} hs_status;
+
+typedef struct {
+  int32_t batch;           /* number of sequences, >= 1 */
+  int32_t n_q_heads;       /* H_q */
+  int32_t n_kv_heads;      /* H_kv; H_q % H_kv == 0 */
+  int32_t head_dim;        /* d: 64 or 128 */
+  const int32_t* cu_q;     /* device [batch+1] prefix sums of n_b */
+  const int32_t* cu_kv;    /* device [batch+1] prefix sums of kv_b */
+  const int32_t* cu_q_host;  /* host copy of cu_q (same values) */
+  const int32_t* cu_kv_host; /* host copy of cu_kv (same values) */
+  float softmax_scale;     /* 0 => 1/sqrt(d) */
+} hs_varlen;
+
+typedef struct {
+  int32_t q_tile;  /* T: queries per selection tile (1 for decode) */
+  int32_t block;   /* B: keys per selectable block; 1 = token-level selection */
+  int32_t topk;    /* k: blocks kept per (tile, KV head); 0 <= k <= 4096 */
+  int32_t window;  /* w: forced recent window (tokens) unioned into the sparse set */
+} hs_sel;
+
+typedef enum { HS_KV_BF16 = 0, HS_KV_FP8_E4M3 = 1 } hs_kv_dtype;
+
+typedef enum {
+  HS_OP_FULL_ATTN_SELECT = 0,
+  HS_OP_TOPK_SELECT = 1,
+  HS_OP_SPARSE_ATTN_PREFILL = 2,
+  HS_OP_SPARSE_ATTN_DECODE = 3,
+  HS_OP_SWA_GATED = 4
+} hs_op;
+
+/* Bytes of workspace that `op` needs for these shapes (0 on invalid input).
+ * The first 256 bytes of every workspace hold the device error word. */
+HS_API size_t hs_workspace_size(int op, const hs_varlen* vl, const hs_sel* sel);
+
+/* Zero the workspace header (error word). Call once on a new workspace. */
+HS_API hs_status hs_workspace_init(void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace error word.
+ * Returns HS_ERR_TIMEOUT if a kernel's bounded wait gave up since the last
+ * check, HS_ERR_CUDA if the stream reports an error, else HS_OK. */
+HS_API hs_status hs_check_error(void* ws, hs_stream_t stream);
+
+/* Static description of a status code. */
+HS_API const char* hs_status_string(hs_status s);
+
+/*
+ * hs_full_attn_select -- the full attention layer of a hybrid block.
+ *
+ * Computes causal scaled dot-product attention (HySparse explainer on
+ * techwalker.com: the master layer runs standard scaled dot-product
+ * attention) and, as a by-product, the key-importance scores that drive the
+ * selection (same page: a lightly modified FlashAttention kernel emits
+ * block-level maximum attention scores reusing the online-softmax row max;
+ * HySparse2 release note: top-k selection is a free by-product):
+ *   s_{q,h,j} = (q_{q,h} . k_{j,g}) * scale,           j <= pos(q)
+ *   o_{q,h}   = sum_j softmax_j(s) v_{j,g},   lse_{q,h} = ln sum_j exp(s)
+ *   score(t, g, b) = max over q in tile t, h in group g, j in block b,
+ *                    j <= pos(q), of exp(s_{q,h,j} - lse_{q,h}).
+ * Blocks with b*B > last position of t are not candidates; their score is 0.
+ * In:  q [T_q,H_q,d], k/v [T_kv,H_kv,d] bf16. Out: o bf16, lse fp32, scores fp32.
+ * Supported: d in {64,128}; G = H_q/H_kv a power of two <= 128; B = 1 or a
+ * power of two <= 128 (B = 1 adds a second QK pass for token-level scores).
+ * Decode (n_b = 1 for every sequence, T = 1) is dispatched to a split-K path.
+ * Errors: HS_ERR_INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch.
+ */
+HS_API hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel,
+                              const void* q, const void* k, const void* v,
+                              void* o, float* lse, float* scores,
+                              void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_topk_select -- keep the k best candidate blocks per (tile, KV head).
+ *
+ * HySparse explainer (techwalker.com): TopK over the block scores picks the
+ * key blocks; HySparse2 release note and demingchina commentary section 03:
+ * token-level selection of 1024 tokens. Candidates of tile t are blocks
+ * b <= floor(last_pos(t) / B). Order: score descending, ties to the lower
+ * index. Output idx ascending, padded with -1; cnt = min(k, #candidates).
+ * The forced recent window is not applied here: the sparse attention calls
+ * union it per query.
+ * In: scores [n_tiles,H_kv,n_blk] fp32 (>= 0). Out: idx [n_tiles,H_kv,k], cnt.
+ */
+HS_API hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* scores,
+                         int32_t* idx, int32_t* cnt,
+                         void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_sparse_attn_prefill -- one sparse layer of a hybrid block.
+ *
+ * This layer's own queries attend over the full layer's K/V (KV Reuse) at
+ * the keys selected for their tile, plus the forced recent window
+ * (QbitAI repost: block-sparse global branch over the TopK blocks of the
+ * shared KV cache; HySparse2 release note: the latest 128 tokens are forced
+ * into the selected set):
+ *   V_q = { j in blocks(idx_t) : j <= pos(q) - w }  U  [max(0, pos(q)-w+1), pos(q)]
+ *   o_{q,h} = sum_{j in V_q} softmax_j(s) v_{j,g};  lse as above.
+ * An empty V_q (only possible with w = 0) yields o = 0 and lse = -inf.
+ * In: q [T_q,H_q,d], k/v (full layer's) [T_kv,H_kv,d], idx/cnt from
+ * hs_topk_select. Out: o bf16, lse fp32 (lse may be NULL).
+ */
+HS_API hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel,
+                                 const void* q, const void* k, const void* v,
+                                 const int32_t* idx, const int32_t* cnt,
+                                 void* o, float* lse,
+                                 void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_sparse_attn_decode -- sparse layer for one new token per sequence.
+ *
+ * Same set V_q as the prefill call with T = 1, computed split-K over the
+ * selected keys and merged by their log-sum-exp. The KV cache may be bf16 or
+ * FP8 e4m3 (the HySparse2 key-data table sizes an FP8 KV cache); FP8 values
+ * decode as x = scale[token, kv_head] * e4m3(code), with separate fp32 scale
+ * arrays for K and V ([T_kv, H_kv]; NULL for bf16).
+ * split_k: number of key chunks per sequence (0 = automatic).
+ * Requires n_b = 1 for every sequence and sel->q_tile = 1.
+ */
+HS_API hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel,
+                                const void* q, hs_kv_dtype kv_dtype,
+                                const void* k, const void* v,
+                                const float* k_scale, const float* v_scale,
+                                const int32_t* idx, const int32_t* cnt, int32_t split_k,
+                                void* o, float* lse,
+                                void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_swa_gated -- HySparse's local branch and the gate that fuses it.
+ *
+ * The sliding-window branch uses the same queries over the layer's OWN small
+ * KV cache (QbitAI repost: window of 128 by default; HySparse explainer: the
+ * window branch must not share the full layer's KV), keys
+ * [max(0, pos(q)-window+1), pos(q)], and the two branch outputs are fused by
+ * a sigmoid gate (both pages). Reading of the gate:
+ *   o = sigmoid(gamma) * o_sparse + (1 - sigmoid(gamma)) * o_swa,
+ * gamma given per (token, query head).
+ * In: q [T_q,H_q,d], k_swa/v_swa [T_kv,H_kv,d] bf16, gamma [T_q,H_q] fp32,
+ * o_sparse [T_q,H_q,d] bf16. Out: o [T_q,H_q,d] bf16 (may alias o_sparse).
+ */
+HS_API hs_status hs_swa_gated(const hs_varlen* vl, int32_t window,
+                       const void* q, const void* k_swa, const void* v_swa,
+                       const float* gamma, const void* o_sparse, void* o,
+                       void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_debug_wait_timeout -- failure-detection self test (no counterpart on the
+ * pages). Launches one tiny kernel that waits on a barrier nothing arrives
+ * at; its bounded wait gives up after `timeout_ns` (1 .. 2e9), records the
+ * failure in the workspace error word and returns, leaving the context
+ * usable. hs_check_error() then reports HS_ERR_TIMEOUT and clears the word.
+ * This is the same bounded wait every pipelined kernel uses.
+ */
+HS_API hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, hs_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS_H_ */

@@ -1,0 +1,88 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hybrid_sparse_attention_tma_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "hs.h")).read()
+    return sorted(set(re.findall(r"HS_API\s+[\w\s\*]+?\b(hs_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_five_calls():
+    names = header_functions()
+    for n in ["hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill", "hs_sparse_attn_decode",
+              "hs_swa_gated"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from hybrid_sparse_attention_tma_b200 import _lib
+    for n in header_functions():
+        assert hasattr(lib, n), n
+    assert sorted(_lib.EXPORTS) == header_functions()
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.hs_status_string(s)
+
+
+def _varlen(cu_q, cu_kv, hq=4, hkv=1, d=64):
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    cq = (ctypes.c_int32 * len(cu_q))(*cu_q)
+    ckv = (ctypes.c_int32 * len(cu_kv))(*cu_kv)
+    vl = L.HsVarlen(len(cu_q) - 1, hq, hkv, d, 16, 16, cq, ckv, 0.0)
+    vl._keep = (cq, ckv)
+    return vl
+
+
+def test_workspace_size_and_validation(lib):
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    vl = _varlen([0, 512], [0, 512])
+    sel = L.HsSel(16, 16, 8, 32)
+    n = lib.hs_workspace_size(L.HS_OP_FULL_ATTN_SELECT, ctypes.byref(vl), ctypes.byref(sel))
+    assert n >= 256 and n % 256 == 0
+    assert lib.hs_workspace_size(L.HS_OP_TOPK_SELECT, ctypes.byref(vl), ctypes.byref(sel)) >= 256
+    bad = _varlen([0, 512], [0, 100])  # fewer keys than queries
+    assert lib.hs_workspace_size(L.HS_OP_FULL_ATTN_SELECT, ctypes.byref(bad), ctypes.byref(sel)) == 0
+
+
+def _call_full(lib, vl, sel, ptr=16, ws=16, ws_bytes=1 << 30):
+    return lib.hs_full_attn_select(ctypes.byref(vl) if vl is not None else None,
+                                   ctypes.byref(sel) if sel is not None else None,
+                                   ptr, ptr, ptr, ptr, ptr, ptr, ws, ws_bytes, None)
+
+
+def test_host_validation_errors(lib):
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    vl = _varlen([0, 512], [0, 512])
+    sel = L.HsSel(16, 16, 8, 32)
+    assert _call_full(lib, None, sel) == L.HS_ERR_INVALID_ARG
+    assert _call_full(lib, vl, None) == L.HS_ERR_INVALID_ARG
+    assert _call_full(lib, vl, sel, ptr=None) == L.HS_ERR_INVALID_ARG
+    assert _call_full(lib, vl, sel, ptr=18) == L.HS_ERR_INVALID_ARG          # misaligned
+    assert _call_full(lib, vl, sel, ws=None) == L.HS_ERR_WORKSPACE
+    assert _call_full(lib, vl, sel, ws_bytes=8) == L.HS_ERR_WORKSPACE
+    assert _call_full(lib, _varlen([0, 512], [0, 512], d=96), sel) == L.HS_ERR_UNSUPPORTED
+    assert _call_full(lib, _varlen([0, 512], [0, 512], hq=6, hkv=4), sel) == L.HS_ERR_INVALID_ARG
+    assert _call_full(lib, vl, L.HsSel(16, 24, 8, 32)) == L.HS_ERR_UNSUPPORTED  # block not a power of 2
+    assert _call_full(lib, vl, L.HsSel(16, 16, 5000, 32)) == L.HS_ERR_UNSUPPORTED
+    assert _call_full(lib, vl, L.HsSel(0, 16, 8, 32)) == L.HS_ERR_INVALID_ARG
+    assert _call_full(lib, _varlen([0, 600], [0, 512]), sel) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_swa_gated(ctypes.byref(vl), 0, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_topk_select(ctypes.byref(vl), ctypes.byref(sel), None, 16, 16, 16, 1 << 20, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
+    assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG

@@ -1,0 +1,151 @@
+"""GPU (libhs through its C ABI) against the fp64 oracle, element by element.
+
+Whole-problem checks at sizes the oracle finishes in seconds (several tiles,
+ragged tails, chunked prefill, GQA/MQA, both head dims), and sampled tiles of
+the full-size HySparse block-level workload in the benchmark's launch
+configuration.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from oracle.block import tile_rows
+import workloads as W
+from tests.parity import (GpuBlock, f64, assert_close_out, assert_close_lse, assert_scores_close,
+                          assert_indices_match)
+
+pytestmark = pytest.mark.gpu
+
+
+def _layers_f64(inp, rows=None):
+    out = []
+    for L in inp.layers:
+        d = {"q": f64(L.q)}
+        if L.k_swa is not None:
+            d.update(k_swa=f64(L.k_swa), v_swa=f64(L.v_swa), gamma=f64(L.gamma))
+        out.append(d)
+    return out
+
+
+def check_block(w, inp, res, tile_ids=None):
+    """Compare every step of one hybrid block on the given tiles (None = all)."""
+    cu_q, cu_kv = w.cu_q(), w.cu_kv()
+    T, B = w.q_tile, w.block
+    q, k, v = f64(inp.q), f64(inp.k), f64(inp.v)
+    tiles = O.make_tiles(cu_q, cu_kv, T)
+    tids = list(range(len(tiles))) if tile_ids is None else list(tile_ids)
+    rows = tile_rows(cu_q, cu_kv, T, tids)
+    # A1: full attention
+    o_o, lse_o = O.full_attention(q, k, v, cu_q, cu_kv, w.n_kv_heads, tiles_T=T, tile_ids=tids)
+    o_g, lse_g = f64(res["o_full"]), f64(res["lse_full"])
+    assert_close_out(o_g[rows], o_o[rows], what="full o")
+    assert_close_lse(lse_g[:, rows], lse_o[:, rows], what="full lse")
+    # A2: scores
+    sc_o = O.importance_scores(q, k, lse_o, cu_q, cu_kv, w.n_kv_heads, T, B, tile_ids=tids)
+    sc_g = f64(res["scores"])
+    assert_scores_close(sc_g, sc_o, tids)
+    # A3: top-k -- exact on the GPU's own scores, tie band against the oracle's
+    idx_g, cnt_g = res["idx"].cpu().numpy(), res["cnt"].cpu().numpy()
+    idx_x, cnt_x = O.topk_select(sc_g, cu_q, cu_kv, T, B, w.topk, tile_ids=tids)
+    kk = max(w.topk, 1)
+    for t in tids:
+        assert (cnt_g[t] == cnt_x[t]).all()
+        assert (idx_g[t, :, :w.topk] == idx_x[t]).all(), f"top-k of GPU scores differs in tile {t}"
+    idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids)
+    assert_indices_match(idx_g[:, :, :w.topk], cnt_g, sc_o, idx_o, cnt_o, tids, kk)
+    # A4 / A5: sparse layers, fed the GPU's (checked) indices
+    for li, (L, Lg) in enumerate(zip(_layers_f64(inp), res["layers"])):
+        o_sp, lse_sp = O.sparse_attention(L["q"], k, v, idx_g[:, :, :w.topk], cnt_g, cu_q, cu_kv, T, B,
+                                          w.window, tile_ids=tids)
+        assert_close_out(f64(Lg["o_sparse"])[rows], o_sp[rows], what=f"layer {li} sparse o")
+        assert_close_lse(f64(Lg["lse_sparse"])[:, rows], lse_sp[:, rows], what=f"layer {li} sparse lse")
+        if w.swa_window > 0:
+            o_swa, _ = O.swa_attention(L["q"], L["k_swa"], L["v_swa"], cu_q, cu_kv, w.swa_window, row_ids=rows)
+            # gate applied to the GPU's bf16 sparse output (the call's actual input)
+            o_gate = O.gated_merge(L["gamma"], f64(Lg["o_sparse"]), o_swa)
+            assert_close_out(f64(Lg["o"])[rows], o_gate[rows], what=f"layer {li} gated o")
+            # and the whole chain against the oracle's own sparse output
+            o_chain = O.gated_merge(L["gamma"], o_sp, o_swa)
+            assert_close_out(f64(Lg["o"])[rows], o_chain[rows], what=f"layer {li} chain o")
+
+
+def run_and_check(w, seed=None, tile_ids=None):
+    inp = W.make_block_inputs(w, device="cuda", seed=seed)
+    res = GpuBlock(w, inp).run()
+    torch.cuda.synchronize()
+    check_block(w, inp, res, tile_ids)
+    return inp, res
+
+
+def test_tiny_config_whole():
+    run_and_check(W.WORKLOADS["tiny"])
+
+
+VARIANTS = {
+    # chunked prefill, ragged tails, GQA group 4, d=128, 64-token blocks, no window
+    "gqa4_d128_b64_w0": W.Workload("v1", ctx=(0, 300, 37), new=(200, 333, 130), n_q_heads=8, n_kv_heads=2,
+                                   head_dim=128, q_tile=64, block=64, topk=3, window=0, n_sparse=1),
+    # MQA with 16 heads, window 128, blocks of 16, tile 16
+    "mqa16_d128_b16_w128": W.Workload("v2", ctx=(0, 257), new=(300, 77), n_q_heads=16, n_kv_heads=1,
+                                      head_dim=128, q_tile=16, block=16, topk=8, window=128, n_sparse=1),
+    # MHA (G=1), d=64, block 32, window 16
+    "mha_d64_b32": W.Workload("v3", ctx=(5,), new=(259,), n_q_heads=2, n_kv_heads=2, head_dim=64,
+                              q_tile=32, block=32, topk=2, window=16, n_sparse=1),
+    # k >= all candidates: sparse must equal full attention
+    "k_all": W.Workload("v4", ctx=(0,), new=(256,), n_q_heads=4, n_kv_heads=1, head_dim=64, q_tile=64,
+                        block=16, topk=64, window=0, n_sparse=1),
+    # k = 0 with a window: sparse = window-only attention
+    "k0_window": W.Workload("v5", ctx=(0,), new=(200,), n_q_heads=4, n_kv_heads=1, head_dim=64, q_tile=16,
+                            block=16, topk=0, window=24, n_sparse=1),
+    # G = 128 (two queries per M tile)
+    "g128": W.Workload("v6", ctx=(60,), new=(9,), n_q_heads=128, n_kv_heads=1, head_dim=128, q_tile=4,
+                       block=8, topk=4, window=8, n_sparse=1),
+    # SWA + gate branch at small size
+    "swa_gate": W.Workload("v7", ctx=(0, 100), new=(300, 200), n_q_heads=8, n_kv_heads=2, head_dim=128,
+                           q_tile=64, block=64, topk=2, window=0, n_sparse=2, swa_window=128),
+}
+
+
+@pytest.mark.parametrize("name", list(VARIANTS))
+def test_variant_whole(name):
+    run_and_check(VARIANTS[name], seed=7)
+
+
+def test_k_all_equals_full_attention_on_gpu():
+    w = VARIANTS["k_all"]
+    inp = W.make_block_inputs(w, device="cuda", seed=3)
+    import hybrid_sparse_attention_tma_b200 as hs
+    blk = GpuBlock(w, inp)
+    res = blk.run()
+    o_f, lse_f, _ = hs.full_attn_select(blk.vl, blk.sel, inp.layers[0].q, inp.k, inp.v)
+    torch.cuda.synchronize()
+    assert_close_out(f64(res["layers"][0]["o_sparse"]), f64(o_f), what="k>=all vs full")
+    assert_close_lse(f64(res["layers"][0]["lse_sparse"]), f64(lse_f), what="k>=all lse vs full")
+
+
+def test_hys_block_full_size_sampled_tiles():
+    """HySparse block-level prefill at full size (32768 tokens, 32/8 heads,
+    d=128, B=64, k=16, SWA 128 + gate), 3 sparse layers, checked on sampled
+    tiles including the first and the last."""
+    w = W.WORKLOADS["hys_block"]
+    n_t = w.n_tiles()
+    rng = np.random.default_rng(11)
+    tiles = sorted({0, n_t - 1, *rng.choice(n_t, size=2, replace=False).tolist()})
+    run_and_check(w, tile_ids=tiles)
+
+
+def test_bounded_wait_timeout_reports_and_context_survives():
+    import ctypes
+    import hybrid_sparse_attention_tma_b200 as hs
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    ws = hs.Workspace("cuda")
+    buf = ws.get(4096)
+    lib = L.load()
+    s = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.hs_debug_wait_timeout(ctypes.c_void_p(buf.data_ptr()), buf.numel(), 2_000_000, s) == L.HS_OK
+    with pytest.raises(hs.HsError) as e:
+        hs.check_error(ws)
+    assert e.value.status == L.HS_ERR_TIMEOUT
+    hs.check_error(ws)  # cleared
+    run_and_check(VARIANTS["k0_window"], seed=1)
