@@ -15,7 +15,7 @@ HS_KV_BF16, HS_KV_FP8_E4M3 = 0, 1
 EXPORTS = [
     "hs_workspace_size", "hs_workspace_init", "hs_check_error", "hs_status_string",
     "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
-    "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout",
+    "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
 ]
 
 
@@ -71,6 +71,8 @@ def load():
     lib.hs_sparse_attn_decode.argtypes = [VL, SEL, vp, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
     lib.hs_swa_gated.restype = i32
     lib.hs_swa_gated.argtypes = [VL, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hs_last_error_detail.restype = i32
+    lib.hs_last_error_detail.argtypes = [ctypes.POINTER(i32)] * 3
     lib.hs_debug_wait_timeout.restype = i32
     lib.hs_debug_wait_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
     _lib = lib
@@ -79,5 +81,10 @@ def load():
 
 def check(fn: str, status: int):
     if status != HS_OK:
-        msg = load().hs_status_string(status).decode()
+        lib = load()
+        msg = lib.hs_status_string(status).decode()
+        if status == HS_ERR_TIMEOUT:
+            a, b, c = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+            lib.hs_last_error_detail(ctypes.byref(a), ctypes.byref(b), ctypes.byref(c))
+            msg += f"; site {a.value}, block {b.value}, item {c.value >> 12}, step {c.value & 0xFFF}"
         raise HsError(fn, status, msg)

@@ -279,12 +279,15 @@ hs_status hs_workspace_init(void* ws, size_t ws_bytes, hs_stream_t stream) {
   return cudaMemsetAsync(ws, 0, kHeaderBytes, S(stream)) == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
+static ErrWord last_err{};
+
 hs_status hs_check_error(void* ws, hs_stream_t stream) {
   if (!ws) return HS_ERR_WORKSPACE;
   if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return HS_ERR_CUDA;
   ErrWord e{};
   if (cudaMemcpy(&e, ws, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return HS_ERR_CUDA;
   if (e.flag != 0) {
+    last_err = e;
     if (cudaMemset(ws, 0, sizeof(ErrWord)) != cudaSuccess) return HS_ERR_CUDA;
     return HS_ERR_TIMEOUT;
   }
@@ -471,6 +474,14 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
   p.wc = wait_ctl(ws);
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
   return dispatch_attn_d<attn::kSparse, 0>(sh.d, m, p, sc, grid, S(stream));
+}
+
+hs_status hs_last_error_detail(int32_t* site, int32_t* block, int32_t* ctx) {
+  if (!site || !block || !ctx) return HS_ERR_INVALID_ARG;
+  *site = last_err.site;
+  *block = last_err.block;
+  *ctx = last_err.ctx;
+  return HS_OK;
 }
 
 hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, hs_stream_t stream) {

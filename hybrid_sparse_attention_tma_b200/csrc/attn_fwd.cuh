@@ -102,6 +102,7 @@ struct Ctl {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_ready[2], o_free[2];
   uint64_t teardown;
+  uint64_t sm_bar;  // bounded barrier over the 256 softmax threads
   uint32_t tmem_base;
   int abort;
   float lse2[kMaxItemRows];
@@ -209,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.o_free[t], 4);
     }
     mbar_init(&c.teardown, 1);
+    mbar_init(&c.sm_bar, 256);
     c.abort = 0;
     fence_mbar_init();
   }
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (n == 0) continue;
         const int rows = it.nq * p.G;
         const int n_qt = rows > 128 ? 2 : 1;
-        if (q_uses > 0 && !mbar_wait(&c.q_empty, (q_uses - 1) & 1, abort_flag, p.wc, 1)) { ok = false; break; }
+        if (q_uses > 0 && !mbar_wait(&c.q_empty, (q_uses - 1) & 1, abort_flag, p.wc, 1, wi << 12)) { ok = false; break; }
         mbar_expect_tx(&c.q_full, n_qt * L::kTileBytes);
         for (int t = 0; t < n_qt; ++t)
           for (int s = 0; s < L::kSlabs; ++s)
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < n && ok; ++i) {
           for (int kind = 0; kind < 2; ++kind) {
             const int s = ctr % kStages;
-            if (!mbar_wait(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, abort_flag, p.wc, 2)) { ok = false; break; }
+            if (!mbar_wait(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, abort_flag, p.wc, 2, (wi << 12) | i)) { ok = false; break; }
             mbar_expect_tx(&c.kv_full[s], L::kTileBytes);
             uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
             const CUtensorMap* mt = kind == 0 ? &map_k : &map_v;
@@ -308,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int n = kp.n_sel + kp.n_win;
         if (n == 0) continue;
         const int n_qt = it.nq * p.G > 128 ? 2 : 1;
-        if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10)) { ok = false; break; }
+        if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10, wi << 12)) { ok = false; break; }
         ++q_uses;
         tc_fence_after();
         auto issue_qk = [&](int t, int stage) {
@@ -337,18 +339,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         // prologue: S_t(0)
         int sk = ctr % kStages;
-        if (!mbar_wait(&c.kv_full[sk], (ctr / kStages) & 1, abort_flag, p.wc, 11)) { ok = false; break; }
+        if (!mbar_wait(&c.kv_full[sk], (ctr / kStages) & 1, abort_flag, p.wc, 11, wi << 12)) { ok = false; break; }
         ++ctr;
         tc_fence_after();
         for (int t = 0; t < n_qt; ++t) issue_qk(t, sk);
         umma_commit(&c.kv_empty[sk]);
         for (int i = 0; i < n && ok; ++i) {
           const int sv = ctr % kStages;
-          if (!mbar_wait(&c.kv_full[sv], (ctr / kStages) & 1, abort_flag, p.wc, 12)) { ok = false; break; }
+          if (!mbar_wait(&c.kv_full[sv], (ctr / kStages) & 1, abort_flag, p.wc, 12, (wi << 12) | i)) { ok = false; break; }
           ++ctr;
           int sk_next = -1;
           for (int t = 0; t < n_qt; ++t) {
-            if (!mbar_wait(&c.p_full[t], (uses[t] + i) & 1, abort_flag, p.wc, 13)) { ok = false; break; }
+            if (!mbar_wait(&c.p_full[t], (uses[t] + i) & 1, abort_flag, p.wc, 13, (wi << 12) | i)) { ok = false; break; }
             if (i == 0 && items_t[t] > 0 &&
                 !mbar_wait(&c.o_free[t], (items_t[t] - 1) & 1, abort_flag, p.wc, 14)) { ok = false; break; }
             tc_fence_after();
@@ -356,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i + 1 < n) {
               if (sk_next < 0) {
                 sk_next = ctr % kStages;
-                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kStages) & 1, abort_flag, p.wc, 15)) { ok = false; break; }
+                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kStages) & 1, abort_flag, p.wc, 15, (wi << 12) | i)) { ok = false; break; }
                 ++ctr;
                 tc_fence_after();
               }
@@ -387,8 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = tmem + t * 256 + (uint32_t(quad * 32) << 16);
     const uint32_t t_o = t_s + 128;
     uint8_t* p_tile = smem + L::kOffP + t * L::kPBytes;
-    int uses = 0, items_t = 0;
+    int uses = 0, items_t = 0, sm_phase = 0;
     bool ok = true;
+    // bounded replacement for a named barrier over warps 0-7
+    auto softmax_sync = [&]() {
+      mbar_arrive(&c.sm_bar);
+      mbar_wait_warp(&c.sm_bar, sm_phase & 1, abort_flag, p.wc, 30);
+      ++sm_phase;
+    };
     for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
@@ -406,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int* idx_row =
             (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
         for (int i = 0; i < n; ++i) {
-          if (!mbar_wait_warp(&c.s_full[t], (uses + i) & 1, abort_flag, p.wc, 20)) { ok = false; break; }
+          if (!mbar_wait_warp(&c.s_full[t], (uses + i) & 1, abort_flag, p.wc, 20, (wi << 12) | i)) { ok = false; break; }
           tc_fence_after();
           uint32_t u[128];
           tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
@@ -492,8 +500,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           l = l * factor + rs;
           // P buffer and O are free once the previous PV of this tile is done
-          if (i > 0 && !mbar_wait_warp(&c.o_ready[t], (uses + i - 1) & 1, abort_flag, p.wc, 21)) { ok = false; break; }
-          if (rescale && i > 0) {
+          if (i > 0 && !mbar_wait_warp(&c.o_ready[t], (uses + i - 1) & 1, abort_flag, p.wc, 21, (wi << 12) | i)) { ok = false; break; }
+          // tcgen05.ld/st are warp-collective: rescale the whole warp's rows
+          // together (rows that keep their max use factor 1)
+          if (__any_sync(0xffffffffu, rescale && i > 0)) {
+            if (!(rescale && i > 0)) factor = 1.f;
             tc_fence_after();
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
@@ -578,7 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (MODE == kFull && SB > 0) {
         c.lse2[vr] = lse2;
         __threadfence_block();
-        named_bar_sync(1, 256);
+        softmax_sync();
         if (ok && !*abort_flag) {
           const int nblk_item = min(p.nblk, (n * 128) / SB);
           const float* sp = p.spill + size_t(blockIdx.x) * p.nblk * kMaxItemRows;
@@ -604,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        named_bar_sync(1, 256);
+        softmax_sync();
       }
     }
   }

@@ -17,7 +17,7 @@ struct ErrWord {
   int flag;     // 0 = ok; 1 = a bounded wait gave up
   int site;     // which wait gave up (kernel-specific code)
   int block;    // blockIdx.x of the first failure
-  int pad;
+  int ctx;      // kernel-specific context of the failure (e.g. item << 12 | step)
 };
 
 // Wait limit in nanoseconds of %globaltimer; a pipeline stage never takes
@@ -78,29 +78,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// A wait gives up when either clock says the limit has passed: %globaltimer
+// (ns) or the SM cycle counter (at most 2 cycles per ns at B200 clocks), so the
+// bound holds even if one of them were not advancing.
+__device__ __forceinline__ bool wait_expired(unsigned long long t0, long long c0, unsigned long long limit_ns) {
+  return (global_ns() - t0 > limit_ns) || (clock64() - c0 > (long long)(2 * limit_ns));
+}
+
+__device__ __forceinline__ void record_failure(const WaitCtl& wc, int site, int ctx) {
+  if (atomicCAS(&wc.err->flag, 0, 1) == 0) {
+    wc.err->site = site;
+    wc.err->block = blockIdx.x;
+    wc.err->ctx = ctx;
+  }
+}
+
 // Bounded wait on phase `parity`. Returns false (and raises the CTA abort
 // flag) if the barrier did not flip within the time limit, or if another warp
 // of the CTA already aborted. Never spins forever.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                            const WaitCtl& wc, int site) {
+                                            const WaitCtl& wc, int site, int ctx) {
   const unsigned long long t0 = global_ns();
+  const long long c0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (global_ns() - t0 > wc.timeout_ns) {
+    if (wait_expired(t0, c0, wc.timeout_ns)) {
       *abort_flag = 1;
-      if (atomicCAS(&wc.err->flag, 0, 1) == 0) {
-        wc.err->site = site;
-        wc.err->block = blockIdx.x;
-      }
+      record_failure(wc, site, ctx);
       return false;
     }
   }
 }
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          const WaitCtl& wc, int site) {
+                                          const WaitCtl& wc, int site, int ctx = 0) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, abort_flag, wc, site);
+  return mbar_wait_slow(bar, parity, abort_flag, wc, site, ctx);
 }
 
 // Drain wait used at teardown: ignores the abort flag (the point is to let
@@ -108,13 +121,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // still bounded by the time limit.
 __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, const WaitCtl& wc, int site) {
   const unsigned long long t0 = global_ns();
+  const long long c0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > wc.timeout_ns) {
-      if (atomicCAS(&wc.err->flag, 0, 1) == 0) {
-        wc.err->site = site;
-        wc.err->block = blockIdx.x;
-      }
+    if (wait_expired(t0, c0, wc.timeout_ns)) {
+      record_failure(wc, site, 0);
       return false;
     }
   }
@@ -123,9 +134,9 @@ __device__ __noinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, con
 // Warp-uniform bounded wait: lane 0 polls, the verdict is broadcast so every
 // lane of the warp takes the same branch before .sync.aligned tcgen05 ops.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                               const WaitCtl& wc, int site) {
+                                               const WaitCtl& wc, int site, int ctx = 0) {
   int ok = 0;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, wc, site) ? 1 : 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort_flag, wc, site, ctx) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
   return ok != 0;
 }

@@ -104,6 +104,11 @@ HS_API hs_status hs_workspace_init(void* ws, size_t ws_bytes, hs_stream_t stream
  * check, HS_ERR_CUDA if the stream reports an error, else HS_OK. */
 HS_API hs_status hs_check_error(void* ws, hs_stream_t stream);
 
+/* Where the last failure seen by hs_check_error() happened: the wait site
+ * code, the CTA index and a kernel-specific context word (work item << 12 |
+ * pipeline step for the attention kernels). For diagnostics only. */
+HS_API hs_status hs_last_error_detail(int32_t* site, int32_t* block, int32_t* ctx);
+
 /* Static description of a status code. */
 HS_API const char* hs_status_string(hs_status s);
 

@@ -71,10 +71,17 @@ def check_block(w, inp, res, tile_ids=None):
 
 
 def run_and_check(w, seed=None, tile_ids=None):
+    import sys, time
+    t0 = time.time()
     inp = W.make_block_inputs(w, device="cuda", seed=seed)
+    torch.cuda.synchronize()
+    t1 = time.time()
     res = GpuBlock(w, inp).run()
     torch.cuda.synchronize()
+    t2 = time.time()
     check_block(w, inp, res, tile_ids)
+    print(f"[{w.name}] inputs {t1 - t0:.1f}s gpu {t2 - t1:.2f}s oracle check {time.time() - t2:.1f}s",
+          file=sys.stderr, flush=True)
     return inp, res
 
 
