@@ -16,6 +16,7 @@ EXPORTS = [
     "hs_workspace_size", "hs_workspace_init", "hs_check_error", "hs_status_string",
     "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
     "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
+    "hs_full_attn_select_noalloc",
 ]
 
 
@@ -71,6 +72,8 @@ def load():
     lib.hs_sparse_attn_decode.argtypes = [VL, SEL, vp, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
     lib.hs_swa_gated.restype = i32
     lib.hs_swa_gated.argtypes = [VL, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hs_full_attn_select_noalloc.restype = i32
+    lib.hs_full_attn_select_noalloc.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, i32, vp]
     lib.hs_last_error_detail.restype = i32
     lib.hs_last_error_detail.argtypes = [ctypes.POINTER(i32)] * 3
     lib.hs_debug_wait_timeout.restype = i32

@@ -241,6 +241,39 @@ __global__ void debug_wait_kernel(WaitCtl wc) {
 
 }  // namespace
 
+// ----------------------------------------------------------------------------
+// Scratch for hs_full_attn_select_noalloc: callers that cannot allocate device
+// memory get this fixed array instead of a workspace. It is resident on every
+// GPU that loads the library until the process exits. Layout: the 256-byte
+// error header, then the per-CTA block-maximum spill.
+// ----------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // 64 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 128;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached; the error header is
+// zeroed at that point.
+hs_status noalloc_scratch(void** out, cudaStream_t s) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return HS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return HS_ERR_CUDA;
+    if (cudaMemsetAsync(ptr, 0, kHeaderBytes, s) != cudaSuccess) return HS_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return HS_OK;
+}
+}  // namespace
+
 // ============================================================================
 extern "C" {
 
@@ -474,6 +507,71 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
   p.wc = wait_ctl(ws);
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
   return dispatch_attn_d<attn::kSparse, 0>(sh.d, m, p, sc, grid, S(stream));
+}
+
+hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                      const void* v, void* o, float* lse, float* scores, int32_t check,
+                                      hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (!q || !k || !v || !o || !scores) return HS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
+  if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
+  if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
+  if (sel->block == 1) return HS_ERR_UNSUPPORTED;
+  const int T = sel->q_tile, B = sel->block;
+  const int nblk = (sh.max_kv + B - 1) / B;
+  // one CTA's spill is nblk x 256 floats; the fixed scratch bounds the grid
+  const size_t per_cta = size_t(nblk) * attn::kMaxItemRows * sizeof(float);
+  const size_t cap = (kNoAllocScratchBytes - kHeaderBytes) / per_cta;
+  if (cap < 1) return HS_ERR_WORKSPACE;  // sequence longer than the fixed scratch can serve
+  cudaStream_t s = S(stream);
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch, s)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;
+  const int n_tiles = n_tiles_of(vl, T);
+  if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
+    return HS_ERR_CUDA;
+  Maps m;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
+      !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128))
+    return HS_ERR_CUDA;
+  m.kb = m.k;
+  m.vb = m.v;
+  static attn::Sched sc;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!fill_sched(vl, sh, attn::kFull, T, 1, &sc)) return HS_ERR_UNSUPPORTED;
+  attn::Params p{};
+  p.G = sh.G;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.Tq = int(sh.Tq);
+  p.scale_log2 = sh.scale * 1.4426950408889634f;
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.scores = scores;
+  p.spill = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + kHeaderBytes);
+  p.nblk = nblk;
+  p.T = T;
+  p.B = B;
+  p.chunks_per_tile = 1;
+  p.wc = WaitCtl{reinterpret_cast<ErrWord*>(scratch), g_timeout_ns};
+  const int grid = int(std::min<size_t>(cap, size_t(std::min(num_sms(), std::max(1, sc.n_items)))));
+  if ((st = dispatch_full(sh.d, B, m, p, sc, grid, s)) != HS_OK) return st;
+  if (check) {
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HS_ERR_CUDA;
+    ErrWord e{};
+    if (cudaMemcpy(&e, scratch, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return HS_ERR_CUDA;
+    if (e.flag != 0) {
+      last_err = e;
+      if (cudaMemset(scratch, 0, sizeof(ErrWord)) != cudaSuccess) return HS_ERR_CUDA;
+      return HS_ERR_TIMEOUT;
+    }
+  }
+  return HS_OK;
 }
 
 hs_status hs_last_error_detail(int32_t* site, int32_t* block, int32_t* ctx) {

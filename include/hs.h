@@ -211,6 +211,41 @@ HS_API hs_status hs_swa_gated(const hs_varlen* vl, int32_t window,
                        void* ws, size_t ws_bytes, hs_stream_t stream);
 
 /*
+ * hs_full_attn_select_noalloc -- hs_full_attn_select for callers that cannot
+ * allocate device memory. The pages have no counterpart to this entry point.
+ *
+ * Who needs it: code that runs where cudaMalloc (or a caching allocator such
+ * as torch's) is unavailable or forbidden -- e.g. a plugin inside another
+ * runtime that owns all device memory, or a latency-critical path that must
+ * not allocate (cudaMalloc can synchronise the device). Such callers cannot
+ * provide the workspace that hs_full_attn_select needs for its block-maximum
+ * spill, so this variant uses a fixed array inside the library instead.
+ *
+ * Scratch: a file-scope device array of 64 MiB, resident on every GPU that
+ * loads the library until the process exits. The caller still passes inputs
+ * and outputs exactly as for hs_full_attn_select. No call allocates or frees
+ * memory (no cudaMalloc/cudaFree or allocating library routine).
+ * First call per device: looks up the array's device address with the device
+ * current and zeroes its error header (an async memset on `stream`); make that
+ * first call before any stream capture on that device.
+ * Sharing: every call on a device uses the same array and leaves its contents
+ * behind. Calls whose kernels overlap on the GPU (e.g. on two streams without
+ * ordering) race on it and give wrong results; order them.
+ * Limits: block-level selection only (B >= 8). The grid is capped so that
+ * grid * ceil(max_kv / B) KB fits in the array; if a single CTA's share
+ * (ceil(max_kv / B) KB) does not fit -- more than 65535 blocks, i.e. max_kv
+ * above ~4.19M tokens at B = 64 --
+ * the call returns HS_ERR_WORKSPACE before launching. Smaller caps only mean
+ * fewer CTAs, not different results.
+ * check != 0: synchronise `stream` after the launch and return HS_ERR_TIMEOUT
+ * if a device-side bounded wait gave up (details via hs_last_error_detail).
+ */
+HS_API hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel,
+                                             const void* q, const void* k, const void* v,
+                                             void* o, float* lse, float* scores,
+                                             int32_t check, hs_stream_t stream);
+
+/*
  * hs_debug_wait_timeout -- failure-detection self test (no counterpart on the
  * pages). Launches one tiny kernel that waits on a barrier nothing arrives
  * at; its bounded wait gives up after `timeout_ns` (1 .. 2e9), records the
