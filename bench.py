@@ -49,7 +49,16 @@ def parse():
     ap.add_argument("--workload", default="hys_block", choices=list(W.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="scale a single-sequence workload to this many new tokens (profiling cases)")
     return ap.parse_args()
+
+
+def workload(args) -> W.Workload:
+    w = W.WORKLOADS[args.workload]
+    if args.tokens and w.batch == 1:
+        w = W.scaled(w, ctx=(0,), new=(args.tokens,))
+    return w
 
 
 def peaks():
@@ -165,7 +174,7 @@ def bench_ours(args, world, rank, local):
     import torch.distributed as dist
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
-    w = W.WORKLOADS[args.workload]
+    w = workload(args)
     inp, vl, blk, layers = make_runner(w, device, seed=1000 + w.config_index + 7919 * rank)
     stream = torch.cuda.current_stream()
 
@@ -361,7 +370,7 @@ def time_oracle(w, n_tiles_sample=1, repeats=1):
 def bench_reference(args, world, rank):
     if rank != 0:
         return None
-    w = W.WORKLOADS[args.workload]
+    w = workload(args)
     import oracle as O  # noqa: F401
     toks, times = time_oracle(w, 1, repeats=args.warmup + args.steps)
     timed = times[args.warmup:]
@@ -395,7 +404,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     out = bench_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        w = W.WORKLOADS[args.workload]
+        w = workload(args)
         toks, times = time_oracle(w, 1, repeats=1)
         out["cpu_baseline"] = {"value": round(toks / sum(times), 3), "unit": "tokens/s", "cores": oracle_threads(),
                                "kind": "oracle",

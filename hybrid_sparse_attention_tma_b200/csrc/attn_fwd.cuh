@@ -422,9 +422,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&u[64]));
           tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&u[96]));
           tmem_ld_wait();
+          // raw logits (the softmax scale is folded into one FFMA per element below)
           float x[128];
 #pragma unroll
-          for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(u[j]) * p.scale_log2;
+          for (int j = 0; j < 128; ++j) x[j] = __uint_as_float(u[j]);
+          const float cs = p.scale_log2;
           // ---- masks ----
           if (MODE == kFull) {
             const int key0 = i * 128;
@@ -462,67 +464,83 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (key < lo || key > pos) x[j] = -INFINITY;
             }
           }
-          // ---- block maxima for the score by-product (full mode) ----
+          // ---- row max (8 independent chains); block maxima for the scores ----
           float mt = -INFINITY;
           if constexpr (MODE == kFull && SB > 0) {
             constexpr int nb = 128 / SB;
+            constexpr int acc = SB < 8 ? SB : 8;
             float* sp = p.spill + (size_t(blockIdx.x) * p.nblk) * kMaxItemRows + vr;
 #pragma unroll
             for (int b = 0; b < nb; ++b) {
-              float mb = -INFINITY;
+              float a[acc];
 #pragma unroll
-              for (int j = b * SB; j < (b + 1) * SB; ++j) mb = fmaxf(mb, x[j]);
+              for (int e = 0; e < acc; ++e) a[e] = x[b * SB + e];
+#pragma unroll
+              for (int j = acc; j < SB; ++j) a[j % acc] = fmaxf(a[j % acc], x[b * SB + j]);
+#pragma unroll
+              for (int st = acc / 2; st > 0; st >>= 1)
+#pragma unroll
+                for (int e = 0; e < st; ++e) a[e] = fmaxf(a[e], a[e + st]);
               const int gb = i * nb + b;
-              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = mb;
-              mt = fmaxf(mt, mb);
+              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = a[0] * cs;  // log2 units
+              mt = fmaxf(mt, a[0]);
             }
           } else {
+            float a[8];
 #pragma unroll
-            for (int j = 0; j < 128; ++j) mt = fmaxf(mt, x[j]);
+            for (int e = 0; e < 8; ++e) a[e] = x[e];
+#pragma unroll
+            for (int j = 8; j < 128; ++j) a[j & 7] = fmaxf(a[j & 7], x[j]);
+#pragma unroll
+            for (int st = 4; st > 0; st >>= 1)
+#pragma unroll
+              for (int e = 0; e < st; ++e) a[e] = fmaxf(a[e], a[e + st]);
+            mt = a[0];
           }
+          mt *= cs;  // log2 units
           // ---- online softmax with lazy rescaling (exact: O and l share m_used) ----
           float factor = 1.f;
           bool rescale = false;
           if (mt > m_used + 8.f) {
-            const float m_new = mt;
-            factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - m_new);
-            m_used = m_new;
+            factor = (m_used == -INFINITY) ? 0.f : ex2(m_used - mt);
+            m_used = mt;
             rescale = true;
           }
-          const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-          float rs = 0.f;
-          uint32_t pk[64];
+          const float nmu = (m_used == -INFINITY) ? 0.f : -m_used;
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int j = 0; j < 128; j += 2) {
-            const float a = ex2(x[j] - mu), b2 = ex2(x[j + 1] - mu);
-            rs += a + b2;
-            pk[j >> 1] = pack_bf16(a, b2);
+          for (int cc = 0; cc < 16; ++cc) {  // 16 chunks of 8 keys = 16 bytes of P
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int j = cc * 8 + 2 * e;
+              const float a0 = ex2(fmaf(x[j], cs, nmu));
+              const float a1 = ex2(fmaf(x[j + 1], cs, nmu));
+              rs[e] += a0 + a1;
+              pk[e] = pack_bf16(a0, a1);
+            }
+            const int chunk = (cc & 7) ^ (r & 7);
+            *reinterpret_cast<uint4*>(p_tile + (cc >> 3) * kSlabBytes + r * 128 + chunk * 16) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          l = l * factor + rs;
-          // P buffer and O are free once the previous PV of this tile is done
-          if (i > 0 && !mbar_wait_warp(&c.o_ready[t], (uses + i - 1) & 1, abort_flag, p.wc, 21, (wi << 12) | i)) { ok = false; break; }
+          l = l * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+          // S_t(i) was committed after PV_t(i-1), and a commit tracks every
+          // earlier tensor-core op of the issuing thread: PV_t(i-1) is done, so
+          // the P buffer and O may be touched without waiting on o_ready.
           // tcgen05.ld/st are warp-collective: rescale the whole warp's rows
-          // together (rows that keep their max use factor 1)
+          // together (rows that keep their max use factor 1).
           if (__any_sync(0xffffffffu, rescale && i > 0)) {
-            if (!(rescale && i > 0)) factor = 1.f;
-            tc_fence_after();
+            const float f = (rescale && i > 0) ? factor : 1.f;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
               uint32_t ov[32];
               tmem_ld32(t_o + ch * 32, ov);
               tmem_ld_wait();
 #pragma unroll
-              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * factor);
+              for (int j = 0; j < 32; ++j) ov[j] = __float_as_uint(__uint_as_float(ov[j]) * f);
               tmem_st32(t_o + ch * 32, ov);
             }
             tmem_st_wait();
-          }
-#pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {
-            const int slab = cc >> 3;
-            const int chunk = (cc & 7) ^ (r & 7);
-            *reinterpret_cast<uint4*>(p_tile + slab * kSlabBytes + r * 128 + chunk * 16) =
-                make_uint4(pk[cc * 4 + 0], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
           }
           fence_proxy_async_smem();
           tc_fence_before();
