@@ -399,7 +399,10 @@ hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* sc
   p.k = sel->topk;
   const long long rows = (long long)table.n_tiles * sh.Hkv;
   if (rows > (1LL << 31) - 1) return HS_ERR_UNSUPPORTED;
-  topk::topk_kernel<<<unsigned(rows), topk::kThreads, 0, S(stream)>>>(p, table);
+  if (p.nblk <= topk::kStageMax)
+    topk::topk_kernel<256, true><<<unsigned(rows), 256, 0, S(stream)>>>(p, table);
+  else
+    topk::topk_kernel<1024, false><<<unsigned(rows), 1024, 0, S(stream)>>>(p, table);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 

@@ -18,9 +18,11 @@
 // A work item is up to 256 "rows" of one sequence and one KV head g; row
 // r = query * G + head-in-group, so every Q-tile holds whole queries and the
 // group's heads share each K/V tile (GQA/MQA packing into the MMA M dim).
-// TMEM (512 columns): S_t at t*256, O_t at t*256+128 (fp32, 128 lanes).
-// SMEM: Q[2] | K/V ring[3] | P[2] | control. All operand tiles use the
-// 128-byte swizzle (8-row x 128-byte atoms), K-major except V (MN-major).
+// TMEM (512 columns): S_t at t*256, O_t at t*256+128 (fp32, 128 lanes); the
+// softmax writes P_t (bf16, two per column) over the first 64 columns of S_t
+// and the PV MMA reads its A operand from there.
+// SMEM: Q[2] | K/V ring[5] | control. All operand tiles use the 128-byte
+// swizzle (8-row x 128-byte atoms), K-major except V (MN-major).
 #pragma once
 
 #include "hs_common.cuh"
@@ -29,9 +31,15 @@ namespace hs {
 namespace attn {
 
 constexpr int kThreads = 320;
-constexpr int kStages = 3;
+constexpr int kStages = 5;
 constexpr int kSlabBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kMaxItemRows = 256;
+// Of the 4 exp2 pairs in each 8-key chunk of P, how many run on the FMA pipe
+// (polynomial) instead of the MUFU unit; balances the two pipes.
+#ifndef HS_EXP2_POLY_PAIRS
+#define HS_EXP2_POLY_PAIRS 1
+#endif
+constexpr int kPolyPairs = HS_EXP2_POLY_PAIRS;
 
 enum Mode : int { kFull = 0, kSparse = 1 };
 
@@ -90,11 +98,9 @@ template <int D>
 struct Layout {
   static constexpr int kSlabs = D / 64;
   static constexpr int kTileBytes = kSlabs * kSlabBytes;  // Q tile / K tile / V tile
-  static constexpr int kPBytes = 2 * kSlabBytes;          // 128 rows x 128 keys bf16
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffP = kOffKV + kStages * kTileBytes;
-  static constexpr int kOffCtl = kOffP + 2 * kPBytes;
+  static constexpr int kOffCtl = kOffKV + kStages * kTileBytes;
 };
 
 struct Ctl {
@@ -302,7 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t q_base = smem_u32(smem + L::kOffQ);
       const uint32_t kv_base = smem_u32(smem + L::kOffKV);
-      const uint32_t p_base = smem_u32(smem + L::kOffP);
       for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
         const Item it = get_item<MODE>(p, sc, wi);
         if (it.nq <= 0) continue;
@@ -327,14 +332,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto issue_pv = [&](int t, int stage, bool acc) {
           const uint32_t d_tmem = tmem + t * 256 + 128;
-          const uint32_t pa = p_base + t * L::kPBytes;
+          const uint32_t pa = tmem + t * 256;  // P_t over the first 64 columns of S_t
           const uint32_t vb = kv_base + stage * L::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t aoff = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-            umma_bf16(d_tmem, sdesc_sw128(pa + aoff, 16, 1024), sdesc_sw128(vb + kk * 2048, kSlabBytes, 1024),
-                      kIdPV, (acc || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16_ts(d_tmem, pa + kk * 8, sdesc_sw128(vb + kk * 2048, kSlabBytes, 1024), kIdPV,
+                         (acc || kk > 0) ? 1u : 0u);
           umma_commit(&c.o_ready[t]);
         };
         // prologue: S_t(0)
@@ -344,6 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = 0; t < n_qt; ++t) issue_qk(t, sk);
         umma_commit(&c.kv_empty[sk]);
+        if (n == 1) umma_commit(&c.q_empty);  // Q is only read by QK: free it early
         for (int i = 0; i < n && ok; ++i) {
           const int sv = ctr % kStages;
           if (!mbar_wait(&c.kv_full[sv], (ctr / kStages) & 1, abort_flag, p.wc, 12, (wi << 12) | i)) { ok = false; break; }
@@ -368,9 +372,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!ok) break;
           umma_commit(&c.kv_empty[sv]);
           if (sk_next >= 0) umma_commit(&c.kv_empty[sk_next]);
+          if (i + 2 == n) umma_commit(&c.q_empty);  // last QK of the item issued
         }
         if (!ok) break;
-        umma_commit(&c.q_empty);
         for (int t = 0; t < n_qt; ++t) {
           uses[t] += n;
           items_t[t] += 1;
@@ -388,7 +392,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int vr = t * 128 + r;      // row inside the item
     const uint32_t t_s = tmem + t * 256 + (uint32_t(quad * 32) << 16);
     const uint32_t t_o = t_s + 128;
-    uint8_t* p_tile = smem + L::kOffP + t * L::kPBytes;
     int uses = 0, items_t = 0, sm_phase = 0;
     bool ok = true;
     // bounded replacement for a named barrier over warps 0-7
@@ -464,38 +467,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (key < lo || key > pos) x[j] = -INFINITY;
             }
           }
-          // ---- row max (8 independent chains); block maxima for the scores ----
+          // ---- row max; block maxima for the scores ----
           float mt = -INFINITY;
           if constexpr (MODE == kFull && SB > 0) {
             constexpr int nb = 128 / SB;
-            constexpr int acc = SB < 8 ? SB : 8;
             float* sp = p.spill + (size_t(blockIdx.x) * p.nblk) * kMaxItemRows + vr;
+            float mb[nb];
 #pragma unroll
             for (int b = 0; b < nb; ++b) {
-              float a[acc];
-#pragma unroll
-              for (int e = 0; e < acc; ++e) a[e] = x[b * SB + e];
-#pragma unroll
-              for (int j = acc; j < SB; ++j) a[j % acc] = fmaxf(a[j % acc], x[b * SB + j]);
-#pragma unroll
-              for (int st = acc / 2; st > 0; st >>= 1)
-#pragma unroll
-                for (int e = 0; e < st; ++e) a[e] = fmaxf(a[e], a[e + st]);
+              mb[b] = max_n<SB>(x + b * SB);
               const int gb = i * nb + b;
-              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = a[0] * cs;  // log2 units
-              mt = fmaxf(mt, a[0]);
+              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = mb[b] * cs;  // log2 units
             }
+            mt = max_n<nb>(mb);
           } else {
-            float a[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = x[e];
-#pragma unroll
-            for (int j = 8; j < 128; ++j) a[j & 7] = fmaxf(a[j & 7], x[j]);
-#pragma unroll
-            for (int st = 4; st > 0; st >>= 1)
-#pragma unroll
-              for (int e = 0; e < st; ++e) a[e] = fmaxf(a[e], a[e + st]);
-            mt = a[0];
+            mt = max_n<128>(x);
           }
           mt *= cs;  // log2 units
           // ---- online softmax with lazy rescaling (exact: O and l share m_used) ----
@@ -507,22 +493,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             rescale = true;
           }
           const float nmu = (m_used == -INFINITY) ? 0.f : -m_used;
-          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          const uint64_t cs2 = f2(cs, cs), nmu2 = f2(nmu, nmu);
+          uint64_t rs2[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+          // S_t is already in registers: P_t overwrites its first 64 columns
 #pragma unroll
-          for (int cc = 0; cc < 16; ++cc) {  // 16 chunks of 8 keys = 16 bytes of P
-            uint32_t pk[4];
+          for (int cq = 0; cq < 4; ++cq) {  // 4 x 32 keys = 4 x 16 columns of packed bf16
+            uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int j = cc * 8 + 2 * e;
-              const float a0 = ex2(fmaf(x[j], cs, nmu));
-              const float a1 = ex2(fmaf(x[j + 1], cs, nmu));
-              rs[e] += a0 + a1;
+            for (int e = 0; e < 16; ++e) {
+              const int j = cq * 32 + 2 * e;
+              float t0, t1, a0, a1;
+              f2_split(f2_fma(f2(x[j], x[j + 1]), cs2, nmu2), t0, t1);
+              if ((e & 3) >= 4 - kPolyPairs) {
+                exp2_poly_pair(t0, t1, a0, a1);
+              } else {
+                a0 = ex2(t0);
+                a1 = ex2(t1);
+              }
+              rs2[e & 1] = f2_add(rs2[e & 1], f2(a0, a1));
               pk[e] = pack_bf16(a0, a1);
             }
-            const int chunk = (cc & 7) ^ (r & 7);
-            *reinterpret_cast<uint4*>(p_tile + (cc >> 3) * kSlabBytes + r * 128 + chunk * 16) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            tmem_st16(t_s + cq * 16, pk);
           }
+          float rs[4];
+          f2_split(rs2[0], rs[0], rs[1]);
+          f2_split(rs2[1], rs[2], rs[3]);
           l = l * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
           // S_t(i) was committed after PV_t(i-1), and a commit tracks every
           // earlier tensor-core op of the issuing thread: PV_t(i-1) is done, so
@@ -542,12 +537,25 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_st_wait();
           }
-          fence_proxy_async_smem();
+          tmem_st_wait();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&c.p_full[t]);
         }
         // ---- epilogue: O / l, lse ----
+        // the gate's inputs do not depend on this item's result: fetch them
+        // while the last PV is still running
+        // (only the window-only instantiation, which serves the gated SWA call,
+        // carries the gate)
+        constexpr bool kGate = (MODE == kSparse && SB == 0);
+        float sg = 0.f;
+        uint4 osrc[kGate ? D / 8 : 1];
+        if (kGate && p.gamma && valid) {
+          sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
+          const uint4* src = reinterpret_cast<const uint4*>(p.o_other + (size_t(qrow) * p.Hq + h) * D);
+#pragma unroll
+          for (int j = 0; j < D / 8; ++j) osrc[j] = __ldg(src + j);
+        }
         if (ok && mbar_wait_warp(&c.o_ready[t], (uses + n - 1) & 1, abort_flag, p.wc, 22)) {
           tc_fence_after();
           const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -561,12 +569,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               float of[32];
 #pragma unroll
               for (int j = 0; j < 32; ++j) of[j] = __uint_as_float(ov[j]) * inv;
-              if (p.gamma) {
-                const float sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
-                const uint4* src = reinterpret_cast<const uint4*>(p.o_other + (size_t(qrow) * p.Hq + h) * D + ch * 32);
+              if (kGate && p.gamma) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                  const uint4 u4 = __ldg(src + j);
+                  const uint4 u4 = osrc[kGate ? ch * 4 + j : 0];
                   const uint32_t w4[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
                   for (int e = 0; e < 4; ++e) {

@@ -204,6 +204,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16. A (M x K, K-major) sits in
+// tensor memory: row m in lane m, two bf16 per 32-bit column along K, so one
+// K = 16 step spans 8 columns.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -234,6 +246,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 #undef HS_S8
+#define HS_S16(i) "r"(r[i + 0]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), "r"(r[i + 5]), \
+                  "r"(r[i + 6]), "r"(r[i + 7])
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      HS_S16(0), HS_S16(8)
+      : "memory");
+}
+#undef HS_S16
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -272,6 +295,69 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// Packed fp32 pairs (sm_100 f32x2 arithmetic): one instruction for two lanes'
+// worth of FMA / ADD, and a 3-input max.
+__device__ __forceinline__ uint64_t f2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// max over N consecutive register-array entries (N even, fully unrolled)
+template <int N>
+__device__ __forceinline__ float max_n(const float* x) {
+  constexpr int A = N >= 16 ? 4 : (N / 4 > 0 ? N / 4 : 1);
+  float a[A];
+#pragma unroll
+  for (int e = 0; e < A; ++e) a[e] = fmaxf(x[2 * e], x[2 * e + 1]);
+#pragma unroll
+  for (int j = 2 * A; j < N; j += 2) a[(j / 2) % A] = max3f(a[(j / 2) % A], x[j], x[j + 1]);
+  if constexpr (A == 4) return fmaxf(max3f(a[0], a[1], a[2]), a[3]);
+  if constexpr (A == 2) return fmaxf(a[0], a[1]);
+  return a[0];
+}
+
+// 2^x for a pair of floats on the FMA/ALU pipes instead of the MUFU unit.
+// Cody-Waite style range reduction: t = x + 1.5*2^23 rounds x to the nearest
+// integer j (held in t's low mantissa bits), f = x - j in [-1/2, 1/2]; a
+// degree-3 minimax polynomial (relative error 7.5e-5, fitted by
+// csrc/fit_exp2_poly.py) gives 2^f; adding t's bits << 23 to the result's bits
+// adds j to its exponent (the constant part of t's bits shifts out). Inputs are
+// clamped to >= -125 so the exponent never underflows into the sign bit; the
+// result there is ~2e-38, i.e. zero for the softmax.
+__device__ __forceinline__ void exp2_poly_pair(float x0, float x1, float& y0, float& y1) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t t = f2_add(x, f2(kMagic, kMagic));
+  const uint64_t j = f2_add(t, f2(-kMagic, -kMagic));
+  const uint64_t fr = f2_fma(j, f2(-1.f, -1.f), x);
+  uint64_t q = f2_fma(fr, f2(5.517166906e-02f, 5.517166906e-02f), f2(2.426111222e-01f, 2.426111222e-01f));
+  q = f2_fma(q, fr, f2(6.932609855e-01f, 6.932609855e-01f));
+  q = f2_fma(q, fr, f2(9.999280735e-01f, 9.999280735e-01f));
+  float q0, q1, t0, t1;
+  f2_split(q, q0, q1);
+  f2_split(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -13,6 +13,11 @@
 // order with a block-wide prefix scan and keeps every entry > tau plus the
 // first (k - #greater) entries == tau. Walking in index order both breaks
 // ties toward the lower index and emits the result already sorted.
+//
+// Two shapes of the same kernel: rows of up to kStageMax candidates are
+// staged once in shared memory by a 256-thread CTA (block-level selection,
+// short rows, many CTAs per SM); longer rows (token level) are streamed from
+// global memory / L2 by a 1024-thread CTA.
 #pragma once
 
 #include "hs_common.cuh"
@@ -21,8 +26,7 @@
 namespace hs {
 namespace topk {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
+constexpr int kStageMax = 8192;  // candidates staged in shared memory (32 KB)
 
 struct Params {
   const float* scores;  // [n_tiles, Hkv, nblk]
@@ -32,7 +36,9 @@ struct Params {
 };
 
 // Block-wide exclusive scan of one int per thread; returns the total.
+template <int THREADS>
 __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total) {
+  constexpr int kWarps = THREADS / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int x = v;
 #pragma unroll
@@ -43,13 +49,13 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   if (lane == 31) warp_sums[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int s = warp_sums[lane];
+    int s = lane < kWarps ? warp_sums[lane] : 0;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, s, off);
       if (lane >= off) s += y;
     }
-    warp_sums[lane] = s;  // inclusive
+    if (lane < kWarps) warp_sums[lane] = s;  // inclusive
   }
   __syncthreads();
   total = warp_sums[kWarps - 1];
@@ -58,27 +64,29 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
   return base + x - v;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int THREADS, bool STAGED>
+__global__ void __launch_bounds__(THREADS)
     topk_kernel(const Params p, const __grid_constant__ SeqTable st) {
+  constexpr int kWarps = THREADS / 32;
   __shared__ int hist[kWarps][256];
-  __shared__ int total_hist[256];
-  __shared__ int warp_sums[kWarps];
+  __shared__ int warp_sums[32];
   __shared__ uint32_t s_prefix;
   __shared__ int s_krem;
+  __shared__ uint32_t staged[STAGED ? kStageMax : 1];
 
   const int row = blockIdx.x;  // tile * Hkv + g
   const int tile = row / p.Hkv;
   const TileInfo ti = tile_info(st, tile);
   const int last_pos = ti.pos0 + ti.n - 1;
   const int n = min(p.nblk, last_pos / p.B + 1);
-  const uint32_t* keys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
+  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
   int* out = p.idx + size_t(row) * p.k;
   const int k = p.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   if (n <= k) {
     // every candidate is kept
-    for (int j = threadIdx.x; j < k; j += kThreads) out[j] = j < n ? j : -1;
+    for (int j = threadIdx.x; j < k; j += THREADS) out[j] = j < n ? j : -1;
     if (threadIdx.x == 0) p.cnt[row] = n;
     return;
   }
@@ -86,6 +94,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 0) p.cnt[row] = 0;
     return;
   }
+  if constexpr (STAGED) {
+    for (int j = threadIdx.x; j < n; j += THREADS) staged[j] = __ldg(gkeys + j);
+    __syncthreads();
+  }
+  auto key_at = [&](int j) -> uint32_t {
+    if constexpr (STAGED) return staged[j];
+    else return __ldg(gkeys + j);
+  };
 
   // ---- radix select of the k-th largest bit pattern ----
   uint32_t prefix = 0;  // fixed high bits of tau
@@ -95,25 +111,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
     for (int b = lane; b < 256; b += 32) hist[warp][b] = 0;
     __syncwarp();
-    for (int j = threadIdx.x; j < n; j += kThreads) {
-      const uint32_t key = __ldg(keys + j);
+    for (int j = threadIdx.x; j < n; j += THREADS) {
+      const uint32_t key = key_at(j);
       if ((key & hi_mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 0xFF], 1);
     }
     __syncthreads();
-    if (threadIdx.x < 256) {
-      int s = 0;
-      for (int w = 0; w < kWarps; ++w) s += hist[w][threadIdx.x];
-      total_hist[threadIdx.x] = s;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int acc = 0, b = 255;
-      for (; b > 0; --b) {
-        if (acc + total_hist[b] >= krem) break;
-        acc += total_hist[b];
+    // bins reduced across warps; warp 0 finds the bucket holding the krem-th largest
+    if (warp == 0) {
+      int cnt8[8];
+      int tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {  // lane handles bins 255 - (lane*8 + e), descending
+        const int b = 255 - (lane * 8 + e);
+        int s = 0;
+        for (int w = 0; w < kWarps; ++w) s += hist[w][b];
+        cnt8[e] = s;
+        tot += s;
       }
-      s_prefix = prefix | (uint32_t(b) << shift);
-      s_krem = krem - acc;
+      // inclusive prefix of the per-lane totals (descending bin order)
+      int inc = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += y;
+      }
+      const int excl = inc - tot;
+      // the lane whose range crosses krem owns the bucket
+      const bool mine = excl < krem && inc >= krem;
+      if (mine) {
+        int acc = excl, e = 0;
+        for (; e < 7; ++e) {
+          if (acc + cnt8[e] >= krem) break;
+          acc += cnt8[e];
+        }
+        const int b = 255 - (lane * 8 + e);
+        s_prefix = prefix | (uint32_t(b) << shift);
+        s_krem = krem - acc;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -124,20 +158,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- ordered compaction ----
   int out_base = 0, eq_base = 0;
-  for (int j0 = 0; j0 < n; j0 += kThreads) {
+  for (int j0 = 0; j0 < n; j0 += THREADS) {
     const int j = j0 + threadIdx.x;
-    const uint32_t key = j < n ? __ldg(keys + j) : 0u;
+    const uint32_t key = j < n ? key_at(j) : 0u;
     const int is_eq = (j < n && key == tau) ? 1 : 0;
     int eq_total;
-    const int eq_rank = eq_base + block_excl_scan(is_eq, warp_sums, eq_total);
+    const int eq_rank = eq_base + block_excl_scan<THREADS>(is_eq, warp_sums, eq_total);
     const int sel = (j < n) && (key > tau || (is_eq && eq_rank < take_eq));
     int sel_total;
-    const int pos = out_base + block_excl_scan(sel, warp_sums, sel_total);
+    const int pos = out_base + block_excl_scan<THREADS>(sel, warp_sums, sel_total);
     if (sel) out[pos] = j;
     out_base += sel_total;
     eq_base += eq_total;
   }
-  for (int j = out_base + threadIdx.x; j < k; j += kThreads) out[j] = -1;
+  for (int j = out_base + threadIdx.x; j < k; j += THREADS) out[j] = -1;
   if (threadIdx.x == 0) p.cnt[row] = out_base;
 }
 
