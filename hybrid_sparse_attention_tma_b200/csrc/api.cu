@@ -13,6 +13,7 @@
 #include "attn_fwd.cuh"
 #include "hs_common.cuh"
 #include "seqtable.cuh"
+#include "token_scores.cuh"
 #include "topk.cuh"
 
 using namespace hs;
@@ -57,6 +58,21 @@ bool make_map_3d(CUtensorMap* m, const void* base, int d, int mid, long long out
   cuuint32_t box[3] = {64, cuuint32_t(box_mid), cuuint32_t(box_outer)};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 2-D row view of a [T][H][d] bf16 tensor (row = t * H + h) for tile::gather4
+// loads: box {64 columns, 1 row}, 128-byte swizzle.
+bool make_map_rows(CUtensorMap* m, const void* base, int d, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -216,13 +232,30 @@ hs_status dispatch_full(int d, int B, const Maps& m, const attn::Params& p, cons
 
 WaitCtl wait_ctl(void* ws) { return WaitCtl{reinterpret_cast<ErrWord*>(ws), g_timeout_ns}; }
 
-size_t full_ws_bytes(const Shape& sh, const hs_sel* sel) {
+size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
     const size_t nblk = (size_t(sh.max_kv) + sel->block - 1) / sel->block;
     b += size_t(num_sms()) * nblk * attn::kMaxItemRows * sizeof(float);
+  } else {
+    b += align_up(sizeof(int) * (size_t(n_tiles_of(vl, sel->q_tile)) + 1), 256);  // token-score item prefix
   }
   return align_up(b, 256);
+}
+
+// Token-level scores: items are (tile, KV head, 512-key range) up to the
+// tile's last query position.
+long long token_score_items(const hs_varlen* vl, int T, int Hkv) {
+  long long n = 0;
+  for (int b = 0; b < vl->batch; ++b) {
+    const int n_b = vl->cu_q_host[b + 1] - vl->cu_q_host[b];
+    const int c_b = vl->cu_kv_host[b + 1] - vl->cu_kv_host[b] - n_b;
+    for (int i = 0; i * T < n_b; ++i) {
+      const int last = c_b + std::min((i + 1) * T, n_b) - 1;
+      n += (long long)Hkv * (last / (tscore::kBlocks * 128) + 1);
+    }
+  }
+  return n;
 }
 
 // Waits on an mbarrier that nothing ever arrives at; the bounded wait gives up
@@ -237,6 +270,20 @@ __global__ void debug_wait_kernel(WaitCtl wc) {
   }
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, wc, 99);
+}
+
+template <int D>
+hs_status launch_token_scores(const Maps& m, const tscore::Params& p, const SeqTable& st, const int* prefix,
+                              int grid, cudaStream_t s) {
+  auto kern = tscore::token_scores_kernel<D>;
+  constexpr int smem = tscore::smem_bytes<D>() > 116 * 1024 ? tscore::smem_bytes<D>() : 116 * 1024;
+  static bool configured = false;
+  if (!configured) {
+    if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
+    configured = true;
+  }
+  kern<<<grid, tscore::kThreads, smem, s>>>(m.q, m.k, p, st, prefix);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
 }  // namespace
@@ -295,7 +342,7 @@ size_t hs_workspace_size(int op, const hs_varlen* vl, const hs_sel* sel) {
   switch (op) {
     case HS_OP_FULL_ATTN_SELECT:
       if (!sel || check_sel(sel) != HS_OK) return 0;
-      return full_ws_bytes(sh, sel);
+      return full_ws_bytes(vl, sh, sel);
     case HS_OP_TOPK_SELECT:
     case HS_OP_SPARSE_ATTN_PREFILL:
     case HS_OP_SWA_GATED:
@@ -336,10 +383,9 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   if ((st = check_sel(sel)) != HS_OK) return st;
   if (!q || !k || !v || !o || !scores) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < full_ws_bytes(sh, sel)) return HS_ERR_WORKSPACE;
+  if (!ws || ws_bytes < full_ws_bytes(vl, sh, sel)) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
-  if (sel->block == 1) return HS_ERR_UNSUPPORTED;  // token-level scores: second QK pass (not built yet)
   if (sh.Tq == 0) return HS_OK;
   const int T = sel->q_tile, B = sel->block;
   const int n_tiles = n_tiles_of(vl, T);
@@ -374,7 +420,31 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   p.chunks_per_tile = 1;
   p.wc = wait_ctl(ws);
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
-  return dispatch_full(sh.d, B, m, p, sc, grid, s);
+  hs_status rc = dispatch_full(sh.d, B, m, p, sc, grid, s);
+  if (rc != HS_OK || B > 1) return rc;
+  // token level: a second QK pass reduces max(s - lse) per key (see token_scores.cuh)
+  if (!lse) return HS_ERR_INVALID_ARG;
+  SeqTable table;
+  if (!fill_seqtable(vl, T, &table)) return HS_ERR_UNSUPPORTED;
+  const long long items = token_score_items(vl, T, sh.Hkv);
+  if (items > (1LL << 30)) return HS_ERR_UNSUPPORTED;
+  int* prefix = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + kHeaderBytes);
+  tscore::item_prefix_kernel<<<1, 1024, 0, s>>>(table, sh.Hkv, prefix);
+  if (cudaGetLastError() != cudaSuccess) return HS_ERR_CUDA;
+  tscore::Params tp{};
+  tp.lse = lse;
+  tp.scores = scores;
+  tp.G = sh.G;
+  tp.Hq = sh.Hq;
+  tp.Hkv = sh.Hkv;
+  tp.Tq = int(sh.Tq);
+  tp.nblk = nblk;
+  tp.scale_log2 = p.scale_log2;
+  tp.n_items = int(items);
+  tp.wc = p.wc;
+  const int tgrid = int(std::min<long long>(num_sms(), std::max<long long>(1, items)));
+  return sh.d == 64 ? launch_token_scores<64>(m, tp, table, prefix, tgrid, s)
+                    : launch_token_scores<128>(m, tp, table, prefix, tgrid, s);
 }
 
 hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* scores, int32_t* idx, int32_t* cnt,
@@ -418,14 +488,18 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
-  if (sel->block == 1 && sel->topk > 0) return HS_ERR_UNSUPPORTED;  // token gather: not built yet
   if (sh.Tq == 0) return HS_OK;
   const int T = sel->q_tile, B = sel->block;
   Maps m;
   if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
-      !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
-      !make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B))
+      !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128))
     return HS_ERR_CUDA;
+  if (B == 1) {
+    if (!make_map_rows(&m.kb, k, sh.d, sh.Tkv * sh.Hkv) || !make_map_rows(&m.vb, v, sh.d, sh.Tkv * sh.Hkv))
+      return HS_ERR_CUDA;
+  } else if (!make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B)) {
+    return HS_ERR_CUDA;
+  }
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -449,6 +523,7 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   p.wc = wait_ctl(ws);
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
   switch (B) {
+    case 1: return dispatch_attn_d<attn::kSparse, 1>(sh.d, m, p, sc, grid, S(stream));
     case 8: return dispatch_attn_d<attn::kSparse, 8>(sh.d, m, p, sc, grid, S(stream));
     case 16: return dispatch_attn_d<attn::kSparse, 16>(sh.d, m, p, sc, grid, S(stream));
     case 32: return dispatch_attn_d<attn::kSparse, 32>(sh.d, m, p, sc, grid, S(stream));

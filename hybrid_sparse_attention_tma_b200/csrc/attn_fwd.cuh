@@ -275,14 +275,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(dst + sl * kSlabBytes, mt, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
             } else {
               const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
-              constexpr int sbk = SB > 0 ? SB : 128;
-              constexpr int nb = 128 / sbk;
-              for (int bi = 0; bi < nb; ++bi) {
-                const int slot = i * nb + bi;
-                const int blk = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
-                for (int sl = 0; sl < L::kSlabs; ++sl)
-                  tma_load_3d(dst + sl * kSlabBytes + bi * sbk * 128, mb, &c.kv_full[s], sl * 64, it.g,
-                              it.kv0 + blk * sbk);
+              if constexpr (SB == 1) {
+                // token level: gather the tile's 128 selected rows, 4 per TMA op,
+                // from the 2-D row view (row = token * H_kv + kv head); padded
+                // slots re-read the first selected row and are masked
+                for (int r4 = 0; r4 < 128; r4 += 4) {
+                  int rows[4];
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const int slot = i * 128 + r4 + e;
+                    const int key = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
+                    rows[e] = (it.kv0 + key) * p.Hkv + it.g;
+                  }
+                  for (int sl = 0; sl < L::kSlabs; ++sl)
+                    tma_load_2d_gather4(dst + sl * kSlabBytes + r4 * 128, mb, &c.kv_full[s], sl * 64, rows[0],
+                                        rows[1], rows[2], rows[3]);
+                }
+              } else {
+                constexpr int sbk = SB > 0 ? SB : 128;
+                constexpr int nb = 128 / sbk;
+                for (int bi = 0; bi < nb; ++bi) {
+                  const int slot = i * nb + bi;
+                  const int blk = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
+                  for (int sl = 0; sl < L::kSlabs; ++sl)
+                    tma_load_3d(dst + sl * kSlabBytes + bi * sbk * 128, mb, &c.kv_full[s], sl * 64, it.g,
+                                it.kv0 + blk * sbk);
+                }
               }
             }
             last_use[s] = ctr;
@@ -439,7 +457,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (key0 + j > pos) x[j] = -INFINITY;
             }
           } else if (i < kp.n_sel) {
-            if constexpr (SB > 0) {
+            if constexpr (SB == 1) {
+              // selected tokens are ascending: those with key <= pos - w form a
+              // prefix of the tile's slots; find its length by binary search
+              const int lim = pos - p.w;
+              const int s0 = i * 128, s1 = min(kp.cnt, s0 + 128);
+              if (s1 - s0 < 128 || __ldg(idx_row + s1 - 1) > lim) {
+                int lo = s0, hi = s1;  // first slot in [s0, s1) with key > lim
+                while (lo < hi) {
+                  const int mid = (lo + hi) >> 1;
+                  if (__ldg(idx_row + mid) <= lim) lo = mid + 1; else hi = mid;
+                }
+                const int nvis = lo - s0;
+#pragma unroll
+                for (int j = 0; j < 128; ++j)
+                  if (j >= nvis) x[j] = -INFINITY;
+              }
+            } else if constexpr (SB > 1) {
               // selected keys must satisfy key <= pos - w; keys of a block are
               // consecutive, so each block gives one threshold on j % SB
               constexpr int nb = 128 / SB;

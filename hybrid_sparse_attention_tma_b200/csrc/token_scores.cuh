@@ -1,0 +1,342 @@
+// token_scores.cuh -- token-level importance scores of the full layer.
+//
+// score(t, g, j) = max over queries q of tile t, heads h of KV group g with
+// j <= pos(q) of exp(s_{q,h,j} - lse_{q,h}) (token-level selection of
+// HySparse2: the full layer's attention scores drive a top-1024 token choice,
+// HySparse2 release note on airebao.com; the score formula is the reading
+// used throughout this library). lse is final only after the forward pass,
+// so the per-key maximum needs the logits again: this kernel recomputes
+// S^T = K_blk * Q_tile^T with the KEYS on the MMA's M dimension. A thread then
+// owns one key (one TMEM lane) and reduces over the row columns with one
+// FFMA + one MAX per element -- no exponentials, no cross-lane traffic; a
+// single exp2 per (tile, key) at the end.
+//
+// CTA: warp 0-3 reducers (thread = key), warp 4 TMA producer, warp 5 UMMA
+// issuer. A work item is (tile, KV head, 512 keys): its 4 key blocks (128
+// keys each) stay in shared memory while the tile's T*G query rows stream
+// through a 3-stage ring of 128-row chunks (with their lse). TMEM holds one
+// 128 x 128 fp32 accumulator per key block (4 x 128 columns).
+#pragma once
+
+#include "hs_common.cuh"
+#include "seqtable.cuh"
+
+namespace hs {
+namespace tscore {
+
+constexpr int kThreads = 192;
+constexpr int kBlocks = 4;   // key blocks per item
+constexpr int kQStages = 3;
+constexpr int kSlabBytes = 128 * 128;
+
+struct Params {
+  const float* lse;  // [Hq, Tq] natural log (from the forward pass)
+  float* scores;     // [n_tiles, Hkv, nblk] (nblk = max_kv)
+  int G, Hq, Hkv, Tq, nblk;
+  float scale_log2;
+  int n_items;
+  WaitCtl wc;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kTile = (D / 64) * kSlabBytes;  // 128 rows x D bf16
+  static constexpr int kOffK = 0;
+  static constexpr int kOffQ = kBlocks * kTile;
+  static constexpr int kOffLse = kOffQ + kQStages * kTile;
+  static constexpr int kOffCtl = kOffLse + kQStages * 128 * 4;
+};
+
+struct Ctl {
+  uint64_t k_full, k_empty;
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t acc_full[kBlocks], acc_free[kBlocks];
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <int D>
+constexpr int smem_bytes() {
+  return Layout<D>::kOffCtl + int(sizeof(Ctl)) + 1024;
+}
+
+// item -> (tile, g, first key); items are enumerated tile by tile, KV head by
+// KV head, in 512-key ranges up to the tile's last query position.
+struct Item {
+  int tile, g, key0, nkeys;  // keys [key0, key0 + nkeys)
+  TileInfo ti;
+  int nchunks;               // 128-row chunks of the tile (rows = n * G)
+};
+
+__device__ __forceinline__ int ranges_of(const TileInfo& ti) {
+  return (ti.pos0 + ti.n - 1) / (kBlocks * 128) + 1;
+}
+
+// items are laid out tile-major: item = tile_item_base(tile) + g * ranges + r.
+// The prefix of items per tile is computed on the fly by a binary search over
+// tiles using the closed form of ranges per tile inside one sequence.
+__device__ __forceinline__ Item get_item(const SeqTable& st, const Params& p, const int* tile_items_prefix, int w) {
+  int lo = 0, hi = st.n_tiles - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_items_prefix[mid] <= w) lo = mid; else hi = mid - 1;
+  }
+  Item it;
+  it.tile = lo;
+  it.ti = tile_info(st, lo);
+  const int nr = ranges_of(it.ti);
+  const int local = w - tile_items_prefix[lo];
+  it.g = local / nr;
+  const int r = local % nr;
+  it.key0 = r * kBlocks * 128;
+  const int last = it.ti.pos0 + it.ti.n - 1;  // candidate keys are <= last
+  it.nkeys = min(kBlocks * 128, last + 1 - it.key0);
+  it.nchunks = (it.ti.n * p.G + 127) / 128;
+  return it;
+}
+
+// Prefix sums of items per tile (Hkv * 512-key ranges), one CTA of 1024 threads.
+__global__ void __launch_bounds__(1024) item_prefix_kernel(const __grid_constant__ SeqTable st, int Hkv, int* out) {
+  __shared__ int part[1024];
+  const int n = st.n_tiles;
+  const int per = (n + 1023) / 1024;
+  const int t0 = threadIdx.x * per, t1 = min(n, t0 + per);
+  int sum = 0;
+  for (int t = t0; t < t1; ++t) sum += Hkv * ranges_of(tile_info(st, t));
+  part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan (Hillis-Steele)
+    const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+    __syncthreads();
+    part[threadIdx.x] += v;
+    __syncthreads();
+  }
+  int acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0;
+  for (int t = t0; t < t1; ++t) {
+    out[t] = acc;
+    acc += Hkv * ranges_of(tile_info(st, t));
+  }
+  if (threadIdx.x == 1023) out[n] = part[1023];
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    token_scores_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                        const Params p, const __grid_constant__ SeqTable st, const int* __restrict__ tile_items_prefix) {
+  using L = Layout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kOffCtl);
+  float* lse_s = reinterpret_cast<float*>(smem + L::kOffLse);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&c.k_full, 1);
+    mbar_init(&c.k_empty, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&c.q_full[s], 1);
+      mbar_init(&c.q_empty[s], 1 + 4);  // MMA done with Q + each reducer warp done with lse
+    }
+    for (int b = 0; b < kBlocks; ++b) {
+      mbar_init(&c.acc_full[b], 1);
+      mbar_init(&c.acc_free[b], 4);
+    }
+    mbar_init(&c.teardown, 1);
+    c.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&c.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = c.tmem_base;
+  volatile int* abort_flag = &c.abort;
+
+  if (warp == 4) {
+    // ===================== producer: K blocks, Q chunks + their lse =====================
+    int qctr = 0, items = 0;
+    int last_q[kQStages] = {-1, -1, -1};
+    int k_loads = 0;
+    bool ok = true;
+    for (int wi = blockIdx.x; wi < p.n_items && ok; wi += gridDim.x) {
+      const Item it = get_item(st, p, tile_items_prefix, wi);
+      if (lane == 0) {
+        if (items > 0 && !mbar_wait(&c.k_empty, (items - 1) & 1, abort_flag, p.wc, 101, wi << 12)) ok = false;
+        if (ok) {
+          mbar_expect_tx(&c.k_full, kBlocks * L::kTile);
+          for (int b = 0; b < kBlocks; ++b)
+            for (int sl = 0; sl < D / 64; ++sl)
+              tma_load_3d(smem + L::kOffK + b * L::kTile + sl * kSlabBytes, &map_k, &c.k_full, sl * 64, it.g,
+                          it.ti.kv0 + it.key0 + b * 128);
+          ++k_loads;
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      ++items;
+      for (int qc = 0; qc < it.nchunks && ok; ++qc) {
+        const int s = qctr % kQStages;
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&c.q_empty[s], ((qctr / kQStages) & 1) ^ 1, abort_flag, p.wc, 102, (wi << 12) | qc);
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) { ok = false; break; }
+        // lse of the chunk's 128 rows (row = query * G + head-in-group), log2 units
+        const int qpc = 128 / p.G;
+        for (int rr = lane; rr < 128; rr += 32) {
+          const int ql = qc * qpc + rr / p.G;
+          const int h = it.g * p.G + rr % p.G;
+          float v = -INFINITY;
+          if (ql < it.ti.n) v = __ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) * 1.4426950408889634f;
+          lse_s[s * 128 + rr] = v;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(&c.q_full[s], L::kTile);
+          for (int sl = 0; sl < D / 64; ++sl)
+            tma_load_3d(smem + L::kOffQ + s * L::kTile + sl * kSlabBytes, &map_q, &c.q_full[s], sl * 64, it.g * p.G,
+                        it.ti.qrow0 + qc * qpc);
+          last_q[s] = qctr;
+        }
+        ++qctr;
+      }
+    }
+    if (lane == 0 && *abort_flag) {
+      for (int s = 0; s < kQStages; ++s)
+        if (last_q[s] >= 0) mbar_wait_drain(&c.q_full[s], (last_q[s] / kQStages) & 1, p.wc, 190);
+      if (k_loads > 0) mbar_wait_drain(&c.k_full, (k_loads - 1) & 1, p.wc, 191);
+    }
+  } else if (warp == 5) {
+    // ===================== UMMA issuer: S^T[key, row] = K_blk . Q_chunk^T =====================
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16_f32(128, 128, false, false);
+      int qctr = 0, items = 0;
+      int acc_cnt[kBlocks] = {0, 0, 0, 0};
+      bool ok = true;
+      const uint32_t k_base = smem_u32(smem + L::kOffK);
+      const uint32_t q_base = smem_u32(smem + L::kOffQ);
+      for (int wi = blockIdx.x; wi < p.n_items && ok; wi += gridDim.x) {
+        const Item it = get_item(st, p, tile_items_prefix, wi);
+        const int nb = (it.nkeys + 127) / 128;
+        if (!mbar_wait(&c.k_full, items & 1, abort_flag, p.wc, 110, wi << 12)) { ok = false; break; }
+        ++items;
+        for (int qc = 0; qc < it.nchunks && ok; ++qc) {
+          const int s = qctr % kQStages;
+          if (!mbar_wait(&c.q_full[s], (qctr / kQStages) & 1, abort_flag, p.wc, 111, (wi << 12) | qc)) { ok = false; break; }
+          tc_fence_after();
+          for (int b = 0; b < nb; ++b) {
+            if (acc_cnt[b] > 0 &&
+                !mbar_wait(&c.acc_free[b], (acc_cnt[b] - 1) & 1, abort_flag, p.wc, 112, (wi << 12) | qc)) { ok = false; break; }
+            ++acc_cnt[b];
+            tc_fence_after();
+            const uint32_t ka = k_base + b * L::kTile, qb = q_base + s * L::kTile;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
+              umma_bf16(tmem + b * 128, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), kId,
+                        kk > 0 ? 1u : 0u);
+            }
+            umma_commit(&c.acc_full[b]);
+          }
+          if (!ok) break;
+          umma_commit(&c.q_empty[s]);
+          ++qctr;
+        }
+        if (!ok) break;
+        umma_commit(&c.k_empty);
+      }
+      umma_commit(&c.teardown);
+      mbar_wait_drain(&c.teardown, 0, p.wc, 192);
+    }
+  } else {
+    // ===================== reducers: thread = key lane =====================
+    const int kl = warp * 32 + lane;  // key within each 128-key block
+    int qctr = 0;
+    int acc_cnt[kBlocks] = {0, 0, 0, 0};
+    bool ok = true;
+    const float cs = p.scale_log2;
+    for (int wi = blockIdx.x; wi < p.n_items; wi += gridDim.x) {
+      const Item it = get_item(st, p, tile_items_prefix, wi);
+      const int nb = (it.nkeys + 127) / 128;
+      const int qpc = 128 / p.G;
+      float best[kBlocks];
+#pragma unroll
+      for (int b = 0; b < kBlocks; ++b) best[b] = -INFINITY;
+      for (int qc = 0; qc < it.nchunks && ok; ++qc) {
+        const int s = qctr % kQStages;
+        const float* ls = lse_s + s * 128;
+        // acquire the producer's lse writes directly (already complete once any
+        // accumulator of this chunk is ready; the stage cannot move on before
+        // this warp releases it)
+        if (!mbar_wait_warp(&c.q_full[s], (qctr / kQStages) & 1, abort_flag, p.wc, 121, (wi << 12) | qc)) { ok = false; break; }
+        // valid columns of this chunk: rows of queries inside the tile
+        const int c_max = min(128, (it.ti.n - qc * qpc) * p.G);
+        const int pos_first = it.ti.pos0 + qc * qpc;  // position of the chunk's first query
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {
+          if (b >= nb) break;
+          if (!mbar_wait_warp(&c.acc_full[b], acc_cnt[b] & 1, abort_flag, p.wc, 120, (wi << 12) | qc)) { ok = false; break; }
+          ++acc_cnt[b];
+          tc_fence_after();
+          const int key = it.key0 + b * 128 + kl;
+          // causal: column c (query pos_first + c / G) sees key iff c >= G * (key - pos_first)
+          const int c_min = max(0, (key - pos_first) * p.G);
+          const bool full = (c_min == 0) && (c_max == 128);
+          const uint32_t taddr = tmem + b * 128 + (uint32_t(warp * 32) << 16);
+          float m = best[b];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            uint32_t v[32];
+            tmem_ld32(taddr + ch * 32, v);
+            tmem_ld_wait();
+            if (full) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                float a0, a1;
+                f2_split(f2_fma(f2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), f2(cs, cs),
+                                f2(-ls[ch * 32 + e], -ls[ch * 32 + e + 1])),
+                         a0, a1);
+                m = max3f(m, a0, a1);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int col = ch * 32 + e;
+                const float a = fmaf(__uint_as_float(v[e]), cs, -ls[col]);
+                if (col >= c_min && col < c_max) m = fmaxf(m, a);
+              }
+            }
+          }
+          best[b] = m;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.acc_free[b]);
+        }
+        if (!ok) break;
+        // this warp is done with the chunk's lse
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.q_empty[s]);
+        ++qctr;
+      }
+      if (ok) {
+        float* out = p.scores + (size_t(it.tile) * p.Hkv + it.g) * p.nblk;
+#pragma unroll
+        for (int b = 0; b < kBlocks; ++b) {
+          const int key = it.key0 + b * 128 + kl;
+          if (b < nb && key < it.key0 + it.nkeys) out[key] = best[b] > -INFINITY ? ex2(best[b]) : 0.f;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tscore
+}  // namespace hs

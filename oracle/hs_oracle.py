@@ -156,26 +156,38 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, visible: np.nd
 # A1  full causal attention (the full layer) -> O, lse
 # ----------------------------------------------------------------------------
 
+def _row_slots(tiles, compact):
+    """Output row range of each tile: its packed rows, or consecutive slots when
+    only the selected tiles' rows are kept (compact)."""
+    out, r = [], 0
+    for t in tiles:
+        out.append(slice(r, r + t.n) if compact else slice(t.row0, t.row0 + t.n))
+        r += t.n
+    return out, r
+
+
 def full_attention(q, k, v, cu_q, cu_kv, n_kv_heads: int, scale=None, tiles_T: int = 0,
-                   tile_ids: Optional[Sequence[int]] = None):
+                   tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """Causal scaled dot-product attention [techwalker-HySparse; QbitAI-HySparse].
 
     o_{q,h} = sum_{j <= pos(q)} softmax_j(s) v_j,  s = q . k_j / sqrt(d),
     lse_{q,h} = ln sum_{j <= pos(q)} exp(s).
 
     Returns (o [T_q, H_q, d], lse [H_q, T_q]); with ``tile_ids`` (and tiles_T)
-    only those tiles' rows are computed and the rest stay NaN.
+    only those tiles' rows are computed and the rest stay NaN; with
+    ``compact`` the outputs hold only those rows, tile after tile.
     """
     Tq, Hq, d = q.shape
     G = Hq // n_kv_heads
     sc = softmax_scale(d, scale)
-    o = np.full((Tq, Hq, d), np.nan)
-    lse = np.full((Hq, Tq), np.nan)
     T = tiles_T if tiles_T else max(1, max(cu_q[b + 1] - cu_q[b] for b in range(len(cu_q) - 1)))
     tiles = make_tiles(cu_q, cu_kv, T)
     if tile_ids is not None:
         tiles = [tiles[i] for i in tile_ids]
-    for t in tiles:
+    slots, n_out = _row_slots(tiles, compact)
+    o = np.full((n_out if compact else Tq, Hq, d), np.nan)
+    lse = np.full((Hq, n_out if compact else Tq), np.nan)
+    for t, rows_out in zip(tiles, slots):
         rows = slice(t.row0, t.row0 + t.n)
         pos = t.pos0 + np.arange(t.n)
         kk = k[t.kv0:t.kv0 + t.kv_len]
@@ -184,8 +196,8 @@ def full_attention(q, k, v, cu_q, cu_kv, n_kv_heads: int, scale=None, tiles_T: i
         for h in range(Hq):
             g = h // G
             oh, lh = masked_attention(q[rows, h], kk[:, g], vv[:, g], vis, sc)
-            o[rows, h] = oh
-            lse[h, rows] = lh
+            o[rows_out, h] = oh
+            lse[h, rows_out] = lh
     return o, lse
 
 
@@ -194,7 +206,7 @@ def full_attention(q, k, v, cu_q, cu_kv, n_kv_heads: int, scale=None, tiles_T: i
 # ----------------------------------------------------------------------------
 
 def importance_scores(q, k, lse, cu_q, cu_kv, n_kv_heads: int, T: int, B: int, scale=None,
-                      tile_ids: Optional[Sequence[int]] = None):
+                      tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """score(t, g, b) = max over queries q in tile t, heads h of KV group g and
     keys j of block b with j <= pos(q) of exp(s_{q,h,j} - lse_{q,h}).
 
@@ -205,6 +217,8 @@ def importance_scores(q, k, lse, cu_q, cu_kv, n_kv_heads: int, T: int, B: int, s
     candidate of tile t iff b*B <= last position of t; non-candidates are 0.
 
     Returns scores [n_tiles, H_kv, ceil(max_kv/B)] (rows not in tile_ids stay 0).
+    ``lse`` is indexed like full_attention's output (compact rows if compact);
+    with ``compact`` the scores hold only the selected tiles, in order.
     """
     Tq, Hq, d = q.shape
     G = Hq // n_kv_heads
@@ -212,9 +226,11 @@ def importance_scores(q, k, lse, cu_q, cu_kv, n_kv_heads: int, T: int, B: int, s
     tiles = make_tiles(cu_q, cu_kv, T)
     max_kv = max(cu_kv[b + 1] - cu_kv[b] for b in range(len(cu_kv) - 1))
     nblk = (max_kv + B - 1) // B
-    scores = np.zeros((len(tiles), n_kv_heads, nblk))
     sel = tiles if tile_ids is None else [tiles[i] for i in tile_ids]
-    for t in sel:
+    slots, _ = _row_slots(sel, compact)
+    scores = np.zeros((len(sel) if compact else len(tiles), n_kv_heads, nblk))
+    for si, (t, rows_out) in enumerate(zip(sel, slots)):
+        out_i = si if compact else t.index
         n_cand_keys = min(t.kv_len, (t.last_pos // B + 1) * B)
         pos = t.pos0 + np.arange(t.n)
         vis = np.arange(n_cand_keys)[None, :] <= pos[:, None]
@@ -223,12 +239,12 @@ def importance_scores(q, k, lse, cu_q, cu_kv, n_kv_heads: int, T: int, B: int, s
             colmax = np.zeros(n_cand_keys)
             for h in range(g * G, (g + 1) * G):
                 s = (q[t.row0:t.row0 + t.n, h] @ kk.T) * sc
-                p = np.where(vis, np.exp(s - lse[h, t.row0:t.row0 + t.n][:, None]), 0.0)
+                p = np.where(vis, np.exp(s - lse[h, rows_out][:, None]), 0.0)
                 colmax = np.maximum(colmax, p.max(axis=0))
             nb = (n_cand_keys + B - 1) // B
             padded = np.zeros(nb * B)
             padded[:n_cand_keys] = colmax
-            scores[t.index, g, :nb] = padded.reshape(nb, B).max(axis=1)
+            scores[out_i, g, :nb] = padded.reshape(nb, B).max(axis=1)
     return scores
 
 
@@ -242,7 +258,7 @@ def n_candidates(t: Tile, B: int) -> int:
 
 
 def topk_select(scores, cu_q, cu_kv, T: int, B: int, k: int,
-                tile_ids: Optional[Sequence[int]] = None):
+                tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """Keep the k highest-scoring candidate blocks of each (tile, KV head).
 
     Order: score descending, ties to the lower block index (north-star rule;
@@ -250,20 +266,21 @@ def topk_select(scores, cu_q, cu_kv, T: int, B: int, k: int,
     order and padded with -1; cnt = min(k, #candidates).
     Returns (idx int32 [n_tiles, H_kv, k], cnt int32 [n_tiles, H_kv]).
     """
-    n_tiles, Hkv, _ = scores.shape
+    n_rows, Hkv, _ = scores.shape
     tiles = make_tiles(cu_q, cu_kv, T)
-    idx = np.full((n_tiles, Hkv, k), -1, dtype=np.int32)
-    cnt = np.zeros((n_tiles, Hkv), dtype=np.int32)
+    idx = np.full((n_rows, Hkv, k), -1, dtype=np.int32)
+    cnt = np.zeros((n_rows, Hkv), dtype=np.int32)
     sel = tiles if tile_ids is None else [tiles[i] for i in tile_ids]
-    for t in sel:
+    for si, t in enumerate(sel):
+        r = si if compact else t.index   # compact: scores/idx rows follow tile_ids
         nc = n_candidates(t, B)
         ids = np.arange(nc)
         for g in range(Hkv):
-            s = scores[t.index, g, :nc]
+            s = scores[r, g, :nc]
             order = np.lexsort((ids, -s))          # primary: -score, secondary: index
             keep = np.sort(order[:min(k, nc)])
-            idx[t.index, g, :len(keep)] = keep
-            cnt[t.index, g] = len(keep)
+            idx[r, g, :len(keep)] = keep
+            cnt[r, g] = len(keep)
     return idx, cnt
 
 
@@ -293,7 +310,7 @@ def sparse_visible(t: Tile, sel_blocks: Sequence[int], B: int, w: int) -> np.nda
 
 
 def sparse_attention(q, k, v, idx, cnt, cu_q, cu_kv, T: int, B: int, w: int, scale=None,
-                     tile_ids: Optional[Sequence[int]] = None):
+                     tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """Sparse layer: softmax attention of this layer's Q over V_q, using the
     full layer's K/V and its tile indices (KV Reuse) [QbitAI-HySparse;
     airebao-HySparse2]. Returns (o [T_q, H_q, d], lse [H_q, T_q]); tiles not in
@@ -304,21 +321,23 @@ def sparse_attention(q, k, v, idx, cnt, cu_q, cu_kv, T: int, B: int, w: int, sca
     Hkv = k.shape[1]
     G = Hq // Hkv
     sc = softmax_scale(d, scale)
-    o = np.full((Tq, Hq, d), np.nan)
-    lse = np.full((Hq, Tq), np.nan)
     tiles = make_tiles(cu_q, cu_kv, T)
     sel = tiles if tile_ids is None else [tiles[i] for i in tile_ids]
-    for t in sel:
+    slots, n_out = _row_slots(sel, compact)
+    o = np.full((n_out if compact else Tq, Hq, d), np.nan)
+    lse = np.full((Hq, n_out if compact else Tq), np.nan)
+    for si, (t, rows_out) in enumerate(zip(sel, slots)):
         rows = slice(t.row0, t.row0 + t.n)
+        r = si if compact else t.index   # compact: idx/cnt rows follow tile_ids
         for g in range(Hkv):
-            vis = sparse_visible(t, idx[t.index, g, :cnt[t.index, g]], B, w)
+            vis = sparse_visible(t, idx[r, g, :cnt[r, g]], B, w)
             cols = np.nonzero(vis.any(axis=0))[0]
             kk = k[t.kv0 + cols, g]
             vv = v[t.kv0 + cols, g]
             for h in range(g * G, (g + 1) * G):
                 oh, lh = masked_attention(q[rows, h], kk, vv, vis[:, cols], sc)
-                o[rows, h] = oh
-                lse[h, rows] = lh
+                o[rows_out, h] = oh
+                lse[h, rows_out] = lh
     return o, lse
 
 
@@ -327,7 +346,7 @@ def sparse_attention(q, k, v, idx, cnt, cu_q, cu_kv, T: int, B: int, w: int, sca
 # ----------------------------------------------------------------------------
 
 def swa_attention(q, k_swa, v_swa, cu_q, cu_kv, window: int, scale=None,
-                  row_ids: Optional[Sequence[int]] = None):
+                  row_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """SWA branch of a HySparse sparse layer: same Q, its own small KV cache,
     keys [max(0, q - window + 1), q] (window 128 by default)
     [QbitAI-HySparse; techwalker-HySparse]. Returns (o, lse [H_q, T_q])."""
@@ -335,12 +354,14 @@ def swa_attention(q, k_swa, v_swa, cu_q, cu_kv, window: int, scale=None,
     Hkv = k_swa.shape[1]
     G = Hq // Hkv
     sc = softmax_scale(d, scale)
-    o = np.full((Tq, Hq, d), np.nan)
-    lse = np.full((Hq, Tq), np.nan)
-    rows_all = range(Tq) if row_ids is None else row_ids
-    seq_of = np.searchsorted(np.asarray(cu_q), np.arange(Tq), side="right") - 1
-    for r in rows_all:
-        b = seq_of[r]
+    rows_all = list(range(Tq)) if row_ids is None else list(row_ids)
+    n_out = len(rows_all) if compact else Tq
+    o = np.full((n_out, Hq, d), np.nan)
+    lse = np.full((Hq, n_out), np.nan)
+    cu = np.asarray(cu_q)
+    for ri, r in enumerate(rows_all):
+        ro = ri if compact else r
+        b = int(np.searchsorted(cu, r, side="right") - 1)
         n_b = cu_q[b + 1] - cu_q[b]
         kv_b = cu_kv[b + 1] - cu_kv[b]
         p = kv_b - n_b + (r - cu_q[b])
@@ -350,8 +371,8 @@ def swa_attention(q, k_swa, v_swa, cu_q, cu_kv, window: int, scale=None,
         for h in range(Hq):
             g = h // G
             oh, lh = masked_attention(q[r:r + 1, h], k_swa[keys, g], v_swa[keys, g], vis, sc)
-            o[r, h] = oh[0]
-            lse[h, r] = lh[0]
+            o[ro, h] = oh[0]
+            lse[h, ro] = lh[0]
     return o, lse
 
 

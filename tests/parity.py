@@ -28,6 +28,25 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").double().numpy()
 
 
+class LazyF64:
+    """Read-only float64 view of a (device) tensor: only the slices the oracle
+    asks for are copied to the host and decoded."""
+
+    def __init__(self, t: torch.Tensor):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def _conv(self, i):
+        if isinstance(i, np.ndarray):
+            return torch.from_numpy(i.astype(np.int64)).to(self.t.device)
+        if isinstance(i, tuple):
+            return tuple(self._conv(x) for x in i)
+        return i
+
+    def __getitem__(self, idx):
+        return f64(self.t[self._conv(idx)])
+
+
 def assert_close_out(got: np.ndarray, want: np.ndarray, max_tol=O_MAX, mean_tol=O_MEAN, what="o"):
     assert got.shape == want.shape, (got.shape, want.shape)
     assert np.isfinite(want).all() and np.isfinite(got).all(), what

@@ -12,62 +12,60 @@ import torch
 import oracle as O
 from oracle.block import tile_rows
 import workloads as W
-from tests.parity import (GpuBlock, f64, assert_close_out, assert_close_lse, assert_scores_close,
+from tests.parity import (GpuBlock, LazyF64, f64, assert_close_out, assert_close_lse, assert_scores_close,
                           assert_indices_match)
 
 pytestmark = pytest.mark.gpu
 
 
-def _layers_f64(inp, rows=None):
-    out = []
-    for L in inp.layers:
-        d = {"q": f64(L.q)}
-        if L.k_swa is not None:
-            d.update(k_swa=f64(L.k_swa), v_swa=f64(L.v_swa), gamma=f64(L.gamma))
-        out.append(d)
-    return out
-
-
 def check_block(w, inp, res, tile_ids=None):
-    """Compare every step of one hybrid block on the given tiles (None = all)."""
+    """Compare every step of one hybrid block on the given tiles (None = all).
+
+    The oracle runs in compact mode: only the sampled tiles' rows are computed
+    and compared, so full-size workloads stay cheap on the host."""
     cu_q, cu_kv = w.cu_q(), w.cu_kv()
     T, B = w.q_tile, w.block
-    q, k, v = f64(inp.q), f64(inp.k), f64(inp.v)
+    dev = inp.q.device
+    q, k, v = LazyF64(inp.q), LazyF64(inp.k), LazyF64(inp.v)
     tiles = O.make_tiles(cu_q, cu_kv, T)
     tids = list(range(len(tiles))) if tile_ids is None else list(tile_ids)
     rows = tile_rows(cu_q, cu_kv, T, tids)
+    rows_t = torch.tensor(rows, device=dev, dtype=torch.long)
+    tids_t = torch.tensor(tids, device=dev, dtype=torch.long)
     # A1: full attention
-    o_o, lse_o = O.full_attention(q, k, v, cu_q, cu_kv, w.n_kv_heads, tiles_T=T, tile_ids=tids)
-    o_g, lse_g = f64(res["o_full"]), f64(res["lse_full"])
-    assert_close_out(o_g[rows], o_o[rows], what="full o")
-    assert_close_lse(lse_g[:, rows], lse_o[:, rows], what="full lse")
+    o_o, lse_o = O.full_attention(q, k, v, cu_q, cu_kv, w.n_kv_heads, tiles_T=T, tile_ids=tids, compact=True)
+    assert_close_out(f64(res["o_full"][rows_t]), o_o, what="full o")
+    assert_close_lse(f64(res["lse_full"][:, rows_t]), lse_o, what="full lse")
     # A2: scores
-    sc_o = O.importance_scores(q, k, lse_o, cu_q, cu_kv, w.n_kv_heads, T, B, tile_ids=tids)
-    sc_g = f64(res["scores"])
-    assert_scores_close(sc_g, sc_o, tids)
+    sc_o = O.importance_scores(q, k, lse_o, cu_q, cu_kv, w.n_kv_heads, T, B, tile_ids=tids, compact=True)
+    sc_g = f64(res["scores"][tids_t])
+    assert_scores_close(sc_g, sc_o, range(len(tids)))
     # A3: top-k -- exact on the GPU's own scores, tie band against the oracle's
-    idx_g, cnt_g = res["idx"].cpu().numpy(), res["cnt"].cpu().numpy()
-    idx_x, cnt_x = O.topk_select(sc_g, cu_q, cu_kv, T, B, w.topk, tile_ids=tids)
-    kk = max(w.topk, 1)
-    for t in tids:
-        assert (cnt_g[t] == cnt_x[t]).all()
-        assert (idx_g[t, :, :w.topk] == idx_x[t]).all(), f"top-k of GPU scores differs in tile {t}"
-    idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids)
-    assert_indices_match(idx_g[:, :, :w.topk], cnt_g, sc_o, idx_o, cnt_o, tids, kk)
+    idx_g = res["idx"][tids_t].cpu().numpy()[:, :, :w.topk]
+    cnt_g = res["cnt"][tids_t].cpu().numpy()
+    idx_x, cnt_x = O.topk_select(sc_g, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True)
+    assert (cnt_g == cnt_x).all(), "cnt of GPU scores differs"
+    assert (idx_g == idx_x).all(), "top-k of GPU scores differs"
+    idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True)
+    assert_indices_match(idx_g, cnt_g, sc_o, idx_o, cnt_o, range(len(tids)), max(w.topk, 1))
     # A4 / A5: sparse layers, fed the GPU's (checked) indices
-    for li, (L, Lg) in enumerate(zip(_layers_f64(inp), res["layers"])):
-        o_sp, lse_sp = O.sparse_attention(L["q"], k, v, idx_g[:, :, :w.topk], cnt_g, cu_q, cu_kv, T, B,
-                                          w.window, tile_ids=tids)
-        assert_close_out(f64(Lg["o_sparse"])[rows], o_sp[rows], what=f"layer {li} sparse o")
-        assert_close_lse(f64(Lg["lse_sparse"])[:, rows], lse_sp[:, rows], what=f"layer {li} sparse lse")
+    for li, (L, Lg) in enumerate(zip(inp.layers, res["layers"])):
+        ql = LazyF64(L.q)
+        o_sp, lse_sp = O.sparse_attention(ql, k, v, idx_g, cnt_g, cu_q, cu_kv, T, B, w.window, tile_ids=tids,
+                                          compact=True)
+        o_sp_g = f64(Lg["o_sparse"][rows_t])
+        assert_close_out(o_sp_g, o_sp, what=f"layer {li} sparse o")
+        assert_close_lse(f64(Lg["lse_sparse"][:, rows_t]), lse_sp, what=f"layer {li} sparse lse")
         if w.swa_window > 0:
-            o_swa, _ = O.swa_attention(L["q"], L["k_swa"], L["v_swa"], cu_q, cu_kv, w.swa_window, row_ids=rows)
+            o_swa, _ = O.swa_attention(ql, LazyF64(L.k_swa), LazyF64(L.v_swa), cu_q, cu_kv, w.swa_window,
+                                       row_ids=rows, compact=True)
+            gamma = f64(L.gamma[rows_t])
             # gate applied to the GPU's bf16 sparse output (the call's actual input)
-            o_gate = O.gated_merge(L["gamma"], f64(Lg["o_sparse"]), o_swa)
-            assert_close_out(f64(Lg["o"])[rows], o_gate[rows], what=f"layer {li} gated o")
+            o_gate = O.gated_merge(gamma, o_sp_g, o_swa)
+            o_l = f64(Lg["o"][rows_t])
+            assert_close_out(o_l, o_gate, what=f"layer {li} gated o")
             # and the whole chain against the oracle's own sparse output
-            o_chain = O.gated_merge(L["gamma"], o_sp, o_swa)
-            assert_close_out(f64(Lg["o"])[rows], o_chain[rows], what=f"layer {li} chain o")
+            assert_close_out(o_l, O.gated_merge(gamma, o_sp, o_swa), what=f"layer {li} chain o")
 
 
 def run_and_check(w, seed=None, tile_ids=None):
@@ -108,6 +106,12 @@ VARIANTS = {
     # G = 128 (two queries per M tile)
     "g128": W.Workload("v6", ctx=(60,), new=(9,), n_q_heads=128, n_kv_heads=1, head_dim=128, q_tile=4,
                        block=8, topk=4, window=8, n_sparse=1),
+    # token level (B = 1): MQA 32 heads, window 32, chunked + ragged
+    "tok_mqa32": W.Workload("v8", ctx=(0, 700), new=(300, 180), n_q_heads=32, n_kv_heads=1, head_dim=128,
+                            q_tile=16, block=1, topk=96, window=32, n_sparse=1, needle_rate=0.02),
+    # token level, GQA 4, d = 64, k larger than some tiles' candidates
+    "tok_gqa4_d64": W.Workload("v9", ctx=(40,), new=(400,), n_q_heads=8, n_kv_heads=2, head_dim=64, q_tile=64,
+                               block=1, topk=200, window=16, n_sparse=1),
     # SWA + gate branch at small size
     "swa_gate": W.Workload("v7", ctx=(0, 100), new=(300, 200), n_q_heads=8, n_kv_heads=2, head_dim=128,
                            q_tile=64, block=64, topk=2, window=0, n_sparse=2, swa_window=128),
@@ -140,6 +144,29 @@ def test_hys_block_full_size_sampled_tiles():
     rng = np.random.default_rng(11)
     tiles = sorted({0, n_t - 1, *rng.choice(n_t, size=2, replace=False).tolist()})
     run_and_check(w, tile_ids=tiles)
+
+
+def test_hys2_token_full_size_sampled_tiles():
+    """HySparse2 token-level prefill at full size (65536 tokens, 64/1 heads,
+    d=128, top-1024 + forced 128, tile 64), 11 sparse layers, sampled tiles."""
+    w = W.WORKLOADS["hys2_prefill"]
+    n_t = w.n_tiles()
+    rng = np.random.default_rng(12)
+    tiles = sorted({0, n_t - 1, *rng.choice(n_t, size=1, replace=False).tolist()})
+    run_and_check(w, tile_ids=tiles)
+
+
+def test_agentic_chunked_full_size_sampled_tiles():
+    """Agentic ragged chunked prefill at full size (contexts 262144/131072/65536/
+    16384 + chunks 8192/4096/8192/2048, 64/1 heads, top-1024 + forced 128),
+    sampled tiles from every sequence."""
+    w = W.WORKLOADS["agentic"]
+    tiles = O.make_tiles(w.cu_q(), w.cu_kv(), w.q_tile)
+    first = {}
+    for t in tiles:
+        first.setdefault(t.seq, []).append(t.index)
+    pick = sorted({first[0][-1], first[1][0], first[2][len(first[2]) // 2], first[3][-1]})
+    run_and_check(w, tile_ids=pick)
 
 
 def test_bounded_wait_timeout_reports_and_context_survives():
