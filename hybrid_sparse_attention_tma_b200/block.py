@@ -12,7 +12,8 @@ from typing import List, Optional
 
 import torch
 
-from . import Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, swa_gated
+from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
+               swa_gated, HS_KV_BF16, HS_KV_FP8_E4M3)
 
 
 @dataclass
@@ -32,6 +33,10 @@ class HybridBlock:
         self.ws = Workspace(device)
         self.device = device
         self._bufs = {}
+        # one query per sequence with single-token tiles: the sparse layers use
+        # the split-K decode path
+        self.decode = q_tile == 1 and block == 1 and all(
+            b - a == 1 for a, b in zip(vl.cu_q_list, vl.cu_q_list[1:]))
 
     def _buf(self, name, shape, dtype):
         t = self._bufs.get(name)
@@ -40,12 +45,13 @@ class HybridBlock:
             self._bufs[name] = t
         return t
 
-    def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False):
+    def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False, fp8_kv=None):
         """Returns dict(o_full, lse_full, scores, idx, cnt, layers=[{o_sparse, lse_sparse, o}]).
 
         With keep_all=False, output buffers are reused across calls (no
         allocation in steady state) and only the last layer's tensors are
-        guaranteed distinct."""
+        guaranteed distinct. fp8_kv = (k_codes, v_codes, k_scale, v_scale) makes the
+        sparse decode layers read an FP8-e4m3 copy of the KV cache."""
         vl, sel = self.vl, self.sel
         Tq, Hq, d = q.shape
         nblk = (vl.max_kv + sel.block - 1) // sel.block
@@ -62,7 +68,16 @@ class HybridBlock:
             tag = str(i) if keep_all else str(i % 2)
             o_sp = self._buf("o_sp" + tag, (Tq, Hq, d), torch.bfloat16)
             lse_sp = self._buf("lse_sp" + tag, (Hq, Tq), torch.float32)
-            sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream)
+            if self.decode:
+                if fp8_kv is not None:
+                    kq, vq, ks, vs = fp8_kv
+                    sparse_attn_decode(vl, sel, L.q, kq, vq, idx, cnt, ks, vs, HS_KV_FP8_E4M3, o=o_sp, lse=lse_sp,
+                                       ws=self.ws, stream=stream)
+                else:
+                    sparse_attn_decode(vl, sel, L.q, k, v, idx, cnt, kv_dtype=HS_KV_BF16, o=o_sp, lse=lse_sp,
+                                       ws=self.ws, stream=stream)
+            else:
+                sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream)
             if self.swa_window > 0:
                 o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
                 swa_gated(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, ws=self.ws,

@@ -13,6 +13,7 @@
 #include "attn_fwd.cuh"
 #include "hs_common.cuh"
 #include "seqtable.cuh"
+#include "decode.cuh"
 #include "token_scores.cuh"
 #include "topk.cuh"
 
@@ -232,7 +233,11 @@ hs_status dispatch_full(int d, int B, const Maps& m, const attn::Params& p, cons
 
 WaitCtl wait_ctl(void* ws) { return WaitCtl{reinterpret_cast<ErrWord*>(ws), g_timeout_ns}; }
 
+size_t full_decode_ws_bytes(const Shape& sh);
+bool is_decode(const hs_varlen* vl, const hs_sel* sel);
+
 size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
+  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= dec::kHeads) return full_decode_ws_bytes(sh);
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
     const size_t nblk = (size_t(sh.max_kv) + sel->block - 1) / sel->block;
@@ -241,6 +246,38 @@ size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
     b += align_up(sizeof(int) * (size_t(n_tiles_of(vl, sel->q_tile)) + 1), 256);  // token-score item prefix
   }
   return align_up(b, 256);
+}
+
+// Decode: one new query per sequence, selection tile 1, token level.
+bool is_decode(const hs_varlen* vl, const hs_sel* sel) {
+  if (sel->q_tile != 1 || sel->block != 1) return false;
+  for (int b = 0; b < vl->batch; ++b)
+    if (vl->cu_q_host[b + 1] - vl->cu_q_host[b] != 1) return false;
+  return true;
+}
+
+int full_decode_splits(const Shape& sh) {
+  const int bg = sh.batch * sh.Hkv;
+  int n = (4 * num_sms() + bg - 1) / bg;
+  const int cap = std::max(1, (sh.max_kv + dec::kFullChunk - 1) / dec::kFullChunk);
+  return std::max(1, std::min(n, cap));
+}
+
+size_t full_decode_ws_bytes(const Shape& sh) {
+  const size_t bg = size_t(sh.batch) * sh.Hkv;
+  const size_t ns = full_decode_splits(sh);
+  return align_up(kHeaderBytes + bg * ns * dec::kHeads * 2 * 4, 256) + align_up(bg * dec::kHeads * 4, 256) +
+         align_up(bg * ns * dec::kHeads * 128 * 4, 256);
+}
+
+int sparse_decode_chunks(const hs_sel* sel) {
+  return std::max(1, (sel->topk + sel->window + dec::kChunk - 1) / dec::kChunk);
+}
+
+size_t sparse_decode_ws_bytes(const Shape& sh, const hs_sel* sel) {
+  const size_t bg = size_t(sh.batch) * sh.Hkv;
+  const size_t nc = sparse_decode_chunks(sel);
+  return align_up(kHeaderBytes + bg * nc * dec::kHeads * 128 * 4, 256) + align_up(bg * nc * dec::kHeads * 2 * 4, 256);
 }
 
 // Token-level scores: items are (tile, KV head, 512-key range) up to the
@@ -348,7 +385,8 @@ size_t hs_workspace_size(int op, const hs_varlen* vl, const hs_sel* sel) {
     case HS_OP_SWA_GATED:
       return kHeaderBytes;
     case HS_OP_SPARSE_ATTN_DECODE:
-      return kHeaderBytes;
+      if (!sel || check_sel(sel) != HS_OK) return 0;
+      return sparse_decode_ws_bytes(sh, sel);
     default:
       return 0;
   }
@@ -393,6 +431,54 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   cudaStream_t s = S(stream);
   if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
     return HS_ERR_CUDA;
+  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= dec::kHeads) {
+    // one query per sequence: exact two-pass split-K over each sequence's keys
+    const int bg = sh.batch * sh.Hkv;
+    const int ns = full_decode_splits(sh);
+    dec::FullParams fp{};
+    fp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    fp.k = reinterpret_cast<const __nv_bfloat16*>(k);
+    fp.v = reinterpret_cast<const __nv_bfloat16*>(v);
+    fp.cu_kv = vl->cu_kv;
+    fp.Hq = sh.Hq;
+    fp.Hkv = sh.Hkv;
+    fp.G = sh.G;
+    fp.n_split = ns;
+    fp.max_kv = sh.max_kv;
+    fp.scale_log2 = sh.scale * 1.4426950408889634f;
+    char* w = reinterpret_cast<char*>(ws);
+    fp.part_ml = reinterpret_cast<float*>(w + kHeaderBytes);
+    char* after_ml = w + align_up(kHeaderBytes + size_t(bg) * ns * dec::kHeads * 2 * 4, 256);
+    fp.lse2 = reinterpret_cast<float*>(after_ml);
+    fp.part_o = reinterpret_cast<float*>(after_ml + align_up(size_t(bg) * dec::kHeads * 4, 256));
+    fp.scores = scores;
+    fp.nblk = nblk;
+    static bool configured = false;
+    if (!configured) {
+      if (set_smem(dec::full_decode_kernel<false>, dec::full_smem_bytes<false>()) != cudaSuccess ||
+          set_smem(dec::full_decode_kernel<true>, dec::full_smem_bytes<true>()) != cudaSuccess)
+        return HS_ERR_CUDA;
+      configured = true;
+    }
+    const dim3 grid(ns, bg);
+    dec::full_decode_kernel<false><<<grid, dec::kThreads, dec::full_smem_bytes<false>(), s>>>(fp);
+    dec::lse_combine_kernel<<<bg, dec::kHeads, 0, s>>>(fp.part_ml, ns, fp.lse2);
+    dec::full_decode_kernel<true><<<grid, dec::kThreads, dec::full_smem_bytes<true>(), s>>>(fp);
+    dec::CombineParams cp{};
+    cp.part_o = fp.part_o;
+    cp.part_ml = fp.part_ml;
+    cp.n_chunks = ns;
+    cp.Hq = sh.Hq;
+    cp.Hkv = sh.Hkv;
+    cp.G = sh.G;
+    cp.Tq = int(sh.Tq);
+    cp.normalised = true;
+    cp.lse2_in = fp.lse2;
+    cp.o = reinterpret_cast<__nv_bfloat16*>(o);
+    cp.lse = lse;
+    dec::combine_kernel<<<bg, 512, 0, s>>>(cp);
+    return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+  }
 
   Maps m;
   if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
@@ -533,10 +619,72 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   }
 }
 
-hs_status hs_sparse_attn_decode(const hs_varlen*, const hs_sel*, const void*, hs_kv_dtype, const void*, const void*,
-                                const float*, const float*, const int32_t*, const int32_t*, int32_t, void*, float*,
-                                void*, size_t, hs_stream_t) {
-  return HS_ERR_UNSUPPORTED;
+hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const void* q, hs_kv_dtype kv_dtype,
+                                const void* k, const void* v, const float* k_scale, const float* v_scale,
+                                const int32_t* idx, const int32_t* cnt, int32_t split_k, void* o, float* lse,
+                                void* ws, size_t ws_bytes, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (!is_decode(vl, sel)) return HS_ERR_INVALID_ARG;  // one query per sequence, q_tile = block = 1
+  if (sh.d != 128 || sh.G > dec::kHeads) return HS_ERR_UNSUPPORTED;
+  if (kv_dtype != HS_KV_BF16 && kv_dtype != HS_KV_FP8_E4M3) return HS_ERR_INVALID_ARG;
+  const bool fp8 = kv_dtype == HS_KV_FP8_E4M3;
+  if (!q || !k || !v || !o || (sel->topk > 0 && (!idx || !cnt)) || (fp8 && (!k_scale || !v_scale)))
+    return HS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
+  if (split_k < 0) return HS_ERR_INVALID_ARG;
+  if (sel->topk + sel->window == 0) return HS_ERR_INVALID_ARG;  // empty visible set
+  if (!ws || ws_bytes < sparse_decode_ws_bytes(sh, sel)) return HS_ERR_WORKSPACE;
+  const int bg = sh.batch * sh.Hkv;
+  const int nc = sparse_decode_chunks(sel);  // 128 keys per chunk; split_k only caps it
+  if (split_k > 0 && split_k < nc) return HS_ERR_UNSUPPORTED;
+  cudaStream_t s = S(stream);
+  dec::SparseParams p{};
+  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  p.k = k;
+  p.v = v;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.idx = idx;
+  p.cnt = sel->topk > 0 ? cnt : nullptr;
+  p.cu_kv = vl->cu_kv;
+  p.topk = sel->topk;
+  p.w = sel->window;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.G = sh.G;
+  p.n_chunks = nc;
+  p.scale_log2 = sh.scale * 1.4426950408889634f;
+  char* w = reinterpret_cast<char*>(ws);
+  p.part_o = reinterpret_cast<float*>(w + kHeaderBytes);
+  p.part_ml = reinterpret_cast<float*>(w + align_up(kHeaderBytes + size_t(bg) * nc * dec::kHeads * 128 * 4, 256));
+  static bool configured = false;
+  if (!configured) {
+    if (set_smem(dec::sparse_decode_kernel<false>, dec::sparse_smem_bytes<false>()) != cudaSuccess ||
+        set_smem(dec::sparse_decode_kernel<true>, dec::sparse_smem_bytes<true>()) != cudaSuccess)
+      return HS_ERR_CUDA;
+    configured = true;
+  }
+  const dim3 grid(nc, bg);
+  if (fp8)
+    dec::sparse_decode_kernel<true><<<grid, dec::kThreads, dec::sparse_smem_bytes<true>(), s>>>(p);
+  else
+    dec::sparse_decode_kernel<false><<<grid, dec::kThreads, dec::sparse_smem_bytes<false>(), s>>>(p);
+  dec::CombineParams cp{};
+  cp.part_o = p.part_o;
+  cp.part_ml = p.part_ml;
+  cp.n_chunks = nc;
+  cp.Hq = sh.Hq;
+  cp.Hkv = sh.Hkv;
+  cp.G = sh.G;
+  cp.Tq = int(sh.Tq);
+  cp.normalised = false;
+  cp.o = reinterpret_cast<__nv_bfloat16*>(o);
+  cp.lse = lse;
+  dec::combine_kernel<<<bg, 512, 0, s>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
 hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const void* k_swa, const void* v_swa,

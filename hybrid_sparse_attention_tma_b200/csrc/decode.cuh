@@ -1,0 +1,604 @@
+// decode.cuh -- one new token per sequence: sparse-layer decode (split-K over
+// the selected set plus the forced window, bf16 or FP8-e4m3 KV) and the full
+// layer's decode with its exact token scores.
+//
+// Decode reads each selected K/V row once and is bound by HBM bandwidth; the
+// KV head's G query heads (64 under MQA) share every K/V row, so the math is
+// a small dense contraction done with warp-level bf16 MMAs (4 warps x 16
+// heads): Q stays in registers, K/V rows are gathered with cp.async into
+// XOR-swizzled shared memory, S and O accumulate in registers.
+//
+// Sparse decode (HySparse2 release note: sparse layers reuse the full layer's
+// KV cache and top-k tokens, with the latest 128 forced in; its key-data table
+// sizes an FP8 KV cache): V_q = {j in idx : j <= pos - w} U [pos-w+1, pos],
+// split into 128-key chunks, one CTA per (sequence, KV head, chunk); the
+// chunks' partial (m, l, O) are merged by log-sum-exp. FP8 rows decode as
+// x = scale[token] * e4m3(code): e4m3 -> bf16 is exact, the K scale multiplies
+// the logits and the V scale multiplies P before the PV product.
+//
+// Full-layer decode: causal attention of the new token over all its keys plus
+// token scores score(j) = max_h exp(s_hj - lse_h). The scores need the final
+// lse, so the layer runs in two exact passes: (1) lse per head from split-K
+// (m, l) partials over K; (2) with lse known, P = exp(s - lse) is final: each
+// CTA writes its keys' scores directly and sums P.V into an fp32 partial;
+// a last kernel adds the partials.
+#pragma once
+
+#include "hs_common.cuh"
+
+namespace hs {
+namespace dec {
+
+constexpr int kThreads = 128;  // 4 warps x 16 heads = 64 heads
+constexpr int kHeads = 64;
+constexpr int kChunk = 128;    // keys per sparse-decode CTA
+constexpr int kFullChunk = 64; // keys per pipeline step of the full-layer decode
+
+// ----------------------------------------------------------------------------
+// warp MMA helpers (m16n8k16, bf16 in, fp32 accumulate)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// two e4m3 codes (low byte first) -> bf16x2, exactly (e4m3 values are bf16 values)
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(two));
+  const __half2 hh = *reinterpret_cast<const __half2*>(&h2);
+  const float2 f = __half22float2(hh);
+  return pack_bf16(f.x, f.y);
+}
+
+// Row r of a [rows][128 bf16] tile: 16-byte chunk c lives at chunk c ^ (r & 7)
+__device__ __forceinline__ uint32_t swz(int r, int c) { return uint32_t(r * 256 + ((c ^ (r & 7)) * 16)); }
+
+// ----------------------------------------------------------------------------
+// Shared pieces
+// ----------------------------------------------------------------------------
+struct SparseParams {
+  const __nv_bfloat16* q;  // [batch, Hq, 128]
+  const void* k;           // [T_kv, Hkv, 128] bf16 or e4m3
+  const void* v;
+  const float* k_scale;    // [T_kv, Hkv] (FP8)
+  const float* v_scale;
+  const int* idx;          // [batch, Hkv, topk]
+  const int* cnt;          // [batch, Hkv]
+  const int* cu_kv;        // device prefix sums of kv_b
+  int topk, w, Hq, Hkv, G, n_chunks;
+  float scale_log2;
+  float* part_o;           // [batch*Hkv, n_chunks, 64, 128]
+  float* part_ml;          // [batch*Hkv, n_chunks, 64, 2]  (m, l) in log2 units
+};
+
+// Load the KV head's 64 query rows (G valid, rest zero) into shared memory.
+__device__ __forceinline__ void load_q_tile(uint8_t* sq, const __nv_bfloat16* q, int b, int g, int Hq, int G) {
+  for (int i = threadIdx.x; i < kHeads * 16; i += kThreads) {  // 64 rows x 16 chunks of 16 B
+    const int r = i >> 4, c = i & 15;
+    const bool valid = r < G;
+    const __nv_bfloat16* src = q + (size_t(b) * Hq + g * G + (valid ? r : 0)) * 128 + c * 8;
+    cp_async16(smem_u32(sq) + swz(r, c), src, valid);
+  }
+}
+
+// Q fragments (A operand) of this warp's 16 heads, all 8 k-steps.
+__device__ __forceinline__ void q_fragments(const uint8_t* sq, uint32_t (&qa)[8][4]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int r = warp * 16 + (lane & 15);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int c = ks * 2 + (lane >> 4);
+    ldsm_x4(smem_u32(sq) + swz(r, c), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+  }
+}
+
+// S[16 heads x NK keys] += Q . K^T for keys stored bf16 in a swizzled tile.
+template <int NK>
+__device__ __forceinline__ void qk_bf16(const uint32_t (&qa)[8][4], const uint8_t* sk, float (&s)[NK / 8][4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int nt = 0; nt < NK / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+  for (int np = 0; np < NK / 16; ++np) {  // pairs of 8-key n-tiles
+    const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int c = ks * 2 + ((lane >> 3) & 1);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(smem_u32(sk) + swz(key, c), b0, b1, b2, b3);
+      mma16816(s[2 * np], qa[ks], b0, b1);
+      mma16816(s[2 * np + 1], qa[ks], b2, b3);
+    }
+  }
+}
+
+// Same with FP8 keys: tile [NK][128 bytes], chunk c of 16 B at c ^ (r & 7).
+template <int NK>
+__device__ __forceinline__ void qk_fp8(const uint32_t (&qa)[8][4], const uint8_t* sk, float (&s)[NK / 8][4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int nt = 0; nt < NK / 8; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+    const int key = nt * 8 + (lane >> 2);
+    const uint8_t* row = sk + key * 128;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int k0 = ks * 16 + 2 * (lane & 3);  // this thread's k pair, and k0 + 8
+      const int c0 = k0 >> 4, o0 = k0 & 15;
+      const uint16_t lo = *reinterpret_cast<const uint16_t*>(row + ((c0 ^ (key & 7)) << 4) + o0);
+      const uint16_t hi = *reinterpret_cast<const uint16_t*>(row + ((c0 ^ (key & 7)) << 4) + o0 + 8);
+      mma16816(s[nt], qa[ks], e4m3x2_to_bf16x2(lo), e4m3x2_to_bf16x2(hi));
+    }
+  }
+}
+
+// O[16 heads x 128] += P[16 x NK] . V[NK x 128], V bf16 swizzled.
+template <int NK>
+__device__ __forceinline__ void pv_bf16(const uint32_t (&pa)[NK / 16][4], const uint8_t* sv, float (&o)[16][4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int ks = 0; ks < NK / 16; ++ks) {
+    const int key = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+    for (int dp = 0; dp < 8; ++dp) {  // pairs of 8-wide d tiles
+      const int c = dp * 2 + (lane >> 4);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(smem_u32(sv) + swz(key, c), b0, b1, b2, b3);
+      mma16816(o[2 * dp], pa[ks], b0, b1);
+      mma16816(o[2 * dp + 1], pa[ks], b2, b3);
+    }
+  }
+}
+
+// FP8 V: B(k = key, n = d) pairs come from two rows; decode per element.
+template <int NK>
+__device__ __forceinline__ void pv_fp8(const uint32_t (&pa)[NK / 16][4], const uint8_t* sv, float (&o)[16][4]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int ks = 0; ks < NK / 16; ++ks) {
+    const int kr = ks * 16 + 2 * (lane & 3);  // keys kr, kr+1 (b0) and kr+8, kr+9 (b1)
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int dcol = nt * 8 + (lane >> 2);
+      const int c = dcol >> 4, off = dcol & 15;
+      auto at = [&](int key) -> uint8_t { return sv[key * 128 + ((c ^ (key & 7)) << 4) + off]; };
+      const uint16_t p0 = uint16_t(at(kr)) | (uint16_t(at(kr + 1)) << 8);
+      const uint16_t p1 = uint16_t(at(kr + 8)) | (uint16_t(at(kr + 9)) << 8);
+      mma16816(o[nt], pa[ks], e4m3x2_to_bf16x2(p0), e4m3x2_to_bf16x2(p1));
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// A6: sparse decode, one CTA per (sequence, KV head, 128-key chunk)
+// ----------------------------------------------------------------------------
+template <bool FP8>
+constexpr int sparse_smem_bytes() {
+  return kHeads * 256 + 2 * kChunk * (FP8 ? 128 : 256) + 3 * kChunk * 4 + 1024;
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparseParams p) {
+  constexpr int kRowBytes = FP8 ? 128 : 256;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = base;
+  uint8_t* sk = sq + kHeads * 256;
+  uint8_t* sv = sk + kChunk * kRowBytes;
+  float* sks = reinterpret_cast<float*>(sv + kChunk * kRowBytes);
+  float* svs = sks + kChunk;
+  int* skey = reinterpret_cast<int*>(svs + kChunk);
+
+  const int chunk = blockIdx.x;
+  const int bg = blockIdx.y;  // sequence * Hkv + g
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int kv0 = __ldg(p.cu_kv + b);
+  const int kv_len = __ldg(p.cu_kv + b + 1) - kv0;
+  const int pos = kv_len - 1;  // the new token is the sequence's last position
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // visible set: selected tokens <= pos - w (a prefix of the ascending list), then the window
+  const int* idx = p.idx + size_t(bg) * p.topk;
+  const int cnt = p.cnt ? __ldg(p.cnt + bg) : 0;
+  const int lim = pos - p.w;
+  int lo = 0, hi = cnt;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(idx + mid) <= lim) lo = mid + 1; else hi = mid;
+  }
+  const int n_sel = lo;
+  const int win_lo = max(0, pos - p.w + 1);
+  const int total = n_sel + (pos - win_lo + 1) * (p.w > 0 ? 1 : 0);
+  const int v0 = chunk * kChunk;
+  const int nk = max(0, min(kChunk, total - v0));
+  float* pml = p.part_ml + (size_t(bg) * p.n_chunks + chunk) * kHeads * 2;
+  if (nk == 0) {
+    if (threadIdx.x < kHeads) {
+      pml[2 * threadIdx.x] = -INFINITY;
+      pml[2 * threadIdx.x + 1] = 0.f;
+    }
+    return;
+  }
+  for (int i = threadIdx.x; i < kChunk; i += kThreads) {
+    const int vi = v0 + i;
+    int key = -1;
+    if (i < nk) key = vi < n_sel ? __ldg(idx + vi) : win_lo + (vi - n_sel);
+    skey[i] = key;
+  }
+  __syncthreads();
+  // gather rows (invalid slots read row 0 of the sequence and are masked)
+  load_q_tile(sq, p.q, b, g, p.Hq, p.G);
+  constexpr int kChunks16 = kRowBytes / 16;
+  for (int i = threadIdx.x; i < kChunk * kChunks16; i += kThreads) {
+    const int r = i / kChunks16, c = i % kChunks16;
+    const int key = skey[r] >= 0 ? skey[r] : 0;
+    const size_t row = (size_t(kv0) + key) * p.Hkv + g;
+    const uint8_t* ks = reinterpret_cast<const uint8_t*>(p.k) + row * kRowBytes + c * 16;
+    const uint8_t* vs = reinterpret_cast<const uint8_t*>(p.v) + row * kRowBytes + c * 16;
+    const uint32_t off = FP8 ? uint32_t(r * 128 + ((c ^ (r & 7)) << 4)) : swz(r, c);
+    cp_async16(smem_u32(sk) + off, ks, true);
+    cp_async16(smem_u32(sv) + off, vs, true);
+  }
+  if (FP8) {
+    for (int i = threadIdx.x; i < kChunk; i += kThreads) {
+      const int key = skey[i] >= 0 ? skey[i] : 0;
+      const size_t row = (size_t(kv0) + key) * p.Hkv + g;
+      sks[i] = __ldg(p.k_scale + row);
+      svs[i] = __ldg(p.v_scale + row);
+    }
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+  __syncthreads();
+
+  uint32_t qa[8][4];
+  q_fragments(sq, qa);
+  float s[kChunk / 8][4];
+  if constexpr (FP8) qk_fp8<kChunk>(qa, sk, s);
+  else qk_bf16<kChunk>(qa, sk, s);
+
+  // softmax partial per head row (rows lane/4 and lane/4 + 8 of this warp)
+  const float cs = p.scale_log2;
+  float m[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+  for (int nt = 0; nt < kChunk / 8; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+      float x = s[nt][e] * cs;
+      if (FP8) x *= sks[col];
+      if (col >= nk) x = -INFINITY;
+      s[nt][e] = x;
+      m[e >> 1] = fmaxf(m[e >> 1], x);
+    }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    m[r] = fmaxf(m[r], __shfl_xor_sync(0xffffffffu, m[r], 1));
+    m[r] = fmaxf(m[r], __shfl_xor_sync(0xffffffffu, m[r], 2));
+  }
+  float l[2] = {0.f, 0.f};
+  uint32_t pa[kChunk / 16][4];
+#pragma unroll
+  for (int nt = 0; nt < kChunk / 8; ++nt) {
+    float pe[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      pe[e] = ex2(s[nt][e] - m[e >> 1]);
+      l[e >> 1] += pe[e];
+      if (FP8) pe[e] *= svs[nt * 8 + 2 * (lane & 3) + (e & 1)];
+    }
+    const int ks = nt >> 1, hi8 = nt & 1;
+    pa[ks][0 + 2 * hi8] = pack_bf16(pe[0], pe[1]);
+    pa[ks][1 + 2 * hi8] = pack_bf16(pe[2], pe[3]);
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+    l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+  }
+  float o[16][4];
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  if constexpr (FP8) pv_fp8<kChunk>(pa, sv, o);
+  else pv_bf16<kChunk>(pa, sv, o);
+
+  // partials: unnormalised O and (m, l) per head
+  float* po = p.part_o + (size_t(bg) * p.n_chunks + chunk) * kHeads * 128;
+  const int h0 = warp * 16 + (lane >> 2);
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt) {
+    const int dcol = nt * 8 + 2 * (lane & 3);
+    *reinterpret_cast<float2*>(po + size_t(h0) * 128 + dcol) = make_float2(o[nt][0], o[nt][1]);
+    *reinterpret_cast<float2*>(po + size_t(h0 + 8) * 128 + dcol) = make_float2(o[nt][2], o[nt][3]);
+  }
+  if ((lane & 3) == 0) {
+    pml[2 * h0] = m[0];
+    pml[2 * h0 + 1] = l[0];
+    pml[2 * (h0 + 8)] = m[1];
+    pml[2 * (h0 + 8) + 1] = l[1];
+  }
+}
+
+// Merge chunk partials: one CTA per (sequence, KV head), thread = (head, 16 dims).
+struct CombineParams {
+  const float* part_o;
+  const float* part_ml;
+  int n_chunks, Hq, Hkv, G, Tq;
+  bool normalised;        // partial O already divided by the final l (full-layer pass 2)
+  const float* lse2_in;   // [batch*Hkv, 64] log2 units (normalised case)
+  __nv_bfloat16* o;       // [batch, Hq, 128]
+  float* lse;             // [Hq, Tq] natural log
+};
+
+__global__ void __launch_bounds__(512) combine_kernel(const CombineParams p) {
+  const int bg = blockIdx.x;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int h = threadIdx.x >> 3;     // 0..63
+  const int d0 = (threadIdx.x & 7) * 16;
+  if (h >= p.G) return;
+  const float* ml = p.part_ml + size_t(bg) * p.n_chunks * kHeads * 2;
+  float M = -INFINITY;
+  if (!p.normalised)
+    for (int c = 0; c < p.n_chunks; ++c) M = fmaxf(M, ml[(size_t(c) * kHeads + h) * 2]);
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  float L = 0.f;
+  for (int c = 0; c < p.n_chunks; ++c) {
+    float wgt = 1.f;
+    if (!p.normalised) {
+      const float mc = ml[(size_t(c) * kHeads + h) * 2];
+      if (mc == -INFINITY) continue;
+      wgt = ex2(mc - M);
+      L += wgt * ml[(size_t(c) * kHeads + h) * 2 + 1];
+    }
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((size_t(bg) * p.n_chunks + c) * kHeads + h) * 128 + d0);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float4 v4 = src[e];
+      acc[4 * e + 0] += wgt * v4.x;
+      acc[4 * e + 1] += wgt * v4.y;
+      acc[4 * e + 2] += wgt * v4.z;
+      acc[4 * e + 3] += wgt * v4.w;
+    }
+  }
+  const float inv = p.normalised ? 1.f : (L > 0.f ? 1.f / L : 0.f);
+  const int hq = g * p.G + h;
+  uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(b) * p.Hq + hq) * 128 + d0);
+  dst[0] = make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                      pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+  dst[1] = make_uint4(pack_bf16(acc[8] * inv, acc[9] * inv), pack_bf16(acc[10] * inv, acc[11] * inv),
+                      pack_bf16(acc[12] * inv, acc[13] * inv), pack_bf16(acc[14] * inv, acc[15] * inv));
+  if (d0 == 0 && p.lse) {
+    float lse2;
+    if (p.normalised) lse2 = p.lse2_in[size_t(bg) * kHeads + h];
+    else lse2 = L > 0.f ? M + __log2f(L) : -INFINITY;
+    p.lse[size_t(hq) * p.Tq + b] = lse2 * 0.69314718055994531f;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// A7: full-layer decode -- pass 1 (per-head lse) and pass 2 (P.V + scores)
+// ----------------------------------------------------------------------------
+struct FullParams {
+  const __nv_bfloat16* q;  // [batch, Hq, 128]
+  const __nv_bfloat16* k;  // [T_kv, Hkv, 128]
+  const __nv_bfloat16* v;
+  const int* cu_kv;
+  int Hq, Hkv, G, n_split, max_kv;
+  float scale_log2;
+  float* part_ml;   // pass 1: [batch*Hkv, n_split, 64, 2]
+  float* lse2;      // [batch*Hkv, 64] (written by the lse combine, read by pass 2)
+  float* part_o;    // pass 2: [batch*Hkv, n_split, 64, 128], already normalised
+  float* scores;    // [batch, Hkv, nblk = max_kv]
+  int nblk;
+};
+
+// keys of split s of a sequence with kv_len keys: [s*len, min((s+1)*len, kv_len))
+__device__ __forceinline__ void split_range(int kv_len, int n_split, int s, int& k0, int& k1) {
+  const int per = ((kv_len + n_split - 1) / n_split + kFullChunk - 1) / kFullChunk * kFullChunk;
+  k0 = min(kv_len, s * per);
+  k1 = min(kv_len, k0 + per);
+}
+
+template <bool PASS2>
+constexpr int full_smem_bytes() {
+  return kHeads * 256 + (PASS2 ? 4 : 2) * kFullChunk * 256 + 1024;
+}
+
+template <bool PASS2>
+__global__ void __launch_bounds__(kThreads) full_decode_kernel(const FullParams p) {
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sq = base;
+  uint8_t* sk[2] = {sq + kHeads * 256, sq + kHeads * 256 + kFullChunk * 256};
+  uint8_t* sv[2] = {sk[1] + kFullChunk * 256, sk[1] + 2 * kFullChunk * 256};
+  __shared__ float red[4][kFullChunk];
+  __shared__ float slse[kHeads];
+
+  const int s = blockIdx.x;
+  const int bg = blockIdx.y;
+  const int b = bg / p.Hkv, g = bg % p.Hkv;
+  const int kv0 = __ldg(p.cu_kv + b);
+  const int kv_len = __ldg(p.cu_kv + b + 1) - kv0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int k0, k1;
+  split_range(kv_len, p.n_split, s, k0, k1);
+  const int n_steps = (k1 - k0 + kFullChunk - 1) / kFullChunk;
+
+  if (PASS2 && threadIdx.x < kHeads) slse[threadIdx.x] = p.lse2[size_t(bg) * kHeads + threadIdx.x];
+  load_q_tile(sq, p.q, b, g, p.Hq, p.G);
+  cp_async_commit();
+  auto issue = [&](int step, int buf) {
+    const int kb = k0 + step * kFullChunk;
+    for (int i = threadIdx.x; i < kFullChunk * 16; i += kThreads) {
+      const int r = i >> 4, c = i & 15;
+      const int key = min(kb + r, kv_len - 1);
+      const size_t row = (size_t(kv0) + key) * p.Hkv + g;
+      cp_async16(smem_u32(sk[buf]) + swz(r, c), p.k + row * 128 + c * 8, true);
+      if (PASS2) cp_async16(smem_u32(sv[buf]) + swz(r, c), p.v + row * 128 + c * 8, true);
+    }
+    cp_async_commit();
+  };
+  if (n_steps > 0) issue(0, 0);
+  cp_async_wait<0>();
+  __syncthreads();
+  uint32_t qa[8][4];
+  q_fragments(sq, qa);
+  const float cs = p.scale_log2;
+  const int h0 = warp * 16 + (lane >> 2);
+  float lse_r[2] = {0.f, 0.f};
+  if (PASS2) {
+    lse_r[0] = slse[h0];
+    lse_r[1] = slse[h0 + 8];
+  }
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  float o[PASS2 ? 16 : 1][4];
+#pragma unroll
+  for (int nt = 0; nt < (PASS2 ? 16 : 1); ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  const bool row_valid[2] = {h0 < p.G, h0 + 8 < p.G};
+
+  for (int st = 0; st < n_steps; ++st) {
+    const int buf = st & 1;
+    if (st + 1 < n_steps) issue(st + 1, buf ^ 1);
+    if (st + 1 < n_steps) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();
+    const int kb = k0 + st * kFullChunk;
+    const int nk = min(kFullChunk, k1 - kb);
+    float sacc[kFullChunk / 8][4];
+    qk_bf16<kFullChunk>(qa, sk[buf], sacc);
+    if constexpr (!PASS2) {
+      // running (m, l) per head row
+      float mt[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < kFullChunk / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+          const float x = col < nk ? sacc[nt][e] * cs : -INFINITY;
+          sacc[nt][e] = x;
+          mt[e >> 1] = fmaxf(mt[e >> 1], x);
+        }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mt[r] = fmaxf(mt[r], __shfl_xor_sync(0xffffffffu, mt[r], 1));
+        mt[r] = fmaxf(mt[r], __shfl_xor_sync(0xffffffffu, mt[r], 2));
+        const float mn = fmaxf(m[r], mt[r]);
+        l[r] *= (m[r] == -INFINITY) ? 0.f : ex2(m[r] - mn);
+        m[r] = mn;
+      }
+#pragma unroll
+      for (int nt = 0; nt < kFullChunk / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) l[e >> 1] += ex2(sacc[nt][e] - m[e >> 1]);
+    } else {
+      // exact probabilities: P = exp2(s*c - lse2); token score = max over heads
+      uint32_t pa[kFullChunk / 16][4];
+      float colmax[kFullChunk / 8][2];
+#pragma unroll
+      for (int nt = 0; nt < kFullChunk / 8; ++nt) {
+        float pe[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+          const bool ok = col < nk && row_valid[e >> 1];
+          pe[e] = ok ? ex2(fmaf(sacc[nt][e], cs, -lse_r[e >> 1])) : 0.f;
+        }
+        colmax[nt][0] = fmaxf(pe[0], pe[2]);
+        colmax[nt][1] = fmaxf(pe[1], pe[3]);
+        const int ks = nt >> 1, hi8 = nt & 1;
+        pa[ks][0 + 2 * hi8] = pack_bf16(pe[0], pe[1]);
+        pa[ks][1 + 2 * hi8] = pack_bf16(pe[2], pe[3]);
+      }
+      // max over the warp's 16 heads: lanes sharing lane & 3 hold the same columns
+#pragma unroll
+      for (int nt = 0; nt < kFullChunk / 8; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float v = colmax[nt][e];
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+          v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+          if (lane < 4) red[warp][nt * 8 + 2 * lane + e] = v;
+        }
+      pv_bf16<kFullChunk>(pa, sv[buf], o);
+      __syncthreads();
+      if (threadIdx.x < kFullChunk && threadIdx.x < nk) {
+        const float sc = fmaxf(fmaxf(red[0][threadIdx.x], red[1][threadIdx.x]),
+                               fmaxf(red[2][threadIdx.x], red[3][threadIdx.x]));
+        p.scores[size_t(bg) * p.nblk + kb + threadIdx.x] = sc;
+      }
+    }
+    __syncthreads();  // buffer `buf` is refilled by the next iteration's issue
+  }
+  if constexpr (!PASS2) {
+    // each of the 4 lanes sharing a head row summed a quarter of the columns
+    // (with the same, quad-uniform running max): add them up
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+      l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+    if ((lane & 3) == 0) {
+      float* pml = p.part_ml + (size_t(bg) * p.n_split + s) * kHeads * 2;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        pml[2 * (h0 + 8 * r)] = m[r];
+        pml[2 * (h0 + 8 * r) + 1] = l[r];
+      }
+    }
+  } else {
+    float* po = p.part_o + (size_t(bg) * p.n_split + s) * kHeads * 128;
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      const int dcol = nt * 8 + 2 * (lane & 3);
+      *reinterpret_cast<float2*>(po + size_t(h0) * 128 + dcol) = make_float2(o[nt][0], o[nt][1]);
+      *reinterpret_cast<float2*>(po + size_t(h0 + 8) * 128 + dcol) = make_float2(o[nt][2], o[nt][3]);
+    }
+  }
+}
+
+// lse2 per (sequence, KV head, head) from the pass-1 partials
+__global__ void __launch_bounds__(64) lse_combine_kernel(const float* part_ml, int n_split, float* lse2) {
+  const int bg = blockIdx.x, h = threadIdx.x;
+  const float* ml = part_ml + size_t(bg) * n_split * kHeads * 2;
+  float M = -INFINITY;
+  for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[(size_t(s) * kHeads + h) * 2]);
+  float L = 0.f;
+  for (int s = 0; s < n_split; ++s) {
+    const float m = ml[(size_t(s) * kHeads + h) * 2];
+    if (m > -INFINITY) L += ex2(m - M) * ml[(size_t(s) * kHeads + h) * 2 + 1];
+  }
+  lse2[size_t(bg) * kHeads + h] = L > 0.f ? M + __log2f(L) : -INFINITY;
+}
+
+}  // namespace dec
+}  // namespace hs

@@ -105,5 +105,9 @@ class GpuBlock:
         self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device)
         self.layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
 
-    def run(self, stream=None):
-        return self.block.forward(self.inp.q, self.inp.k, self.inp.v, self.layers, stream=stream, keep_all=True)
+    def run(self, stream=None, fp8=False):
+        fp8_kv = None
+        if fp8:
+            fp8_kv = (self.inp.k_fp8, self.inp.v_fp8, self.inp.k_scale, self.inp.v_scale)
+        return self.block.forward(self.inp.q, self.inp.k, self.inp.v, self.layers, stream=stream, keep_all=True,
+                                  fp8_kv=fp8_kv)

@@ -13,12 +13,28 @@ import oracle as O
 from oracle.block import tile_rows
 import workloads as W
 from tests.parity import (GpuBlock, LazyF64, f64, assert_close_out, assert_close_lse, assert_scores_close,
-                          assert_indices_match)
+                          assert_indices_match, FP8_MAX)
 
 pytestmark = pytest.mark.gpu
 
 
-def check_block(w, inp, res, tile_ids=None):
+class _Dequant:
+    """float64 view of an FP8 KV cache: e4m3 codes times per-token scales."""
+
+    def __init__(self, codes, scale):
+        self.c, self.s = codes, scale
+        self.shape = tuple(codes.shape)
+
+    def __getitem__(self, idx):
+        if isinstance(idx, tuple):
+            idx = tuple(torch.from_numpy(i.astype(np.int64)).to(self.c.device) if isinstance(i, np.ndarray) else i
+                        for i in idx)
+        codes = self.c[idx].cpu().numpy()
+        sc = self.s[idx[:2] if isinstance(idx, tuple) else idx].cpu().numpy()
+        return O.dequant_fp8(codes, sc) if codes.ndim > sc.ndim else O.e4m3_to_f64(codes) * sc
+
+
+def check_block(w, inp, res, tile_ids=None, fp8=False):
     """Compare every step of one hybrid block on the given tiles (None = all).
 
     The oracle runs in compact mode: only the sampled tiles' rows are computed
@@ -48,14 +64,19 @@ def check_block(w, inp, res, tile_ids=None):
     assert (idx_g == idx_x).all(), "top-k of GPU scores differs"
     idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True)
     assert_indices_match(idx_g, cnt_g, sc_o, idx_o, cnt_o, range(len(tids)), max(w.topk, 1))
-    # A4 / A5: sparse layers, fed the GPU's (checked) indices
+    # A4 / A5 / A6: sparse layers, fed the GPU's (checked) indices
+    kd, vd = (_Dequant(inp.k_fp8, inp.k_scale), _Dequant(inp.v_fp8, inp.v_scale)) if fp8 else (k, v)
     for li, (L, Lg) in enumerate(zip(inp.layers, res["layers"])):
         ql = LazyF64(L.q)
-        o_sp, lse_sp = O.sparse_attention(ql, k, v, idx_g, cnt_g, cu_q, cu_kv, T, B, w.window, tile_ids=tids,
+        o_sp, lse_sp = O.sparse_attention(ql, kd, vd, idx_g, cnt_g, cu_q, cu_kv, T, B, w.window, tile_ids=tids,
                                           compact=True)
         o_sp_g = f64(Lg["o_sparse"][rows_t])
         assert_close_out(o_sp_g, o_sp, what=f"layer {li} sparse o")
         assert_close_lse(f64(Lg["lse_sparse"][:, rows_t]), lse_sp, what=f"layer {li} sparse lse")
+        if fp8:  # and against the bf16-KV oracle within the FP8 bound
+            o_bf, _ = O.sparse_attention(ql, k, v, idx_g, cnt_g, cu_q, cu_kv, T, B, w.window, tile_ids=tids,
+                                         compact=True)
+            assert_close_out(o_sp_g, o_bf, max_tol=FP8_MAX, mean_tol=1.0, what=f"layer {li} fp8 vs bf16 KV")
         if w.swa_window > 0:
             o_swa, _ = O.swa_attention(ql, LazyF64(L.k_swa), LazyF64(L.v_swa), cu_q, cu_kv, w.swa_window,
                                        row_ids=rows, compact=True)
@@ -68,16 +89,16 @@ def check_block(w, inp, res, tile_ids=None):
             assert_close_out(o_l, O.gated_merge(gamma, o_sp, o_swa), what=f"layer {li} chain o")
 
 
-def run_and_check(w, seed=None, tile_ids=None):
+def run_and_check(w, seed=None, tile_ids=None, fp8=False):
     import sys, time
     t0 = time.time()
     inp = W.make_block_inputs(w, device="cuda", seed=seed)
     torch.cuda.synchronize()
     t1 = time.time()
-    res = GpuBlock(w, inp).run()
+    res = GpuBlock(w, inp).run(fp8=fp8)
     torch.cuda.synchronize()
     t2 = time.time()
-    check_block(w, inp, res, tile_ids)
+    check_block(w, inp, res, tile_ids, fp8=fp8)
     print(f"[{w.name}] inputs {t1 - t0:.1f}s gpu {t2 - t1:.2f}s oracle check {time.time() - t2:.1f}s",
           file=sys.stderr, flush=True)
     return inp, res
@@ -167,6 +188,31 @@ def test_agentic_chunked_full_size_sampled_tiles():
         first.setdefault(t.seq, []).append(t.index)
     pick = sorted({first[0][-1], first[1][0], first[2][len(first[2]) // 2], first[3][-1]})
     run_and_check(w, tile_ids=pick)
+
+
+DECODE = {
+    # MQA 64 heads, ragged contexts (one not a multiple of anything), k = 64, w = 32
+    "dec_mqa": W.Workload("d1", ctx=(300, 1000, 128, 2000, 63), new=(1,) * 5, n_q_heads=64, n_kv_heads=1,
+                          head_dim=128, q_tile=1, block=1, topk=64, window=32, n_sparse=2),
+    # GQA group 8 (only 8 of the 64 MMA rows valid), several KV heads
+    "dec_gqa8": W.Workload("d2", ctx=(700, 90), new=(1, 1), n_q_heads=32, n_kv_heads=4, head_dim=128,
+                           q_tile=1, block=1, topk=40, window=16, n_sparse=1),
+}
+
+
+@pytest.mark.parametrize("name", list(DECODE))
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_whole(name, fp8):
+    w = DECODE[name].with_(fp8_kv=True)
+    run_and_check(w, seed=5, fp8=fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_full_size_sampled_sequences(fp8):
+    """Token-level decode at full size: 64 sequences x 131072 cached tokens,
+    64/1 heads, top-1024 + forced 128, bf16 and FP8-e4m3 KV (per-token scales)."""
+    w = W.WORKLOADS["decode"].with_(fp8_kv=True, n_sparse=2)
+    run_and_check(w, tile_ids=[0, 17, 63], fp8=fp8)
 
 
 def test_bounded_wait_timeout_reports_and_context_survives():
