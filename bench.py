@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--workload", default="hys_block", choices=list(W.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fp8-kv", action="store_true", help="decode: sparse layers read an FP8-e4m3 KV cache")
     ap.add_argument("--tokens", type=int, default=0,
                     help="scale a single-sequence workload to this many new tokens (profiling cases)")
     return ap.parse_args()
@@ -170,43 +171,99 @@ def make_runner(w, device, seed):
     return inp, vl, blk, layers
 
 
+def visible_counts(w, idx, cnt):
+    """sum over (tile, KV head, query) of |V_q| for the sparse layers, from the
+    selection actually produced (used for the useful-FLOP and byte counts)."""
+    dev = idx.device
+    tiles_pos0, tiles_n = [], []
+    for a, b, ka, kb in zip(w.cu_q()[:-1], w.cu_q()[1:], w.cu_kv()[:-1], w.cu_kv()[1:]):
+        n_b, c_b = b - a, (kb - ka) - (b - a)
+        for i in range(0, n_b, w.q_tile):
+            tiles_pos0.append(c_b + i)
+            tiles_n.append(min(w.q_tile, n_b - i))
+    pos0 = torch.tensor(tiles_pos0, device=dev)
+    ntq = torch.tensor(tiles_n, device=dev)
+    qoff = torch.arange(w.q_tile, device=dev)
+    pos = pos0[:, None] + qoff[None, :]                      # [tiles, T]
+    qvalid = qoff[None, :] < ntq[:, None]
+    k = w.topk
+    total = torch.zeros((), dtype=torch.float64, device=dev)
+    for g in range(w.n_kv_heads):
+        ids = idx[:, g, :k].long()
+        valid = torch.arange(k, device=dev)[None, :] < cnt[:, g, None]
+        lim = pos - w.window                                 # selected keys must be <= pos - w
+        start = ids * w.block                                # block start positions
+        # keys of each selected block that are <= lim: clip(lim - start + 1, 0, B)
+        per = (lim[:, :, None] - start[:, None, :] + 1).clamp(0, w.block)
+        per = per * valid[:, None, :]
+        sel = per.sum(-1)
+        win = torch.minimum(pos + 1, torch.full_like(pos, w.window)) if w.window > 0 else torch.zeros_like(pos)
+        total += ((sel + win) * qvalid).sum().double()
+    return float(total)
+
+
+def swa_pairs(w):
+    tot = 0
+    for c, n in zip(w.ctx, w.new):
+        for p_ in range(c, c + n):
+            tot += min(p_ + 1, w.swa_window)
+    return tot
+
+
 def bench_ours(args, world, rank, local):
     import torch.distributed as dist
+    import hybrid_sparse_attention_tma_b200 as hs
+    from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
+                                                  sparse_attn_decode, swa_gated, HS_KV_BF16, HS_KV_FP8_E4M3)
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
     w = workload(args)
+    if args.fp8_kv:
+        w = w.with_(fp8_kv=True)
     inp, vl, blk, layers = make_runner(w, device, seed=1000 + w.config_index + 7919 * rank)
     stream = torch.cuda.current_stream()
-
-    def step():
-        return blk.forward(inp.q, inp.k, inp.v, layers, stream=stream)
+    fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if args.fp8_kv else None
 
     for _ in range(max(3, args.warmup)):
-        step()
+        blk.forward(inp.q, inp.k, inp.v, layers, stream=stream, fp8_kv=fp8_kv)
     torch.cuda.synchronize()
-    import hybrid_sparse_attention_tma_b200 as hs
     hs.check_error(blk.ws)
 
-    # per-kernel events for the dominant kernel (full attention + select)
-    full_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    from hybrid_sparse_attention_tma_b200 import full_attn_select, topk_select, sparse_attn_prefill, swa_gated
+    kinds = ["full", "topk", "sparse", "swa"]
+    ev = {kd: [] for kd in kinds}
 
-    def step_instrumented(i):
-        sel = blk.sel
-        bufs = blk._bufs
-        full_ev[i][0].record(stream)
-        full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"], bufs["scores"],
-                         ws=blk.ws, stream=stream)
-        full_ev[i][1].record(stream)
-        topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws, stream=stream)
+    def rec(kind, fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ev[kind].append((a, b))
+
+    def step_instrumented():
+        sel, bufs = blk.sel, blk._bufs
+        rec("full", lambda: full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"],
+                                             bufs["scores"], ws=blk.ws, stream=stream))
+        rec("topk", lambda: topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws,
+                                        stream=stream))
         for j, L in enumerate(layers):
             tag = str(j % 2)
-            sparse_attn_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["o_sp" + tag],
-                                bufs["lse_sp" + tag], ws=blk.ws, stream=stream)
+            if blk.decode:
+                if fp8_kv is not None:
+                    rec("sparse", lambda: sparse_attn_decode(vl, sel, L.q, inp.k_fp8, inp.v_fp8, bufs["idx"],
+                                                             bufs["cnt"], inp.k_scale, inp.v_scale, HS_KV_FP8_E4M3,
+                                                             o=bufs["o_sp" + tag], lse=bufs["lse_sp" + tag],
+                                                             ws=blk.ws, stream=stream))
+                else:
+                    rec("sparse", lambda: sparse_attn_decode(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
+                                                             kv_dtype=HS_KV_BF16, o=bufs["o_sp" + tag],
+                                                             lse=bufs["lse_sp" + tag], ws=blk.ws, stream=stream))
+            else:
+                rec("sparse", lambda: sparse_attn_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
+                                                          bufs["o_sp" + tag], bufs["lse_sp" + tag], ws=blk.ws,
+                                                          stream=stream))
             if blk.swa_window > 0:
-                swa_gated(vl, blk.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, bufs["o_sp" + tag],
-                          bufs["o_l" + tag], ws=blk.ws, stream=stream)
+                rec("swa", lambda: swa_gated(vl, blk.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, bufs["o_sp" + tag],
+                                             bufs["o_l" + tag], ws=blk.ws, stream=stream))
 
     if world > 1:
         dist.barrier()
@@ -218,8 +275,8 @@ def bench_ours(args, world, rank, local):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for i in range(args.steps):
-        step_instrumented(i)
+    for _ in range(args.steps):
+        step_instrumented()
     t1.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -227,43 +284,83 @@ def bench_ours(args, world, rank, local):
         dist.barrier()
     hs.check_error(blk.ws)
     ms_total = t0.elapsed_time(t1)
-    full_ms = statistics.mean(a.elapsed_time(b) for a, b in full_ev)
-    vals = torch.tensor([ms_total, full_ms], dtype=torch.float64, device=device)
+    kms = {kd: (sum(a.elapsed_time(b) for a, b in ev[kd]) / len(ev[kd]) if ev[kd] else 0.0) for kd in kinds}
+    vals = torch.tensor([ms_total] + [kms[kd] for kd in kinds], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total, full_ms = vals.tolist()
+    ms_total = vals[0].item()
+    kms = {kd: vals[i + 1].item() for i, kd in enumerate(kinds)}
     ms_step = ms_total / args.steps
     tokens = w.total_q
     value = world * tokens / (ms_step / 1e3)
 
+    # ---- algorithmic work of each kernel launch ----
+    hbm, tf_burst, tf_sust, src = peaks()
+    d, hq, hkv, G = w.head_dim, w.n_q_heads, w.n_kv_heads, w.group
+    kv_bytes = w.total_kv * hkv * d * 2
+    q_bytes = w.total_q * hq * d * 2
+    nblk = (w.max_kv + w.block - 1) // w.block
+    n_tiles = w.n_tiles()
+    vis = visible_counts(w, blk._bufs["idx"], blk._bufs["cnt"])  # sum_q,g |V_q|
+    kernels = {}
+
+    def entry(kind, ms, amount, bound):
+        if ms <= 0:
+            return
+        if bound == "tensor":
+            ach = amount / (ms / 1e3) / 1e12
+            kernels[kind] = {"bound": "tensor", "ms_per_launch": round(ms, 4), "achieved": round(ach, 1),
+                             "unit": "TFLOP/s", "peak": tf_burst, "frac": round(ach / tf_burst, 4),
+                             "algorithmic_flop_per_launch": amount}
+        else:
+            ach = amount / (ms / 1e3) / 1e9
+            kernels[kind] = {"bound": "hbm", "ms_per_launch": round(ms, 4), "achieved": round(ach, 1),
+                             "unit": "GB/s", "peak": hbm, "frac": round(ach / hbm, 4),
+                             "algorithmic_bytes_per_launch": amount}
+
+    if blk.decode:
+        # full-layer decode: every K/V row once, Q, O, lse and the token scores
+        entry("full", kms["full"], kv_bytes * 2 + q_bytes * 2 + n_tiles * hkv * nblk * 4, "hbm")
+        row = d * (1 if args.fp8_kv else 2) + (4 if args.fp8_kv else 0)
+        entry("sparse", kms["sparse"], vis * 2 * row + q_bytes * 2, "hbm")
+    else:
+        entry("full", kms["full"], full_flops(w), "tensor")
+        entry("sparse", kms["sparse"], 4.0 * d * G * vis, "tensor")
+    entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
+    if w.swa_window > 0:
+        entry("swa", kms["swa"], 4.0 * d * hq * swa_pairs(w), "tensor")
+    per_step = {"full": 1, "topk": 1, "sparse": len(layers), "swa": len(layers) if w.swa_window else 0}
+    for kd, e in kernels.items():
+        e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
+    dom = dict(kernels["full"])
+    dom["kernel"] = ("full-layer decode (two split-K passes + combines)" if blk.decode
+                     else "attn_fwd_kernel<d, full, B> (+ token-score pass when B = 1)")
+    dom["traffic"] = traffic_for("attn_fwd_full", args.workload)
+    dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
+
     # ---- e2e through the public API with host buffers ----
     e2e = None
     if not args.no_e2e:
-        e2e = bench_e2e(args, w, inp, vl, blk, layers, device, world)
+        e2e = bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv)
 
-    hbm, tf_burst, tf_sust, src = peaks()
-    flops = full_flops(w)
-    achieved = flops / (full_ms / 1e3) / 1e12
-    roof = {"bound": "tensor", "kernel": "attn_fwd_kernel<128,full,64>", "achieved": round(achieved, 1),
-            "peak": tf_burst, "unit": "TFLOP/s", "frac": round(achieved / tf_burst, 4),
-            "traffic": traffic_for("attn_fwd_full", args.workload),
-            "peak_kind": f"{src} bf16 burst", "algorithmic_flop_per_launch": flops,
-            "ms_per_launch": round(full_ms, 4)}
+    kind = ("decode" if blk.decode else ("HySparse block-level prefill" if w.block > 1 else "HySparse2 token-level prefill"))
+    desc = (f"{w.name}: {kind}, {w.batch}x ctx {list(w.ctx)[:4]} + new {list(w.new)[:4]} tokens, "
+            f"{hq}/{hkv} heads, d={d}, B={w.block}, k={w.topk}, w={w.window}"
+            + (f", SWA {w.swa_window}+gate" if w.swa_window else "")
+            + f", 1 full + {w.n_sparse} sparse" + (", FP8-e4m3 KV in the sparse layers" if args.fp8_kv else ""))
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-           "data": "synthetic (seeded N(0,1) bf16, 1% planted keys)",
-           "config": {"workload": f"{w.name}: HySparse block-level prefill, 1x{w.total_q} tokens, "
-                                  f"{w.n_q_heads}/{w.n_kv_heads} heads, d={w.head_dim}, B={w.block}, "
-                                  f"k={w.topk}, SWA {w.swa_window}+gate, 1 full + {w.n_sparse} sparse",
-                      "tokens_per_step_per_gpu": tokens, "l2": "inputs larger than L2 (~2 GB/step)",
-                      "parallelism": f"independent blocks x{world}"},
-           "roofline": roof, "gpu_launches": blk.launches_per_forward(len(layers)) * args.steps,
+           "data": "synthetic (seeded N(0,1) bf16" + (", planted keys)" if w.needle_rate else ")"),
+           "config": {"workload": desc, "tokens_per_step_per_gpu": tokens,
+                      "l2": "inputs larger than L2", "parallelism": f"independent blocks x{world}"},
+           "roofline": dom, "kernels": kernels,
+           "gpu_launches": blk.launches_per_forward(len(layers)) * args.steps,
            "clocks": clk, "e2e": e2e}
     return out
 
 
-def bench_e2e(args, w, inp, vl, blk, layers, device, world):
+def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
     """Same metric through HybridBlock.forward with the step's inputs copied
     from pinned host memory each step and the last layer's output read back."""
     from hybrid_sparse_attention_tma_b200.block import SparseLayerIn
@@ -296,7 +393,7 @@ def bench_e2e(args, w, inp, vl, blk, layers, device, world):
                 dl.k_swa.copy_(d["k_swa"], non_blocking=True)
                 dl.v_swa.copy_(d["v_swa"], non_blocking=True)
                 dl.gamma.copy_(d["gamma"], non_blocking=True)
-        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream)
+        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream, fp8_kv=fp8_kv)
         out_host.copy_(res["layers"][-1]["o"], non_blocking=True)
 
     for _ in range(3):

@@ -88,5 +88,14 @@ class HybridBlock:
         return {"o_full": o, "lse_full": lse, "scores": scores, "idx": idx, "cnt": cnt, "layers": outs}
 
     def launches_per_forward(self, n_layers: int) -> int:
-        """Kernels of this library launched by one forward (memsets excluded)."""
-        return 2 + n_layers * (2 if self.swa_window > 0 else 1)
+        """Kernels of this library launched by one forward (memsets excluded):
+        full layer 1 (block scores) / 3 (token scores: forward, item prefix,
+        score pass) / 4 (decode: two passes and two combines); top-k 1; each
+        sparse layer 1 (prefill) or 2 (decode: partials + combine), plus 1 for
+        the gated SWA branch."""
+        if self.decode:
+            full = 4
+        else:
+            full = 1 if self.sel.block > 1 else 3
+        sparse = 2 if self.decode else 1
+        return full + 1 + n_layers * (sparse + (1 if self.swa_window > 0 else 0))

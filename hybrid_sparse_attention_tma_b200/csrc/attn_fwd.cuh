@@ -241,79 +241,89 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ===================== TMA producer =====================
-    if (lane == 0) {
-      int ctr = 0;        // K/V ring uses
-      int q_uses = 0;     // Q loads issued
-      int last_use[kStages] = {-1, -1, -1};
-      bool ok = true;
-      for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
-        const Item it = get_item<MODE>(p, sc, wi);
-        if (it.nq <= 0) continue;
-        const KvPlan kp = kv_plan(p, it, MODE);
-        const int n = kp.n_sel + kp.n_win;
-        if (n == 0) continue;
-        const int rows = it.nq * p.G;
-        const int n_qt = rows > 128 ? 2 : 1;
-        if (q_uses > 0 && !mbar_wait(&c.q_empty, (q_uses - 1) & 1, abort_flag, p.wc, 1, wi << 12)) { ok = false; break; }
+    // Lane 0 owns the barriers and issues the tile loads; for token-level
+    // gathers all 32 lanes fetch indices and issue gather4 loads in parallel.
+    int ctr = 0;        // K/V ring uses
+    int q_uses = 0;     // Q loads issued
+    int last_use[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_use[s] = -1;
+    bool ok = true;
+    auto wait0 = [&](uint64_t* bar, uint32_t parity, int site, int ctx) -> bool {
+      int r = 1;
+      if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc, site, ctx) ? 1 : 0;
+      return __shfl_sync(0xffffffffu, r, 0) != 0;
+    };
+    for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
+      const Item it = get_item<MODE>(p, sc, wi);
+      if (it.nq <= 0) continue;
+      const KvPlan kp = kv_plan(p, it, MODE);
+      const int n = kp.n_sel + kp.n_win;
+      if (n == 0) continue;
+      const int rows = it.nq * p.G;
+      const int n_qt = rows > 128 ? 2 : 1;
+      if (q_uses > 0 && !wait0(&c.q_empty, (q_uses - 1) & 1, 1, wi << 12)) { ok = false; break; }
+      if (lane == 0) {
         mbar_expect_tx(&c.q_full, n_qt * L::kTileBytes);
         for (int t = 0; t < n_qt; ++t)
           for (int s = 0; s < L::kSlabs; ++s)
             tma_load_3d(smem + L::kOffQ + t * L::kTileBytes + s * kSlabBytes, &map_q, &c.q_full, s * 64,
                         it.g * p.G, it.qrow0 + t * (128 / p.G));
-        ++q_uses;
-        const int* idx_row = (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
-        for (int i = 0; i < n && ok; ++i) {
-          for (int kind = 0; kind < 2; ++kind) {
-            const int s = ctr % kStages;
-            if (!mbar_wait(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, abort_flag, p.wc, 2, (wi << 12) | i)) { ok = false; break; }
-            mbar_expect_tx(&c.kv_full[s], L::kTileBytes);
-            uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
-            const CUtensorMap* mt = kind == 0 ? &map_k : &map_v;
-            if (MODE == kFull || i >= kp.n_sel) {
-              const int key0 = (MODE == kFull) ? i * 128 : kp.win_lo + (i - kp.n_sel) * 128;
+      }
+      ++q_uses;
+      const int* idx_row = (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
+      for (int i = 0; i < n && ok; ++i) {
+        for (int kind = 0; kind < 2; ++kind) {
+          const int s = ctr % kStages;
+          if (!wait0(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, 2, (wi << 12) | i)) { ok = false; break; }
+          if (lane == 0) mbar_expect_tx(&c.kv_full[s], L::kTileBytes);
+          __syncwarp();
+          uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
+          const CUtensorMap* mt = kind == 0 ? &map_k : &map_v;
+          if (MODE == kFull || i >= kp.n_sel) {
+            const int key0 = (MODE == kFull) ? i * 128 : kp.win_lo + (i - kp.n_sel) * 128;
+            if (lane == 0)
               for (int sl = 0; sl < L::kSlabs; ++sl)
                 tma_load_3d(dst + sl * kSlabBytes, mt, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
-            } else {
-              const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
-              if constexpr (SB == 1) {
-                // token level: gather the tile's 128 selected rows, 4 per TMA op,
-                // from the 2-D row view (row = token * H_kv + kv head); padded
-                // slots re-read the first selected row and are masked
-                for (int r4 = 0; r4 < 128; r4 += 4) {
-                  int rows[4];
+          } else {
+            const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
+            if constexpr (SB == 1) {
+              // token level: lane l gathers selected rows 4l..4l+3 of the tile
+              // from the 2-D row view (row = token * H_kv + kv head); padded
+              // slots re-read the first selected row and are masked
+              const int r4 = lane * 4;
+              int rws[4];
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const int slot = i * 128 + r4 + e;
-                    const int key = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
-                    rows[e] = (it.kv0 + key) * p.Hkv + it.g;
-                  }
-                  for (int sl = 0; sl < L::kSlabs; ++sl)
-                    tma_load_2d_gather4(dst + sl * kSlabBytes + r4 * 128, mb, &c.kv_full[s], sl * 64, rows[0],
-                                        rows[1], rows[2], rows[3]);
-                }
-              } else {
-                constexpr int sbk = SB > 0 ? SB : 128;
-                constexpr int nb = 128 / sbk;
-                for (int bi = 0; bi < nb; ++bi) {
-                  const int slot = i * nb + bi;
-                  const int blk = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
-                  for (int sl = 0; sl < L::kSlabs; ++sl)
-                    tma_load_3d(dst + sl * kSlabBytes + bi * sbk * 128, mb, &c.kv_full[s], sl * 64, it.g,
-                                it.kv0 + blk * sbk);
-                }
+              for (int e = 0; e < 4; ++e) {
+                const int slot = i * 128 + r4 + e;
+                const int key = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
+                rws[e] = (it.kv0 + key) * p.Hkv + it.g;
+              }
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                tma_load_2d_gather4(dst + sl * kSlabBytes + r4 * 128, mb, &c.kv_full[s], sl * 64, rws[0], rws[1],
+                                    rws[2], rws[3]);
+            } else if (lane == 0) {
+              constexpr int sbk = SB > 0 ? SB : 128;
+              constexpr int nb = 128 / sbk;
+              for (int bi = 0; bi < nb; ++bi) {
+                const int slot = i * nb + bi;
+                const int blk = __ldg(idx_row + (slot < kp.cnt ? slot : 0));
+                for (int sl = 0; sl < L::kSlabs; ++sl)
+                  tma_load_3d(dst + sl * kSlabBytes + bi * sbk * 128, mb, &c.kv_full[s], sl * 64, it.g,
+                              it.kv0 + blk * sbk);
               }
             }
-            last_use[s] = ctr;
-            ++ctr;
           }
+          last_use[s] = ctr;
+          ++ctr;
         }
       }
-      // drain: never leave the CTA with TMA writes in flight
-      if (*abort_flag) {
-        for (int s = 0; s < kStages; ++s)
-          if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kStages) & 1, p.wc, 90);
-        if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 91);
-      }
+    }
+    // drain: never leave the CTA with TMA writes in flight
+    if (lane == 0 && *abort_flag) {
+      for (int s = 0; s < kStages; ++s)
+        if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kStages) & 1, p.wc, 90);
+      if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 91);
     }
   } else if (warp == 9) {
     // ===================== UMMA issuer =====================
