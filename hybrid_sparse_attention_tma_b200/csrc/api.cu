@@ -208,7 +208,7 @@ hs_status launch_attn(const Maps& m, const attn::Params& p, const attn::Sched& s
     if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
     configured = true;
   }
-  kern<<<grid, attn::kThreads, smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, p, sc);
+  kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, p, sc);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
@@ -241,7 +241,7 @@ size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
     const size_t nblk = (size_t(sh.max_kv) + sel->block - 1) / sel->block;
-    b += size_t(num_sms()) * nblk * attn::kMaxItemRows * sizeof(float);
+    b += size_t(num_sms()) * 2 * nblk * attn::kMaxItemRows * sizeof(float);  // double-buffered spill
   } else {
     b += align_up(sizeof(int) * (size_t(n_tiles_of(vl, sel->q_tile)) + 1), 256);  // token-score item prefix
   }
@@ -749,8 +749,9 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   if (sel->block == 1) return HS_ERR_UNSUPPORTED;
   const int T = sel->q_tile, B = sel->block;
   const int nblk = (sh.max_kv + B - 1) / B;
-  // one CTA's spill is nblk x 256 floats; the fixed scratch bounds the grid
-  const size_t per_cta = size_t(nblk) * attn::kMaxItemRows * sizeof(float);
+  // one CTA's spill is 2 x nblk x 256 floats (double-buffered); the fixed
+  // scratch bounds the grid
+  const size_t per_cta = 2 * size_t(nblk) * attn::kMaxItemRows * sizeof(float);
   const size_t cap = (kNoAllocScratchBytes - kHeaderBytes) / per_cta;
   if (cap < 1) return HS_ERR_WORKSPACE;  // sequence longer than the fixed scratch can serve
   cudaStream_t s = S(stream);

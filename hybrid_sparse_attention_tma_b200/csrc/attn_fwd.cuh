@@ -31,6 +31,12 @@ namespace hs {
 namespace attn {
 
 constexpr int kThreads = 320;
+// The full layer with block scores adds two warps (10, 11) that reduce each
+// work item's spilled block maxima while the softmax warps move on.
+template <int MODE, int SB>
+constexpr int threads_for() {
+  return (MODE == 0 && SB > 0) ? 384 : 320;
+}
 constexpr int kStages = 5;
 constexpr int kSlabBytes = 128 * 128;  // 128 rows x 64 bf16
 constexpr int kMaxItemRows = 256;
@@ -79,7 +85,7 @@ struct Params {
   float* lse;  // [Hq, Tq] natural log, may be null
   // block-score by-product (full mode with SB = B > 1)
   float* scores;  // [n_tiles, Hkv, nblk]
-  float* spill;   // [gridDim.x][nblk][256]
+  float* spill;   // [gridDim.x][2][nblk][256] (double-buffered per CTA)
   int nblk;
   int T, B;
   int chunks_per_tile;  // sparse mode: ceil(T*G / 256)
@@ -108,7 +114,9 @@ struct Ctl {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_ready[2], o_free[2];
   uint64_t teardown;
-  uint64_t sm_bar;  // bounded barrier over the 256 softmax threads
+  uint64_t sc_ready;    // softmax warps: item's spill + lse2 written (count 8)
+  uint64_t lse_taken;   // score warps: lse2 copied to registers (count 2)
+  uint64_t sc_free[2];  // score warps: spill buffer [parity] consumed (count 2)
   uint32_t tmem_base;
   int abort;
   float lse2[kMaxItemRows];
@@ -190,7 +198,7 @@ __device__ __forceinline__ KvPlan kv_plan(const Params& p, const Item& it, int m
 // The kernel
 // ------------------------------------------------------------------------
 template <int D, int MODE, int SB>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kb,
                     const __grid_constant__ CUtensorMap map_vb, const Params p,
@@ -216,7 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.o_free[t], 4);
     }
     mbar_init(&c.teardown, 1);
-    mbar_init(&c.sm_bar, 256);
+    mbar_init(&c.sc_ready, 8);
+    mbar_init(&c.lse_taken, 2);
+    mbar_init(&c.sc_free[0], 2);
+    mbar_init(&c.sc_free[1], 2);
     c.abort = 0;
     fence_mbar_init();
   }
@@ -412,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&c.teardown);
       mbar_wait_drain(&c.teardown, 0, p.wc, 92);
     }
-  } else {
+  } else if (warp < 8) {
     // ===================== softmax warpgroups =====================
     const int t = warp >> 2;       // Q-tile
     const int quad = warp & 3;     // TMEM lane quadrant
@@ -420,14 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int vr = t * 128 + r;      // row inside the item
     const uint32_t t_s = tmem + t * 256 + (uint32_t(quad * 32) << 16);
     const uint32_t t_o = t_s + 128;
-    int uses = 0, items_t = 0, sm_phase = 0;
+    int uses = 0, items_t = 0, sc_items = 0;
     bool ok = true;
-    // bounded replacement for a named barrier over warps 0-7
-    auto softmax_sync = [&]() {
-      mbar_arrive(&c.sm_bar);
-      mbar_wait_warp(&c.sm_bar, sm_phase & 1, abort_flag, p.wc, 30);
-      ++sm_phase;
-    };
     for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
@@ -441,6 +446,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int pos = it.pos0 + ql;
       const int qrow = it.qrow0 + ql;
       float m_used = -INFINITY, l = 0.f;
+      const int par = sc_items & 1;  // spill buffer of this item (full mode with scores)
+      if constexpr (MODE == kFull && SB > 0) {
+        if (sc_items >= 2 && ok &&
+            !mbar_wait_warp(&c.sc_free[par], ((sc_items >> 1) - 1) & 1, abort_flag, p.wc, 31, wi << 12))
+          ok = false;
+      }
       if (active && n > 0 && ok) {
         const int* idx_row =
             (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
@@ -515,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float mt = -INFINITY;
           if constexpr (MODE == kFull && SB > 0) {
             constexpr int nb = 128 / SB;
-            float* sp = p.spill + (size_t(blockIdx.x) * p.nblk) * kMaxItemRows + vr;
+            float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows + vr;
             float mb[nb];
 #pragma unroll
             for (int b = 0; b < nb; ++b) {
@@ -653,38 +664,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float lse2 = (l > 0.f) ? m_used + __log2f(l) : -INFINITY;
       if (valid && active && p.lse) p.lse[size_t(h) * p.Tq + qrow] = lse2 * 0.69314718055994531f;
       if (valid && n == 0 && p.lse) p.lse[size_t(h) * p.Tq + qrow] = -INFINITY;
-      // ---- score epilogue (full mode, B > 1): max over the tile's rows ----
+      // ---- hand the item's lse to the score warps (full mode, B > 1) ----
       if constexpr (MODE == kFull && SB > 0) {
+        if (sc_items >= 1 && ok &&
+            !mbar_wait_warp(&c.lse_taken, (sc_items - 1) & 1, abort_flag, p.wc, 32, wi << 12))
+          ok = false;
         c.lse2[vr] = lse2;
-        __threadfence_block();
-        softmax_sync();
-        if (ok && !*abort_flag) {
-          const int nblk_item = min(p.nblk, (n * 128) / SB);
-          const float* sp = p.spill + size_t(blockIdx.x) * p.nblk * kMaxItemRows;
-          const int sw = warp;  // 0..7
-          for (int b = sw; b < nblk_item; b += 8) {
-            int qa = 0;
-            while (qa < it.nq) {
-              const int in_tile = (it.qoff + qa) % p.T;
-              const int tid = it.tile0 + (it.qoff + qa) / p.T;
-              const int qb = min(it.nq, qa + (p.T - in_tile));
-              const int tile_last = min(it.pos0 + qa - in_tile + p.T - 1, it.kv_len - 1);
-              if (b * SB <= tile_last) {
-                float v = -INFINITY;
-                for (int rr = qa * p.G + lane; rr < qb * p.G; rr += 32)
-                  v = fmaxf(v, sp[size_t(b) * kMaxItemRows + rr] - c.lse2[rr]);
+        __threadfence_block();  // spill stores and lse2 visible before the arrive
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.sc_ready);
+        ++sc_items;
+      }
+    }
+  } else {
+    // ===================== score warps (10, 11) =====================
+    // score(t, g, b) = max over the tile's rows r of exp2(m_{r,b} - lse2_r):
+    // the per-row block maxima m were spilled during the main loop; with the
+    // final lse2 known they are reduced here, off the softmax critical path.
+    const int wq = warp - 10;                 // rows [128 wq, 128 wq + 128)
+    const int r0 = wq * 128 + lane * 4;       // this lane's 4 rows
+    int sc_items = 0;
+    if constexpr (MODE == kFull && SB > 0)
+    for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
+      const Item it = get_item<MODE>(p, sc, wi);
+      if (it.nq <= 0) continue;
+      const KvPlan kp = kv_plan(p, it, MODE);
+      const int n = kp.n_sel + kp.n_win;
+      if (!mbar_wait_warp(&c.sc_ready, sc_items & 1, abort_flag, p.wc, 40, wi << 12)) break;
+      float l2[4];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                if (lane == 0 && v > -INFINITY)
-                  atomicMax(reinterpret_cast<unsigned int*>(p.scores + (size_t(tid) * p.Hkv + it.g) * p.nblk + b),
-                            __float_as_uint(ex2(v)));
-              }
-              qa = qb;
-            }
+      for (int e = 0; e < 4; ++e) l2[e] = c.lse2[r0 + e];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.lse_taken);
+      const int par = sc_items & 1;
+      const int rows = it.nq * p.G;
+      const int w_lo = wq * 128, w_hi = min(rows, wq * 128 + 128);
+      if (w_lo < w_hi) {
+        const float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows;
+        const int nblk_item = min(p.nblk, (n * 128) / SB);
+        // selection tiles intersecting this warp's rows (row = query * G + head)
+        const int q_lo = w_lo / p.G, q_hi = (w_hi + p.G - 1) / p.G;
+        const int t_first = (it.qoff + q_lo) / p.T, t_last = (it.qoff + q_hi - 1) / p.T;
+        for (int b = 0; b < nblk_item; ++b) {
+          const float4 v4 = *reinterpret_cast<const float4*>(sp + size_t(b) * kMaxItemRows + r0);
+          const float vv[4] = {v4.x - l2[0], v4.y - l2[1], v4.z - l2[2], v4.w - l2[3]};
+          for (int tt = t_first; tt <= t_last; ++tt) {
+            // rows of tile tt inside the item: queries [tt*T - qoff, (tt+1)*T - qoff)
+            const int ra = max(w_lo, (tt * p.T - it.qoff) * p.G);
+            const int rb = min(w_hi, ((tt + 1) * p.T - it.qoff) * p.G);
+            const int tile_last = min(it.pos0 - it.qoff + (tt + 1) * p.T - 1, it.kv_len - 1);
+            if (b * SB > tile_last) continue;  // not a candidate of this tile
+            float v = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (r0 + e >= ra && r0 + e < rb) v = fmaxf(v, vv[e]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+            if (lane == 0 && v > -INFINITY)
+              atomicMax(reinterpret_cast<unsigned int*>(p.scores + (size_t(it.tile0 + tt) * p.Hkv + it.g) * p.nblk + b),
+                        __float_as_uint(ex2(v)));
           }
         }
-        softmax_sync();
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.sc_free[par]);
+      ++sc_items;
     }
   }
 

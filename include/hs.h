@@ -232,9 +232,9 @@ HS_API hs_status hs_swa_gated(const hs_varlen* vl, int32_t window,
  * behind. Calls whose kernels overlap on the GPU (e.g. on two streams without
  * ordering) race on it and give wrong results; order them.
  * Limits: block-level selection only (B >= 8). The grid is capped so that
- * grid * ceil(max_kv / B) KB fits in the array; if a single CTA's share
- * (ceil(max_kv / B) KB) does not fit -- more than 65535 blocks, i.e. max_kv
- * above ~4.19M tokens at B = 64 --
+ * grid * 2 * ceil(max_kv / B) KB fits in the array; if a single CTA's share
+ * (2 * ceil(max_kv / B) KB) does not fit -- more than 32767 blocks, i.e.
+ * max_kv above ~2.1M tokens at B = 64 --
  * the call returns HS_ERR_WORKSPACE before launching. Smaller caps only mean
  * fewer CTAs, not different results.
  * check != 0: synchronise `stream` after the launch and return HS_ERR_TIMEOUT

@@ -57,8 +57,8 @@ def test_noalloc_rejects_oversized_problem_before_launch():
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200 import _lib as L
     lib = L.load()
-    # 65536 blocks of 8 keys would need 64 MiB for a single CTA's spill
-    n = 8 * 65536
+    # 32768 blocks of 8 keys would need 64 MiB for a single CTA's double-buffered spill
+    n = 8 * 32768
     vl = hs.Varlen([0, 1], [0, n], 4, 1, 64, device="cuda")
     sel = hs.Sel(16, 8, 8, 0)
     dummy = torch.empty(16, dtype=torch.bfloat16, device="cuda")
