@@ -194,21 +194,25 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// Tensor maps of one attention launch. g / o (the other branch's output and
+// this call's output, boxes of 64 rows = 64/G queries x G heads) are used by
+// the gated sliding-window call only; the other calls pass copies of q.
 struct Maps {
-  CUtensorMap q, k, v, kb, vb;
+  CUtensorMap q, k, v, kb, vb, g, o;
 };
 
 // Launch the tcgen05 attention kernel.
 template <int D, int MODE, int SB>
 hs_status launch_attn(const Maps& m, const attn::Params& p, const attn::Sched& sc, int grid, cudaStream_t st) {
   auto kern = attn::attn_fwd_kernel<D, MODE, SB>;
-  constexpr int smem = attn::smem_bytes<D>() > 116 * 1024 ? attn::smem_bytes<D>() : 116 * 1024;
+  constexpr int need = attn::smem_bytes<D, MODE == attn::kSparse && SB == 0>();
+  constexpr int smem = need > 116 * 1024 ? need : 116 * 1024;
   static bool configured = false;
   if (!configured) {
     if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
     configured = true;
   }
-  kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, p, sc);
+  kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, m.g, m.o, p, sc);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
@@ -486,6 +490,7 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
+  m.g = m.o = m.q;
   static attn::Sched sc;  // large; filled per call under the host lock below
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -586,6 +591,7 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   } else if (!make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B)) {
     return HS_ERR_CUDA;
   }
+  m.g = m.o = m.q;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -708,6 +714,7 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
+  m.g = m.o = m.q;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -730,6 +737,9 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
   p.w = window;
   p.gamma = gamma;
   p.o_other = reinterpret_cast<const __nv_bfloat16*>(o_sparse);
+  // 64-row rounds of whole queries need G | 64; G = 128 mixes with direct loads/stores
+  p.o_tma = sh.G <= 64 && make_map_3d(&m.g, o_sparse, sh.d, sh.Hq, sh.Tq, sh.G, 64 / sh.G) &&
+            make_map_3d(&m.o, o, sh.d, sh.Hq, sh.Tq, sh.G, 64 / sh.G);
   p.wc = wait_ctl(ws);
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
   return dispatch_attn_d<attn::kSparse, 0>(sh.d, m, p, sc, grid, S(stream));
@@ -767,6 +777,7 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
+  m.g = m.o = m.q;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);

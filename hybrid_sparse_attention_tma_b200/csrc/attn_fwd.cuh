@@ -22,7 +22,11 @@
 // softmax writes P_t (bf16, two per column) over the first 64 columns of S_t
 // and the PV MMA reads its A operand from there.
 // SMEM: Q[2] | K/V ring[5] | control. All operand tiles use the 128-byte
-// swizzle (8-row x 128-byte atoms), K-major except V (MN-major).
+// swizzle (8-row x 128-byte atoms), K-major except V (MN-major). The gated
+// sliding-window instantiation runs a 3-stage ring and spends the freed space
+// on a 256-row output buffer: the softmax warpgroups TMA-load the other
+// branch's output into it when an item starts, mix their result in place and
+// TMA-store it.
 #pragma once
 
 #include "hs_common.cuh"
@@ -97,16 +101,20 @@ struct Params {
   // gate epilogue (sliding-window branch): o = sig(gamma) * o_other + (1 - sig(gamma)) * o_this
   const float* gamma;                // [Tq, Hq] or null
   const __nv_bfloat16* o_other;      // [Tq, Hq, D] sparse-branch output
+  int o_tma;                         // gated call: o_other / o move through smem by TMA (64 % G == 0)
   WaitCtl wc;
 };
 
-template <int D>
+template <int D, bool GATE>
 struct Layout {
   static constexpr int kSlabs = D / 64;
   static constexpr int kTileBytes = kSlabs * kSlabBytes;  // Q tile / K tile / V tile
+  static constexpr int kNStages = GATE ? 3 : kStages;     // K/V ring depth
+  static constexpr int kRound = 64 * D * 2;  // 64 output rows (bf16) as 128-byte swizzled 64-column slabs
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
-  static constexpr int kOffCtl = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffO = kOffKV + kNStages * kTileBytes;  // [2 warpgroups][2 rounds] (GATE only)
+  static constexpr int kOffCtl = kOffO + (GATE ? 4 * kRound : 0);
 };
 
 struct Ctl {
@@ -114,6 +122,8 @@ struct Ctl {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_ready[2], o_free[2];
   uint64_t teardown;
+  uint64_t wg_bar[2];   // per softmax warpgroup: bounded barrier of its 4 warps
+  uint64_t g_full[2];   // per softmax warpgroup: other-branch output landed (gated call)
   uint64_t sc_ready;    // softmax warps: item's spill + lse2 written (count 8)
   uint64_t lse_taken;   // score warps: lse2 copied to registers (count 2)
   uint64_t sc_free[2];  // score warps: spill buffer [parity] consumed (count 2)
@@ -122,11 +132,12 @@ struct Ctl {
   float lse2[kMaxItemRows];
 };
 
-template <int D>
+template <int D, bool GATE>
 constexpr int smem_bytes() {
   // + 1024 for manual 1024-byte alignment of the dynamic smem base
-  return Layout<D>::kOffCtl + int(sizeof(Ctl)) + 1024;
+  return Layout<D, GATE>::kOffCtl + int(sizeof(Ctl)) + 1024;
 }
+static_assert(smem_bytes<128, true>() <= 232448 && smem_bytes<128, false>() <= 232448, "smem over 227 KB");
 
 
 template <int MODE>
@@ -201,9 +212,13 @@ template <int D, int MODE, int SB>
 __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kb,
-                    const __grid_constant__ CUtensorMap map_vb, const Params p,
+                    const __grid_constant__ CUtensorMap map_vb, const __grid_constant__ CUtensorMap map_g,
+                    const __grid_constant__ CUtensorMap map_o, const Params p,
                     const __grid_constant__ Sched sc) {
-  using L = Layout<D>;
+  // the window-only instantiation serves the gated sliding-window call
+  constexpr bool kGate = (MODE == kSparse && SB == 0);
+  using L = Layout<D, kGate>;
+  constexpr int kNS = L::kNStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kOffCtl);
@@ -224,6 +239,10 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       mbar_init(&c.o_free[t], 4);
     }
     mbar_init(&c.teardown, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&c.wg_bar[t], 4);
+      mbar_init(&c.g_full[t], 1);
+    }
     mbar_init(&c.sc_ready, 8);
     mbar_init(&c.lse_taken, 2);
     mbar_init(&c.sc_free[0], 2);
@@ -243,6 +262,10 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       prefetch_tensormap(&map_kb);
       prefetch_tensormap(&map_vb);
     }
+    if (kGate && p.o_tma) {
+      prefetch_tensormap(&map_g);
+      prefetch_tensormap(&map_o);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -256,9 +279,9 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     // gathers all 32 lanes fetch indices and issue gather4 loads in parallel.
     int ctr = 0;        // K/V ring uses
     int q_uses = 0;     // Q loads issued
-    int last_use[kStages];
+    int last_use[kNS];
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) last_use[s] = -1;
+    for (int s = 0; s < kNS; ++s) last_use[s] = -1;
     bool ok = true;
     auto wait0 = [&](uint64_t* bar, uint32_t parity, int site, int ctx) -> bool {
       int r = 1;
@@ -285,8 +308,8 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       const int* idx_row = (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
       for (int i = 0; i < n && ok; ++i) {
         for (int kind = 0; kind < 2; ++kind) {
-          const int s = ctr % kStages;
-          if (!wait0(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, 2, (wi << 12) | i)) { ok = false; break; }
+          const int s = ctr % kNS;
+          if (!wait0(&c.kv_empty[s], ((ctr / kNS) & 1) ^ 1, 2, (wi << 12) | i)) { ok = false; break; }
           if (lane == 0) mbar_expect_tx(&c.kv_full[s], L::kTileBytes);
           __syncwarp();
           uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
@@ -332,8 +355,8 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     }
     // drain: never leave the CTA with TMA writes in flight
     if (lane == 0 && *abort_flag) {
-      for (int s = 0; s < kStages; ++s)
-        if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kStages) & 1, p.wc, 90);
+      for (int s = 0; s < kNS; ++s)
+        if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kNS) & 1, p.wc, 90);
       if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 91);
     }
   } else if (warp == 9) {
@@ -345,8 +368,9 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       int uses[2] = {0, 0};        // S/P/O phases per Q-tile
       int items_t[2] = {0, 0};     // items in which tile t took part (o_free phase)
       bool ok = true;
-      const uint32_t q_base = smem_u32(smem + L::kOffQ);
-      const uint32_t kv_base = smem_u32(smem + L::kOffKV);
+      const uint64_t q_desc0 = sdesc_sw128(smem_u32(smem + L::kOffQ), 16, 1024);
+      const uint64_t k_desc0 = sdesc_sw128(smem_u32(smem + L::kOffKV), 16, 1024);
+      const uint64_t v_desc0 = sdesc_sw128(smem_u32(smem + L::kOffKV), kSlabBytes, 1024);
       for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
         const Item it = get_item<MODE>(p, sc, wi);
         if (it.nq <= 0) continue;
@@ -357,39 +381,41 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10, wi << 12)) { ok = false; break; }
         ++q_uses;
         tc_fence_after();
+        // Descriptors are built once; a K step only adds its byte offset / 16
+        // to the 14-bit start-address field (no carry: smem < 256 KB). Keeping
+        // the issuing thread's work per MMA to an add lets the tensor pipe run
+        // back to back (a 128x128x16 MMA takes 64 cycles).
         auto issue_qk = [&](int t, int stage) {
           const uint32_t d_tmem = tmem + t * 256;
-          const uint32_t qa = q_base + t * L::kTileBytes;
-          const uint32_t kb = kv_base + stage * L::kTileBytes;
+          const uint64_t qd = q_desc0 + uint64_t((t * L::kTileBytes) >> 4);
+          const uint64_t kd = k_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-            umma_bf16(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), kIdQK,
-                      kk > 0 ? 1u : 0u);
+            const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
+            umma_bf16(d_tmem, qd + off, kd + off, kIdQK, kk > 0 ? 1u : 0u);
           }
           umma_commit(&c.s_full[t]);
         };
         auto issue_pv = [&](int t, int stage, bool acc) {
           const uint32_t d_tmem = tmem + t * 256 + 128;
           const uint32_t pa = tmem + t * 256;  // P_t over the first 64 columns of S_t
-          const uint32_t vb = kv_base + stage * L::kTileBytes;
+          const uint64_t vd = v_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
+          umma_bf16_ts(d_tmem, pa, vd, kIdPV, acc ? 1u : 0u);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16_ts(d_tmem, pa + kk * 8, sdesc_sw128(vb + kk * 2048, kSlabBytes, 1024), kIdPV,
-                         (acc || kk > 0) ? 1u : 0u);
+          for (int kk = 1; kk < 8; ++kk) umma_bf16_ts(d_tmem, pa + kk * 8, vd + uint64_t(kk * (2048 >> 4)), kIdPV, 1u);
           umma_commit(&c.o_ready[t]);
         };
         // prologue: S_t(0)
-        int sk = ctr % kStages;
-        if (!mbar_wait(&c.kv_full[sk], (ctr / kStages) & 1, abort_flag, p.wc, 11, wi << 12)) { ok = false; break; }
+        int sk = ctr % kNS;
+        if (!mbar_wait(&c.kv_full[sk], (ctr / kNS) & 1, abort_flag, p.wc, 11, wi << 12)) { ok = false; break; }
         ++ctr;
         tc_fence_after();
         for (int t = 0; t < n_qt; ++t) issue_qk(t, sk);
         umma_commit(&c.kv_empty[sk]);
         if (n == 1) umma_commit(&c.q_empty);  // Q is only read by QK: free it early
         for (int i = 0; i < n && ok; ++i) {
-          const int sv = ctr % kStages;
-          if (!mbar_wait(&c.kv_full[sv], (ctr / kStages) & 1, abort_flag, p.wc, 12, (wi << 12) | i)) { ok = false; break; }
+          const int sv = ctr % kNS;
+          if (!mbar_wait(&c.kv_full[sv], (ctr / kNS) & 1, abort_flag, p.wc, 12, (wi << 12) | i)) { ok = false; break; }
           ++ctr;
           int sk_next = -1;
           for (int t = 0; t < n_qt; ++t) {
@@ -400,8 +426,8 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
             issue_pv(t, sv, i > 0);
             if (i + 1 < n) {
               if (sk_next < 0) {
-                sk_next = ctr % kStages;
-                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kStages) & 1, abort_flag, p.wc, 15, (wi << 12) | i)) { ok = false; break; }
+                sk_next = ctr % kNS;
+                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kNS) & 1, abort_flag, p.wc, 15, (wi << 12) | i)) { ok = false; break; }
                 ++ctr;
                 tc_fence_after();
               }
@@ -433,6 +459,17 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     const uint32_t t_o = t_s + 128;
     int uses = 0, items_t = 0, sc_items = 0;
     bool ok = true;
+    // gated call: this warpgroup's two 64-row rounds of the output buffer, the
+    // phase of its bounded barrier and of g_full, and the loads it issued
+    uint8_t* o_buf = smem + L::kOffO + t * 2 * L::kRound;
+    int wg_phase = 0, g_uses = 0, g_issued = 0;
+    auto wg_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.wg_bar[t]);
+      const bool r = mbar_wait_warp(&c.wg_bar[t], wg_phase & 1, abort_flag, p.wc, 33);
+      ++wg_phase;
+      return r;
+    };
     for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
@@ -447,12 +484,30 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       const int qrow = it.qrow0 + ql;
       float m_used = -INFINITY, l = 0.f;
       const int par = sc_items & 1;  // spill buffer of this item (full mode with scores)
+      float sg = 0.f;                // gate of this row (gated call)
+      if constexpr (kGate) {
+        if (p.gamma && valid) sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
+      }
       if constexpr (MODE == kFull && SB > 0) {
         if (sc_items >= 2 && ok &&
             !mbar_wait_warp(&c.sc_free[par], ((sc_items >> 1) - 1) & 1, abort_flag, p.wc, 31, wi << 12))
           ok = false;
       }
       if (active && n > 0 && ok) {
+        if constexpr (kGate) {
+          // the other branch's output does not depend on this item: load its
+          // rows now, behind the whole softmax loop (the buffer's previous
+          // store was read out before this thread left the last epilogue)
+          if (p.o_tma && p.gamma && quad == 0 && lane == 0) {
+            const int nr = min(2, (rows - t * 128 + 63) / 64);
+            mbar_expect_tx(&c.g_full[t], nr * L::kRound);
+            for (int rd = 0; rd < nr; ++rd)
+              for (int sl = 0; sl < L::kSlabs; ++sl)
+                tma_load_3d(o_buf + rd * L::kRound + sl * (64 * 128), &map_g, &c.g_full[t], sl * 64, it.g * p.G,
+                            it.qrow0 + (t * 128 + rd * 64) / p.G);
+            ++g_issued;
+          }
+        }
         const int* idx_row =
             (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
         for (int i = 0; i < n; ++i) {
@@ -598,52 +653,89 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           if (lane == 0) mbar_arrive(&c.p_full[t]);
         }
         // ---- epilogue: O / l, lse ----
-        // the gate's inputs do not depend on this item's result: fetch them
-        // while the last PV is still running
-        // (only the window-only instantiation, which serves the gated SWA call,
-        // carries the gate)
-        constexpr bool kGate = (MODE == kSparse && SB == 0);
-        float sg = 0.f;
-        uint4 osrc[kGate ? D / 8 : 1];
-        if (kGate && p.gamma && valid) {
-          sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
-          const uint4* src = reinterpret_cast<const uint4*>(p.o_other + (size_t(qrow) * p.Hq + h) * D);
-#pragma unroll
-          for (int j = 0; j < D / 8; ++j) osrc[j] = __ldg(src + j);
-        }
         if (ok && mbar_wait_warp(&c.o_ready[t], (uses + n - 1) & 1, abort_flag, p.wc, 22)) {
           tc_fence_after();
           const float inv = l > 0.f ? 1.f / l : 0.f;
           __nv_bfloat16* orow = p.o + (size_t(qrow) * p.Hq + h) * D;
+          if constexpr (kGate) {
+            // o = sig(gamma) o_other + (1 - sig(gamma)) o_this. With o_tma the
+            // other branch's rows sit in this warpgroup's buffer in the TMA
+            // box layout; each thread overwrites its row in place and one
+            // thread stores the full 64-row rounds (partial ones go direct).
+            const bool gate = p.gamma != nullptr;
+            if (p.o_tma && gate && ok) {
+              if (mbar_wait_warp(&c.g_full[t], g_uses & 1, abort_flag, p.wc, 23, wi << 12)) ++g_uses;
+              else ok = false;
+            }
+            const int rnd = quad >> 1;
+            const int row_base = t * 128 + rnd * 64;
+            const bool tma_round = p.o_tma && row_base + 64 <= rows;
+            const int rr = vr - row_base;  // 0..63
+            uint8_t* rbuf = o_buf + rnd * L::kRound + rr * 128;
+            const uint4* src = reinterpret_cast<const uint4*>(p.o_other + (size_t(qrow) * p.Hq + h) * D);
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+            if (ok) {
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t ov[32];
-            tmem_ld32(t_o + ch * 32, ov);
-            tmem_ld_wait();
-            if (valid) {
-              float of[32];
-#pragma unroll
-              for (int j = 0; j < 32; ++j) of[j] = __uint_as_float(ov[j]) * inv;
-              if (kGate && p.gamma) {
+              for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t ov[32];
+                tmem_ld32(t_o + ch * 32, ov);
+                tmem_ld_wait();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                  const uint4 u4 = osrc[kGate ? ch * 4 + j : 0];
-                  const uint32_t w4[4] = {u4.x, u4.y, u4.z, u4.w};
+                  uint4* chunk = reinterpret_cast<uint4*>(rbuf + (ch >> 1) * (64 * 128) +
+                                                          ((((ch & 1) * 4 + j) ^ (rr & 7)) << 4));
+                  float of[8];
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&w4[e]);
-                    const float2 f2 = __bfloat1622float2(b2);
-                    of[8 * j + 2 * e] = sg * f2.x + (1.f - sg) * of[8 * j + 2 * e];
-                    of[8 * j + 2 * e + 1] = sg * f2.y + (1.f - sg) * of[8 * j + 2 * e + 1];
+                  for (int e = 0; e < 8; ++e) of[e] = __uint_as_float(ov[8 * j + e]) * inv;
+                  if (gate && valid) {
+                    const uint4 u4 = p.o_tma ? *chunk : __ldg(src + ch * 4 + j);
+                    const uint32_t w4[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                      const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                      of[2 * e] = sg * f2.x + (1.f - sg) * of[2 * e];
+                      of[2 * e + 1] = sg * f2.y + (1.f - sg) * of[2 * e + 1];
+                    }
                   }
+                  const uint4 res = make_uint4(pack_bf16(of[0], of[1]), pack_bf16(of[2], of[3]),
+                                               pack_bf16(of[4], of[5]), pack_bf16(of[6], of[7]));
+                  if (tma_round) *chunk = res;
+                  else if (valid) dst[ch * 4 + j] = res;
                 }
               }
-              uint32_t pk2[16];
+            }
+            if (p.o_tma) {
+              fence_proxy_async_smem();
+              if (!wg_sync()) {
+                ok = false;
+              } else if (quad == 0 && lane == 0 && ok) {
+                for (int rd = 0; rd < 2; ++rd) {
+                  const int rb = t * 128 + rd * 64;
+                  if (rb + 64 <= rows)
+                    for (int sl = 0; sl < L::kSlabs; ++sl)
+                      tma_store_3d(&map_o, o_buf + rd * L::kRound + sl * (64 * 128), sl * 64, it.g * p.G,
+                                   it.qrow0 + rb / p.G);
+                }
+                bulk_commit();
+                bulk_wait_read0();  // the buffer may be refilled once the stores have read it
+              }
+            }
+          } else {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) pk2[j] = pack_bf16(of[2 * j], of[2 * j + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t ov[32];
+              tmem_ld32(t_o + ch * 32, ov);
+              tmem_ld_wait();
+              if (valid) {
+                uint32_t pk2[16];
 #pragma unroll
-              for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk2[4 * j], pk2[4 * j + 1], pk2[4 * j + 2], pk2[4 * j + 3]);
+                for (int j = 0; j < 16; ++j)
+                  pk2[j] = pack_bf16(__uint_as_float(ov[2 * j]) * inv, __uint_as_float(ov[2 * j + 1]) * inv);
+                uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  dst[j] = make_uint4(pk2[4 * j], pk2[4 * j + 1], pk2[4 * j + 2], pk2[4 * j + 3]);
+              }
             }
           }
           tc_fence_before();
@@ -674,6 +766,13 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&c.sc_ready);
         ++sc_items;
+      }
+    }
+    if constexpr (kGate) {
+      // never leave with TMA traffic on this warpgroup's buffer in flight
+      if (quad == 0 && lane == 0) {
+        if (g_issued > g_uses) mbar_wait_drain(&c.g_full[t], (g_issued - 1) & 1, p.wc, 93);
+        bulk_wait0();
       }
     }
   } else {

@@ -215,8 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int qctr = 0, items = 0;
       int acc_cnt[kBlocks] = {0, 0, 0, 0};
       bool ok = true;
-      const uint32_t k_base = smem_u32(smem + L::kOffK);
-      const uint32_t q_base = smem_u32(smem + L::kOffQ);
+      // descriptors built once; a K step adds its offset / 16 to the start field
+      const uint64_t k_desc0 = sdesc_sw128(smem_u32(smem + L::kOffK), 16, 1024);
+      const uint64_t q_desc0 = sdesc_sw128(smem_u32(smem + L::kOffQ), 16, 1024);
       for (int wi = blockIdx.x; wi < p.n_items && ok; wi += gridDim.x) {
         const Item it = get_item(st, p, tile_items_prefix, wi);
         const int nb = (it.nkeys + 127) / 128;
@@ -231,12 +232,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 !mbar_wait(&c.acc_free[b], (acc_cnt[b] - 1) & 1, abort_flag, p.wc, 112, (wi << 12) | qc)) { ok = false; break; }
             ++acc_cnt[b];
             tc_fence_after();
-            const uint32_t ka = k_base + b * L::kTile, qb = q_base + s * L::kTile;
+            const uint64_t ka = k_desc0 + uint64_t((b * L::kTile) >> 4);
+            const uint64_t qb = q_desc0 + uint64_t((s * L::kTile) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * kSlabBytes + (kk & 3) * 32;
-              umma_bf16(tmem + b * 128, sdesc_sw128(ka + off, 16, 1024), sdesc_sw128(qb + off, 16, 1024), kId,
-                        kk > 0 ? 1u : 0u);
+              const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
+              umma_bf16(tmem + b * 128, ka + off, qb + off, kId, kk > 0 ? 1u : 0u);
             }
             umma_commit(&c.acc_full[b]);
           }
