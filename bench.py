@@ -161,6 +161,26 @@ def dist_setup():
     return world, rank, local
 
 
+def rank_seed(w, rank: int) -> int:
+    """Seed of the independent block rank `rank` processes (distinct per rank)."""
+    return 1000 + w.config_index + 7919 * rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of per-rank timings (every rank gets the result); the
+    only collective of the bench, outside the timed region."""
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_rate(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
+    """Tokens/s of the whole job: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def make_runner(w, device, seed):
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200.block import HybridBlock, SparseLayerIn
@@ -220,7 +240,7 @@ def bench_ours(args, world, rank, local):
     w = workload(args)
     if args.fp8_kv:
         w = w.with_(fp8_kv=True)
-    inp, vl, blk, layers = make_runner(w, device, seed=1000 + w.config_index + 7919 * rank)
+    inp, vl, blk, layers = make_runner(w, device, seed=rank_seed(w, rank))
     stream = torch.cuda.current_stream()
     fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if args.fp8_kv else None
 
@@ -285,14 +305,12 @@ def bench_ours(args, world, rank, local):
     hs.check_error(blk.ws)
     ms_total = t0.elapsed_time(t1)
     kms = {kd: (sum(a.elapsed_time(b) for a, b in ev[kd]) / len(ev[kd]) if ev[kd] else 0.0) for kd in kinds}
-    vals = torch.tensor([ms_total] + [kms[kd] for kd in kinds], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    ms_total = vals[0].item()
-    kms = {kd: vals[i + 1].item() for i, kd in enumerate(kinds)}
+    vals = max_over_ranks([ms_total] + [kms[kd] for kd in kinds], device)
+    ms_total = vals[0]
+    kms = {kd: vals[i + 1] for i, kd in enumerate(kinds)}
     ms_step = ms_total / args.steps
     tokens = w.total_q
-    value = world * tokens / (ms_step / 1e3)
+    value = whole_job_rate(world, tokens, ms_step)
 
     # ---- algorithmic work of each kernel launch ----
     hbm, tf_burst, tf_sust, src = peaks()
@@ -328,7 +346,12 @@ def bench_ours(args, world, rank, local):
         entry("sparse", kms["sparse"], 4.0 * d * G * vis, "tensor")
     entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
     if w.swa_window > 0:
-        entry("swa", kms["swa"], 4.0 * d * hq * swa_pairs(w), "tensor")
+        # window of 128 keys: its FLOPs take < 1/3 of the time its bytes need at
+        # the HBM peak, so the branch is bound by HBM: Q, K_swa, V_swa, o_sparse
+        # and gamma read once, O written once
+        entry("swa", kms["swa"], 3 * q_bytes + 2 * kv_bytes + w.total_q * hq * 4, "hbm")
+        if "swa" in kernels:
+            kernels["swa"]["flop_per_launch"] = 4.0 * d * hq * swa_pairs(w)
     per_step = {"full": 1, "topk": 1, "sparse": len(layers), "swa": len(layers) if w.swa_window else 0}
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
@@ -407,12 +430,8 @@ def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
-    t = torch.tensor([ms], dtype=torch.float64, device=device)
-    if world > 1:
-        import torch.distributed as dist
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = t.item()
-    return {"value": round(world * w.total_q / (ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    ms = max_over_ranks([ms], device)[0]
+    return {"value": round(whole_job_rate(world, w.total_q, ms), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
