@@ -5,8 +5,9 @@ Workload (default): HySparse block-level prefill, 1 x 32768 tokens, 32 query
 heads / 8 KV heads, d = 128, 64-token blocks, top-16, separate SWA window 128
 + sigmoid gate, 1 full layer feeding 3 sparse layers; seeded synthetic bf16
 N(0,1) inputs with 1 % planted keys. A "step" is one pass of the whole block:
-hs_full_attn_select -> hs_topk_select -> 3 x (hs_sparse_attn_prefill ->
-hs_swa_gated). The per-step working set (~2 GB) is larger than the 126 MB L2.
+hs_full_attn_select -> hs_topk_select -> 3 x hs_sparse_swa_gated_prefill (the
+sparse branch, the own-cache window branch and the gate of one layer in one
+launch). The per-step working set (~2 GB) is larger than the 126 MB L2.
 
 Multi-GPU (torchrun): every rank runs its own independent block (its own
 sequences); no data-path collective. value = tokens of all ranks / max-over-
@@ -234,7 +235,8 @@ def bench_ours(args, world, rank, local):
     import torch.distributed as dist
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
-                                                  sparse_attn_decode, swa_gated, HS_KV_BF16, HS_KV_FP8_E4M3)
+                                                  sparse_attn_decode, sparse_swa_gated_prefill, HS_KV_BF16,
+                                                  HS_KV_FP8_E4M3)
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
     w = workload(args)
@@ -245,7 +247,7 @@ def bench_ours(args, world, rank, local):
     fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if args.fp8_kv else None
 
     for _ in range(max(3, args.warmup)):
-        blk.forward(inp.q, inp.k, inp.v, layers, stream=stream, fp8_kv=fp8_kv)
+        blk.forward(inp.q, inp.k, inp.v, layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
     torch.cuda.synchronize()
     hs.check_error(blk.ws)
 
@@ -277,13 +279,15 @@ def bench_ours(args, world, rank, local):
                     rec("sparse", lambda: sparse_attn_decode(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
                                                              kv_dtype=HS_KV_BF16, o=bufs["o_sp" + tag],
                                                              lse=bufs["lse_sp" + tag], ws=blk.ws, stream=stream))
+            elif blk.swa_window > 0:
+                # the whole sparse layer: sparse branch, own-cache window, gate
+                rec("sparse", lambda: sparse_swa_gated_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
+                                                               blk.swa_window, L.k_swa, L.v_swa, L.gamma,
+                                                               o=bufs["o_l" + tag], ws=blk.ws, stream=stream))
             else:
                 rec("sparse", lambda: sparse_attn_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
                                                           bufs["o_sp" + tag], bufs["lse_sp" + tag], ws=blk.ws,
                                                           stream=stream))
-            if blk.swa_window > 0:
-                rec("swa", lambda: swa_gated(vl, blk.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, bufs["o_sp" + tag],
-                                             bufs["o_l" + tag], ws=blk.ws, stream=stream))
 
     if world > 1:
         dist.barrier()
@@ -343,15 +347,11 @@ def bench_ours(args, world, rank, local):
         entry("sparse", kms["sparse"], vis * 2 * row + q_bytes * 2, "hbm")
     else:
         entry("full", kms["full"], full_flops(w), "tensor")
-        entry("sparse", kms["sparse"], 4.0 * d * G * vis, "tensor")
+        # a fused layer also runs the own-cache window branch (4 d H_q per
+        # visible (query, key) pair of the window)
+        swa_flop = 4.0 * d * hq * swa_pairs(w) if w.swa_window > 0 else 0.0
+        entry("sparse", kms["sparse"], 4.0 * d * G * vis + swa_flop, "tensor")
     entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
-    if w.swa_window > 0:
-        # window of 128 keys: its FLOPs take < 1/3 of the time its bytes need at
-        # the HBM peak, so the branch is bound by HBM: Q, K_swa, V_swa, o_sparse
-        # and gamma read once, O written once
-        entry("swa", kms["swa"], 3 * q_bytes + 2 * kv_bytes + w.total_q * hq * 4, "hbm")
-        if "swa" in kernels:
-            kernels["swa"]["flop_per_launch"] = 4.0 * d * hq * swa_pairs(w)
     per_step = {"full": 1, "topk": 1, "sparse": len(layers), "swa": len(layers) if w.swa_window else 0}
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
@@ -416,7 +416,7 @@ def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
                 dl.k_swa.copy_(d["k_swa"], non_blocking=True)
                 dl.v_swa.copy_(d["v_swa"], non_blocking=True)
                 dl.gamma.copy_(d["gamma"], non_blocking=True)
-        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream, fp8_kv=fp8_kv)
+        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
         out_host.copy_(res["layers"][-1]["o"], non_blocking=True)
 
     for _ in range(3):

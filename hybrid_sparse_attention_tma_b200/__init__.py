@@ -17,7 +17,8 @@ from . import _lib as L
 from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
 
 __all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
-           "sparse_attn_decode", "swa_gated", "workspace_size", "check_error", "HsError"]
+           "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "workspace_size", "check_error",
+           "HsError"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -155,6 +156,23 @@ def sparse_attn_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, o=None, lse
         ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), _ptr(o),
         _ptr(lse), _ptr(buf), buf.numel(), _stream(stream)))
     return o, lse
+
+
+def sparse_swa_gated_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, swa_window: int, k_swa, v_swa, gamma,
+                             o=None, o_sparse=None, lse_sparse=None, ws: Optional[Workspace] = None, stream=None):
+    """A whole HySparse sparse layer in one launch: block-sparse branch over the
+    reused cache, own-cache sliding window, sigmoid gate. o_sparse / lse_sparse
+    are written only when given. Returns o."""
+    lib = L.load()
+    dev = q.device
+    o = torch.empty_like(q) if o is None else o
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_SPARSE_SWA_GATED_PREFILL, vl, sel), stream)
+    L.check("hs_sparse_swa_gated_prefill", lib.hs_sparse_swa_gated_prefill(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), swa_window,
+        _ptr(k_swa), _ptr(v_swa), _ptr(gamma), _ptr(o), _ptr(o_sparse), _ptr(lse_sparse), _ptr(buf), buf.numel(),
+        _stream(stream)))
+    return o
 
 
 def sparse_attn_decode(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, k_scale=None, v_scale=None,

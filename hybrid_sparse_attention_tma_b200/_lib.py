@@ -8,7 +8,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libhs.so")
 
 HS_OK, HS_ERR_INVALID_ARG, HS_ERR_UNSUPPORTED, HS_ERR_WORKSPACE, HS_ERR_CUDA, HS_ERR_TIMEOUT = range(6)
-HS_OP_FULL_ATTN_SELECT, HS_OP_TOPK_SELECT, HS_OP_SPARSE_ATTN_PREFILL, HS_OP_SPARSE_ATTN_DECODE, HS_OP_SWA_GATED = range(5)
+(HS_OP_FULL_ATTN_SELECT, HS_OP_TOPK_SELECT, HS_OP_SPARSE_ATTN_PREFILL, HS_OP_SPARSE_ATTN_DECODE, HS_OP_SWA_GATED,
+ HS_OP_SPARSE_SWA_GATED_PREFILL) = range(6)
 HS_KV_BF16, HS_KV_FP8_E4M3 = 0, 1
 
 # Every function the header declares; the CPU test checks the library exports them all.
@@ -16,7 +17,7 @@ EXPORTS = [
     "hs_workspace_size", "hs_workspace_init", "hs_check_error", "hs_status_string",
     "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
     "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
-    "hs_full_attn_select_noalloc",
+    "hs_full_attn_select_noalloc", "hs_sparse_swa_gated_prefill",
 ]
 
 
@@ -72,6 +73,8 @@ def load():
     lib.hs_sparse_attn_decode.argtypes = [VL, SEL, vp, i32, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, sz, vp]
     lib.hs_swa_gated.restype = i32
     lib.hs_swa_gated.argtypes = [VL, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hs_sparse_swa_gated_prefill.restype = i32
+    lib.hs_sparse_swa_gated_prefill.argtypes = [VL, SEL, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hs_full_attn_select_noalloc.restype = i32
     lib.hs_full_attn_select_noalloc.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, i32, vp]
     lib.hs_last_error_detail.restype = i32

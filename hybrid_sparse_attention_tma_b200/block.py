@@ -13,7 +13,7 @@ from typing import List, Optional
 import torch
 
 from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
-               swa_gated, HS_KV_BF16, HS_KV_FP8_E4M3)
+               swa_gated, sparse_swa_gated_prefill, HS_KV_BF16, HS_KV_FP8_E4M3)
 
 
 @dataclass
@@ -26,10 +26,13 @@ class SparseLayerIn:
 
 class HybridBlock:
     def __init__(self, vl: Varlen, q_tile: int, block: int, topk: int, window: int, swa_window: int = 0,
-                 device="cuda"):
+                 device="cuda", fused: bool = True):
         self.vl = vl
         self.sel = Sel(q_tile, block, topk, window)
         self.swa_window = swa_window
+        # prefill layers with a window branch run as one fused launch
+        # (hs_sparse_swa_gated_prefill) unless fused=False (two launches)
+        self.fused = fused
         self.ws = Workspace(device)
         self.device = device
         self._bufs = {}
@@ -45,13 +48,16 @@ class HybridBlock:
             self._bufs[name] = t
         return t
 
-    def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False, fp8_kv=None):
+    def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False, fp8_kv=None,
+                intermediates: bool = True):
         """Returns dict(o_full, lse_full, scores, idx, cnt, layers=[{o_sparse, lse_sparse, o}]).
 
         With keep_all=False, output buffers are reused across calls (no
         allocation in steady state) and only the last layer's tensors are
         guaranteed distinct. fp8_kv = (k_codes, v_codes, k_scale, v_scale) makes the
-        sparse decode layers read an FP8-e4m3 copy of the KV cache."""
+        sparse decode layers read an FP8-e4m3 copy of the KV cache. With
+        intermediates=False a fused layer does not write o_sparse / lse_sparse
+        (they are returned as None)."""
         vl, sel = self.vl, self.sel
         Tq, Hq, d = q.shape
         nblk = (vl.max_kv + sel.block - 1) // sel.block
@@ -76,6 +82,14 @@ class HybridBlock:
                 else:
                     sparse_attn_decode(vl, sel, L.q, k, v, idx, cnt, kv_dtype=HS_KV_BF16, o=o_sp, lse=lse_sp,
                                        ws=self.ws, stream=stream)
+            elif self.swa_window > 0 and self.fused:
+                o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
+                if not intermediates:
+                    o_sp = lse_sp = None
+                sparse_swa_gated_prefill(vl, sel, L.q, k, v, idx, cnt, self.swa_window, L.k_swa, L.v_swa, L.gamma,
+                                         o=o_l, o_sparse=o_sp, lse_sparse=lse_sp, ws=self.ws, stream=stream)
+                outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
+                continue
             else:
                 sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream)
             if self.swa_window > 0:
@@ -91,11 +105,13 @@ class HybridBlock:
         """Kernels of this library launched by one forward (memsets excluded):
         full layer 1 (block scores) / 3 (token scores: forward, item prefix,
         score pass) / 4 (decode: two passes and two combines); top-k 1; each
-        sparse layer 1 (prefill) or 2 (decode: partials + combine), plus 1 for
-        the gated SWA branch."""
+        sparse layer 1 (prefill, with its window branch and gate when fused)
+        or 2 (decode: partials + combine), plus 1 for an unfused gated SWA
+        branch."""
         if self.decode:
             full = 4
         else:
             full = 1 if self.sel.block > 1 else 3
         sparse = 2 if self.decode else 1
-        return full + 1 + n_layers * (sparse + (1 if self.swa_window > 0 else 0))
+        swa = 1 if (self.swa_window > 0 and not (self.fused and not self.decode)) else 0
+        return full + 1 + n_layers * (sparse + swa)

@@ -198,21 +198,21 @@ cudaError_t set_smem(K kernel, int bytes) {
 // this call's output, boxes of 64 rows = 64/G queries x G heads) are used by
 // the gated sliding-window call only; the other calls pass copies of q.
 struct Maps {
-  CUtensorMap q, k, v, kb, vb, g, o;
+  CUtensorMap q, k, v, kb, vb, g, o, ks, vs;  // ks / vs: the fused sparse layer's own window cache
 };
 
 // Launch the tcgen05 attention kernel.
 template <int D, int MODE, int SB>
 hs_status launch_attn(const Maps& m, const attn::Params& p, const attn::Sched& sc, int grid, cudaStream_t st) {
   auto kern = attn::attn_fwd_kernel<D, MODE, SB>;
-  constexpr int need = attn::smem_bytes<D, MODE == attn::kSparse && SB == 0>();
+  constexpr int need = attn::smem_bytes<D, (MODE == attn::kSparse && SB == 0) || MODE == attn::kFused>();
   constexpr int smem = need > 116 * 1024 ? need : 116 * 1024;
   static bool configured = false;
   if (!configured) {
     if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
     configured = true;
   }
-  kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, m.g, m.o, p, sc);
+  kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, m.g, m.o, m.ks, m.vs, p, sc);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
@@ -387,6 +387,7 @@ size_t hs_workspace_size(int op, const hs_varlen* vl, const hs_sel* sel) {
     case HS_OP_TOPK_SELECT:
     case HS_OP_SPARSE_ATTN_PREFILL:
     case HS_OP_SWA_GATED:
+    case HS_OP_SPARSE_SWA_GATED_PREFILL:
       return kHeaderBytes;
     case HS_OP_SPARSE_ATTN_DECODE:
       if (!sel || check_sel(sel) != HS_OK) return 0;
@@ -490,7 +491,7 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
-  m.g = m.o = m.q;
+  m.g = m.o = m.ks = m.vs = m.q;
   static attn::Sched sc;  // large; filled per call under the host lock below
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -567,15 +568,30 @@ hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* sc
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
-hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
-                                 const void* v, const int32_t* idx, const int32_t* cnt, void* o, float* lse,
-                                 void* ws, size_t ws_bytes, hs_stream_t stream) {
+// One sparse layer: the plain sparse branch, or (swa != null) the fused layer
+// with the sliding-window branch and the gate.
+struct SwaArgs {
+  int32_t window;
+  const void* k_swa;
+  const void* v_swa;
+  const float* gamma;
+  void* o_sparse;  // optional
+};
+
+static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const int32_t* cnt, void* o, float* lse, const SwaArgs* swa,
+                              void* ws, size_t ws_bytes, hs_stream_t stream) {
   Shape sh;
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
   if (!q || !k || !v || !o || (sel->topk > 0 && (!idx || !cnt))) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
+  if (swa) {
+    if (swa->window < 1 || !swa->k_swa || !swa->v_swa || !swa->gamma) return HS_ERR_INVALID_ARG;
+    if (!aligned16(swa->k_swa) || !aligned16(swa->v_swa) || (swa->o_sparse && !aligned16(swa->o_sparse)))
+      return HS_ERR_INVALID_ARG;
+  }
   if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
@@ -591,7 +607,10 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   } else if (!make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B)) {
     return HS_ERR_CUDA;
   }
-  m.g = m.o = m.q;
+  m.g = m.o = m.ks = m.vs = m.q;
+  if (swa && (!make_map_3d(&m.ks, swa->k_swa, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
+              !make_map_3d(&m.vs, swa->v_swa, sh.d, sh.Hkv, sh.Tkv, 1, 128)))
+    return HS_ERR_CUDA;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -613,7 +632,25 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
   p.topk = sel->topk;
   p.w = sel->window;
   p.wc = wait_ctl(ws);
+  if (swa) {
+    p.ws = swa->window;
+    p.gamma = swa->gamma;
+    p.o_mid = reinterpret_cast<__nv_bfloat16*>(swa->o_sparse);
+    // the final output goes through the smem buffer by TMA in 64-row rounds of whole queries (G | 64)
+    p.o_tma = sh.G <= 64 && make_map_3d(&m.o, o, sh.d, sh.Hq, sh.Tq, sh.G, 64 / sh.G);
+  }
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
+  if (swa) {
+    switch (B) {
+      case 1: return dispatch_attn_d<attn::kFused, 1>(sh.d, m, p, sc, grid, S(stream));
+      case 8: return dispatch_attn_d<attn::kFused, 8>(sh.d, m, p, sc, grid, S(stream));
+      case 16: return dispatch_attn_d<attn::kFused, 16>(sh.d, m, p, sc, grid, S(stream));
+      case 32: return dispatch_attn_d<attn::kFused, 32>(sh.d, m, p, sc, grid, S(stream));
+      case 64: return dispatch_attn_d<attn::kFused, 64>(sh.d, m, p, sc, grid, S(stream));
+      case 128: return dispatch_attn_d<attn::kFused, 128>(sh.d, m, p, sc, grid, S(stream));
+      default: return HS_ERR_UNSUPPORTED;
+    }
+  }
   switch (B) {
     case 1: return dispatch_attn_d<attn::kSparse, 1>(sh.d, m, p, sc, grid, S(stream));
     case 8: return dispatch_attn_d<attn::kSparse, 8>(sh.d, m, p, sc, grid, S(stream));
@@ -623,6 +660,21 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
     case 128: return dispatch_attn_d<attn::kSparse, 128>(sh.d, m, p, sc, grid, S(stream));
     default: return HS_ERR_UNSUPPORTED;
   }
+}
+
+hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                                 void* ws, size_t ws_bytes, hs_stream_t stream) {
+  return sparse_layer(vl, sel, q, k, v, idx, cnt, o, lse, nullptr, ws, ws_bytes, stream);
+}
+
+hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                      const void* v, const int32_t* idx, const int32_t* cnt, int32_t swa_window,
+                                      const void* k_swa, const void* v_swa, const float* gamma, void* o,
+                                      void* o_sparse, float* lse_sparse, void* ws, size_t ws_bytes,
+                                      hs_stream_t stream) {
+  const SwaArgs swa{swa_window, k_swa, v_swa, gamma, o_sparse};
+  return sparse_layer(vl, sel, q, k, v, idx, cnt, o, lse_sparse, &swa, ws, ws_bytes, stream);
 }
 
 hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const void* q, hs_kv_dtype kv_dtype,
@@ -714,7 +766,7 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
-  m.g = m.o = m.q;
+  m.g = m.o = m.ks = m.vs = m.q;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);
@@ -777,7 +829,7 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
     return HS_ERR_CUDA;
   m.kb = m.k;
   m.vb = m.v;
-  m.g = m.o = m.q;
+  m.g = m.o = m.ks = m.vs = m.q;
   static attn::Sched sc;
   static std::mutex mu;
   std::lock_guard<std::mutex> lock(mu);

@@ -51,7 +51,10 @@ constexpr int kMaxItemRows = 256;
 #endif
 constexpr int kPolyPairs = HS_EXP2_POLY_PAIRS;
 
-enum Mode : int { kFull = 0, kSparse = 1 };
+// kFused: a whole HySparse sparse layer in one pass -- the selected blocks /
+// tokens (+ forced window) of the shared cache, then the sliding-window branch
+// over the layer's own K_swa / V_swa, then the sigmoid gate.
+enum Mode : int { kFull = 0, kSparse = 1, kFused = 2 };
 
 // One work item: up to 256 rows (whole queries x the KV head's group) of one
 // sequence and one KV head.
@@ -102,6 +105,9 @@ struct Params {
   const float* gamma;                // [Tq, Hq] or null
   const __nv_bfloat16* o_other;      // [Tq, Hq, D] sparse-branch output
   int o_tma;                         // gated call: o_other / o move through smem by TMA (64 % G == 0)
+  // fused sparse layer: SWA window over K_swa / V_swa, optional o_sparse output
+  int ws;
+  __nv_bfloat16* o_mid;              // [Tq, Hq, D] sparse-branch output or null (lse_sparse goes to lse)
   WaitCtl wc;
 };
 
@@ -185,6 +191,10 @@ struct KvPlan {
   int n_win;  // window tiles (sparse, w > 0)
   int win_lo; // first window key (position)
   int cnt;    // selected blocks
+  int n_swa;  // fused sparse layer: tiles of the own-cache sliding window
+  int swa_lo; // its first key (position)
+  __device__ __forceinline__ int n1() const { return n_sel + n_win; }  // tiles of the shared cache
+  __device__ __forceinline__ int total() const { return n_sel + n_win + n_swa; }
 };
 
 __device__ __forceinline__ KvPlan kv_plan(const Params& p, const Item& it, int mode) {
@@ -201,6 +211,10 @@ __device__ __forceinline__ KvPlan kv_plan(const Params& p, const Item& it, int m
       k.win_lo = max(0, it.pos0 - p.w + 1);
       k.n_win = (last_pos - k.win_lo + 1 + 127) / 128;
     }
+    if (mode == kFused) {
+      k.swa_lo = max(0, it.pos0 - p.ws + 1);
+      k.n_swa = (last_pos - k.swa_lo + 1 + 127) / 128;
+    }
   }
   return k;
 }
@@ -213,11 +227,16 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kb,
                     const __grid_constant__ CUtensorMap map_vb, const __grid_constant__ CUtensorMap map_g,
-                    const __grid_constant__ CUtensorMap map_o, const Params p,
+                    const __grid_constant__ CUtensorMap map_o, const __grid_constant__ CUtensorMap map_ks,
+                    const __grid_constant__ CUtensorMap map_vs, const Params p,
                     const __grid_constant__ Sched sc) {
-  // the window-only instantiation serves the gated sliding-window call
+  // the window-only instantiation serves the gated sliding-window call; the
+  // fused sparse layer computes its gate input itself
   constexpr bool kGate = (MODE == kSparse && SB == 0);
-  using L = Layout<D, kGate>;
+  constexpr bool kFuse = (MODE == kFused);
+  constexpr bool kBuf = kGate || kFuse;  // 256-row output buffer + gate epilogue
+  constexpr bool kSp = (MODE != kFull);
+  using L = Layout<D, kBuf>;
   constexpr int kNS = L::kNStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -258,13 +277,17 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     prefetch_tensormap(&map_q);
     prefetch_tensormap(&map_k);
     prefetch_tensormap(&map_v);
-    if (MODE == kSparse) {
+    if (kSp) {
       prefetch_tensormap(&map_kb);
       prefetch_tensormap(&map_vb);
     }
-    if (kGate && p.o_tma) {
+    if (kBuf && p.o_tma) {
       prefetch_tensormap(&map_g);
       prefetch_tensormap(&map_o);
+    }
+    if (kFuse) {
+      prefetch_tensormap(&map_ks);
+      prefetch_tensormap(&map_vs);
     }
   }
   tc_fence_before();
@@ -292,7 +315,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
-      const int n = kp.n_sel + kp.n_win;
+      const int n = kp.total();
       if (n == 0) continue;
       const int rows = it.nq * p.G;
       const int n_qt = rows > 128 ? 2 : 1;
@@ -305,7 +328,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
                         it.g * p.G, it.qrow0 + t * (128 / p.G));
       }
       ++q_uses;
-      const int* idx_row = (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
+      const int* idx_row = kSp ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
       for (int i = 0; i < n && ok; ++i) {
         for (int kind = 0; kind < 2; ++kind) {
           const int s = ctr % kNS;
@@ -315,10 +338,16 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           uint8_t* dst = smem + L::kOffKV + s * L::kTileBytes;
           const CUtensorMap* mt = kind == 0 ? &map_k : &map_v;
           if (MODE == kFull || i >= kp.n_sel) {
-            const int key0 = (MODE == kFull) ? i * 128 : kp.win_lo + (i - kp.n_sel) * 128;
+            // contiguous 128-key tiles: causal (full), forced window, or the
+            // fused layer's own-cache sliding window
+            const bool own = kFuse && i >= kp.n1();
+            const int key0 = (MODE == kFull) ? i * 128
+                             : own ? kp.swa_lo + (i - kp.n1()) * 128
+                                   : kp.win_lo + (i - kp.n_sel) * 128;
+            const CUtensorMap* mc = own ? (kind == 0 ? &map_ks : &map_vs) : mt;
             if (lane == 0)
               for (int sl = 0; sl < L::kSlabs; ++sl)
-                tma_load_3d(dst + sl * kSlabBytes, mt, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
+                tma_load_3d(dst + sl * kSlabBytes, mc, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
           } else {
             const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
             if constexpr (SB == 1) {
@@ -375,7 +404,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         const Item it = get_item<MODE>(p, sc, wi);
         if (it.nq <= 0) continue;
         const KvPlan kp = kv_plan(p, it, MODE);
-        const int n = kp.n_sel + kp.n_win;
+        const int n = kp.total();
         if (n == 0) continue;
         const int n_qt = it.nq * p.G > 128 ? 2 : 1;
         if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10, wi << 12)) { ok = false; break; }
@@ -423,7 +452,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
             if (i == 0 && items_t[t] > 0 &&
                 !mbar_wait(&c.o_free[t], (items_t[t] - 1) & 1, abort_flag, p.wc, 14)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, sv, i > 0);
+            issue_pv(t, sv, i > 0 && !(kFuse && i == kp.n1()));  // fused: the SWA branch starts a fresh O
             if (i + 1 < n) {
               if (sk_next < 0) {
                 sk_next = ctr % kNS;
@@ -474,7 +503,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
-      const int n = kp.n_sel + kp.n_win;
+      const int n = kp.total();
       const int rows = it.nq * p.G;
       const bool active = (t == 0) || rows > 128;
       const bool valid = vr < rows;
@@ -485,7 +514,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       float m_used = -INFINITY, l = 0.f;
       const int par = sc_items & 1;  // spill buffer of this item (full mode with scores)
       float sg = 0.f;                // gate of this row (gated call)
-      if constexpr (kGate) {
+      if constexpr (kBuf) {
         if (p.gamma && valid) sg = 1.f / (1.f + __expf(-__ldg(p.gamma + size_t(qrow) * p.Hq + h)));
       }
       if constexpr (MODE == kFull && SB > 0) {
@@ -509,10 +538,50 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           }
         }
         const int* idx_row =
-            (MODE == kSparse) ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
+            kSp ? p.idx + (size_t(it.tile0) * p.Hkv + it.g) * p.topk : nullptr;
         for (int i = 0; i < n; ++i) {
           if (!mbar_wait_warp(&c.s_full[t], (uses + i) & 1, abort_flag, p.wc, 20, (wi << 12) | i)) { ok = false; break; }
           tc_fence_after();
+          if constexpr (kFuse) {
+            if (i == kp.n1()) {
+              // The shared-cache phase is complete: this S was committed after
+              // its last PV. o_sparse = O / l goes to this row's slot of the
+              // output buffer (and to o_mid if asked), lse_sparse to lse; the
+              // sliding-window branch then starts from an empty softmax state
+              // (its first PV overwrites O).
+              const float inv = l > 0.f ? 1.f / l : 0.f;
+              const int rr = vr - (t * 128 + (quad >> 1) * 64);
+              uint8_t* rbuf = o_buf + (quad >> 1) * L::kRound + rr * 128;
+              uint4* mid = (p.o_mid && valid) ? reinterpret_cast<uint4*>(p.o_mid + (size_t(qrow) * p.Hq + h) * D)
+                                              : nullptr;
+#pragma unroll
+              for (int ch = 0; ch < D / 32; ++ch) {
+                uint32_t ov[32];
+                if (i > 0) {
+                  tmem_ld32(t_o + ch * 32, ov);
+                  tmem_ld_wait();
+                } else {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) ov[j] = 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const uint4 res = make_uint4(
+                      pack_bf16(__uint_as_float(ov[8 * j + 0]) * inv, __uint_as_float(ov[8 * j + 1]) * inv),
+                      pack_bf16(__uint_as_float(ov[8 * j + 2]) * inv, __uint_as_float(ov[8 * j + 3]) * inv),
+                      pack_bf16(__uint_as_float(ov[8 * j + 4]) * inv, __uint_as_float(ov[8 * j + 5]) * inv),
+                      pack_bf16(__uint_as_float(ov[8 * j + 6]) * inv, __uint_as_float(ov[8 * j + 7]) * inv));
+                  *reinterpret_cast<uint4*>(rbuf + (ch >> 1) * (64 * 128) + ((((ch & 1) * 4 + j) ^ (rr & 7)) << 4)) =
+                      res;
+                  if (mid) mid[ch * 4 + j] = res;
+                }
+              }
+              if (valid && p.lse)
+                p.lse[size_t(h) * p.Tq + qrow] = (l > 0.f ? m_used + __log2f(l) : -INFINITY) * 0.69314718055994531f;
+              m_used = -INFINITY;
+              l = 0.f;
+            }
+          }
           uint32_t u[128];
           tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
           tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
@@ -569,8 +638,10 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
               }
             }
           } else {
-            const int key0 = kp.win_lo + (i - kp.n_sel) * 128;
-            const int lo = pos - p.w + 1;
+            // forced window of the shared cache, or the fused layer's own window
+            const bool own = kFuse && i >= kp.n1();
+            const int key0 = own ? kp.swa_lo + (i - kp.n1()) * 128 : kp.win_lo + (i - kp.n_sel) * 128;
+            const int lo = pos - (own ? p.ws : p.w) + 1;
 #pragma unroll
             for (int j = 0; j < 128; ++j) {
               const int key = key0 + j;
@@ -634,8 +705,9 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           // the P buffer and O may be touched without waiting on o_ready.
           // tcgen05.ld/st are warp-collective: rescale the whole warp's rows
           // together (rows that keep their max use factor 1).
-          if (__any_sync(0xffffffffu, rescale && i > 0)) {
-            const float f = (rescale && i > 0) ? factor : 1.f;
+          const int i0 = (kFuse && i >= kp.n1()) ? kp.n1() : 0;  // first tile of this softmax
+          if (__any_sync(0xffffffffu, rescale && i > i0)) {
+            const float f = (rescale && i > i0) ? factor : 1.f;
 #pragma unroll
             for (int ch = 0; ch < D / 32; ++ch) {
               uint32_t ov[32];
@@ -657,13 +729,15 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           tc_fence_after();
           const float inv = l > 0.f ? 1.f / l : 0.f;
           __nv_bfloat16* orow = p.o + (size_t(qrow) * p.Hq + h) * D;
-          if constexpr (kGate) {
-            // o = sig(gamma) o_other + (1 - sig(gamma)) o_this. With o_tma the
-            // other branch's rows sit in this warpgroup's buffer in the TMA
-            // box layout; each thread overwrites its row in place and one
-            // thread stores the full 64-row rounds (partial ones go direct).
+          if constexpr (kBuf) {
+            // o = sig(gamma) o_other + (1 - sig(gamma)) o_this. The other
+            // branch's rows sit in this warpgroup's buffer in the TMA box
+            // layout (gated call with o_tma: loaded by TMA at item start; fused
+            // layer: written by this thread at the phase switch); each thread
+            // overwrites its row in place and one thread stores the full
+            // 64-row rounds (partial ones go direct).
             const bool gate = p.gamma != nullptr;
-            if (p.o_tma && gate && ok) {
+            if (kGate && p.o_tma && gate && ok) {
               if (mbar_wait_warp(&c.g_full[t], g_uses & 1, abort_flag, p.wc, 23, wi << 12)) ++g_uses;
               else ok = false;
             }
@@ -688,7 +762,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
 #pragma unroll
                   for (int e = 0; e < 8; ++e) of[e] = __uint_as_float(ov[8 * j + e]) * inv;
                   if (gate && valid) {
-                    const uint4 u4 = p.o_tma ? *chunk : __ldg(src + ch * 4 + j);
+                    const uint4 u4 = (kFuse || p.o_tma) ? *chunk : __ldg(src + ch * 4 + j);
                     const uint32_t w4[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -719,6 +793,9 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
                 bulk_commit();
                 bulk_wait_read0();  // the buffer may be refilled once the stores have read it
               }
+              // fused layer: the whole warpgroup refills the buffer at the next
+              // phase switch, so every warp waits for the stores' reads
+              if (kFuse && !wg_sync()) ok = false;
             }
           } else {
 #pragma unroll
@@ -754,7 +831,8 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         }
       }
       const float lse2 = (l > 0.f) ? m_used + __log2f(l) : -INFINITY;
-      if (valid && active && p.lse) p.lse[size_t(h) * p.Tq + qrow] = lse2 * 0.69314718055994531f;
+      // (the fused layer reports the sparse branch's lse, written at its phase switch)
+      if (!kFuse && valid && active && p.lse) p.lse[size_t(h) * p.Tq + qrow] = lse2 * 0.69314718055994531f;
       if (valid && n == 0 && p.lse) p.lse[size_t(h) * p.Tq + qrow] = -INFINITY;
       // ---- hand the item's lse to the score warps (full mode, B > 1) ----
       if constexpr (MODE == kFull && SB > 0) {
@@ -768,7 +846,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         ++sc_items;
       }
     }
-    if constexpr (kGate) {
+    if constexpr (kBuf) {
       // never leave with TMA traffic on this warpgroup's buffer in flight
       if (quad == 0 && lane == 0) {
         if (g_issued > g_uses) mbar_wait_drain(&c.g_full[t], (g_issued - 1) & 1, p.wc, 93);
@@ -788,7 +866,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
-      const int n = kp.n_sel + kp.n_win;
+      const int n = kp.total();
       if (!mbar_wait_warp(&c.sc_ready, sc_items & 1, abort_flag, p.wc, 40, wi << 12)) break;
       float l2[4];
 #pragma unroll

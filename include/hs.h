@@ -89,7 +89,8 @@ typedef enum {
   HS_OP_TOPK_SELECT = 1,
   HS_OP_SPARSE_ATTN_PREFILL = 2,
   HS_OP_SPARSE_ATTN_DECODE = 3,
-  HS_OP_SWA_GATED = 4
+  HS_OP_SWA_GATED = 4,
+  HS_OP_SPARSE_SWA_GATED_PREFILL = 5
 } hs_op;
 
 /* Bytes of workspace that `op` needs for these shapes (0 on invalid input).
@@ -209,6 +210,29 @@ HS_API hs_status hs_swa_gated(const hs_varlen* vl, int32_t window,
                        const void* q, const void* k_swa, const void* v_swa,
                        const float* gamma, const void* o_sparse, void* o,
                        void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
+ * hs_sparse_swa_gated_prefill -- a whole HySparse sparse layer in one launch:
+ * the block-sparse global branch of hs_sparse_attn_prefill, the sliding-window
+ * branch of hs_swa_gated over the layer's own K_swa / V_swa, and the sigmoid
+ * gate (QbitAI repost: each sparse layer has the two branches, fused by a
+ * sigmoid gate; HySparse explainer: the window branch keeps its own cache):
+ *   o = sigmoid(gamma) * o_sparse + (1 - sigmoid(gamma)) * o_swa.
+ * Results equal hs_sparse_attn_prefill followed by hs_swa_gated, except that
+ * the gate mixes the fp32 window output with o_sparse rounded to bf16 once
+ * (as the two-call path does) without o_sparse passing through HBM.
+ * In: q [T_q,H_q,d]; k/v (full layer's) [T_kv,H_kv,d]; idx/cnt from
+ * hs_topk_select; swa_window >= 1; k_swa/v_swa [T_kv,H_kv,d] bf16;
+ * gamma [T_q,H_q] fp32.
+ * Out: o [T_q,H_q,d] bf16; o_sparse [T_q,H_q,d] bf16 and lse_sparse [H_q,T_q]
+ * fp32 of the sparse branch, each optional (NULL skips the write).
+ */
+HS_API hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* sel,
+                                      const void* q, const void* k, const void* v,
+                                      const int32_t* idx, const int32_t* cnt,
+                                      int32_t swa_window, const void* k_swa, const void* v_swa,
+                                      const float* gamma, void* o, void* o_sparse, float* lse_sparse,
+                                      void* ws, size_t ws_bytes, hs_stream_t stream);
 
 /*
  * hs_full_attn_select_noalloc -- hs_full_attn_select for callers that cannot

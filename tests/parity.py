@@ -95,19 +95,20 @@ def assert_indices_match(idx_g, cnt_g, scores_o, idx_o, cnt_o, tiles, k):
 class GpuBlock:
     """Runs one hybrid block through the library's public block runner."""
 
-    def __init__(self, w, inp, device="cuda"):
+    def __init__(self, w, inp, device="cuda", fused=True):
         import hybrid_sparse_attention_tma_b200 as hs
         from hybrid_sparse_attention_tma_b200.block import HybridBlock, SparseLayerIn
         self.w = w
         self.inp = inp
         self.vl = hs.Varlen(w.cu_q(), w.cu_kv(), w.n_q_heads, w.n_kv_heads, w.head_dim, device=device)
         self.sel = hs.Sel(w.q_tile, w.block, w.topk, w.window)
-        self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device)
+        self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device,
+                                 fused=fused)
         self.layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
 
-    def run(self, stream=None, fp8=False):
+    def run(self, stream=None, fp8=False, intermediates=True):
         fp8_kv = None
         if fp8:
             fp8_kv = (self.inp.k_fp8, self.inp.v_fp8, self.inp.k_scale, self.inp.v_scale)
         return self.block.forward(self.inp.q, self.inp.k, self.inp.v, self.layers, stream=stream, keep_all=True,
-                                  fp8_kv=fp8_kv)
+                                  fp8_kv=fp8_kv, intermediates=intermediates)

@@ -89,13 +89,13 @@ def check_block(w, inp, res, tile_ids=None, fp8=False):
             assert_close_out(o_l, O.gated_merge(gamma, o_sp, o_swa), what=f"layer {li} chain o")
 
 
-def run_and_check(w, seed=None, tile_ids=None, fp8=False):
+def run_and_check(w, seed=None, tile_ids=None, fp8=False, fused=True):
     import sys, time
     t0 = time.time()
     inp = W.make_block_inputs(w, device="cuda", seed=seed)
     torch.cuda.synchronize()
     t1 = time.time()
-    res = GpuBlock(w, inp).run(fp8=fp8)
+    res = GpuBlock(w, inp, fused=fused).run(fp8=fp8)
     torch.cuda.synchronize()
     t2 = time.time()
     check_block(w, inp, res, tile_ids, fp8=fp8)
@@ -142,6 +142,24 @@ VARIANTS = {
 @pytest.mark.parametrize("name", list(VARIANTS))
 def test_variant_whole(name):
     run_and_check(VARIANTS[name], seed=7)
+
+
+def test_swa_gate_two_call_path():
+    """The unfused layer (hs_sparse_attn_prefill then hs_swa_gated) against the oracle."""
+    run_and_check(VARIANTS["swa_gate"], seed=7, fused=False)
+
+
+def test_fused_layer_without_intermediates_writes_the_same_output():
+    """o_sparse / lse_sparse are optional outputs of the fused layer: leaving
+    them out changes no bit of o."""
+    w = VARIANTS["swa_gate"]
+    inp = W.make_block_inputs(w, device="cuda", seed=9)
+    blk = GpuBlock(w, inp)
+    a = [L["o"].clone() for L in blk.run()["layers"]]
+    b = blk.run(intermediates=False)["layers"]
+    for x, y in zip(a, b):
+        assert y["o_sparse"] is None and y["lse_sparse"] is None
+        assert torch.equal(x, y["o"])
 
 
 def test_k_all_equals_full_attention_on_gpu():
