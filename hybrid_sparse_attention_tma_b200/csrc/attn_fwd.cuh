@@ -14,7 +14,9 @@
 //   warps 0-3  softmax warpgroup for Q-tile 0 (128 rows = TMEM lanes)
 //   warps 4-7  softmax warpgroup for Q-tile 1
 //   warp  8    TMA producer (Q tiles, K/V tiles or gathered blocks)
-//   warp  9    UMMA issuer (one thread) + TMEM owner
+//   warp  9    UMMA issuer (one thread) + TMEM owner; the gated window-only
+//              call issues Q-tile 1's MMAs from warp 10
+//   warps 10-11 score warps (full layer with block scores only)
 // A work item is up to 256 "rows" of one sequence and one KV head g; row
 // r = query * G + head-in-group, so every Q-tile holds whole queries and the
 // group's heads share each K/V tile (GQA/MQA packing into the MMA M dim).
@@ -23,10 +25,11 @@
 // and the PV MMA reads its A operand from there.
 // SMEM: Q[2] | K/V ring[5] | control. All operand tiles use the 128-byte
 // swizzle (8-row x 128-byte atoms), K-major except V (MN-major). The gated
-// sliding-window instantiation runs a 3-stage ring and spends the freed space
-// on a 256-row output buffer: the softmax warpgroups TMA-load the other
-// branch's output into it when an item starts, mix their result in place and
-// TMA-store it.
+// sliding-window instantiation and the fused sparse layer run a 3-stage ring
+// and spend the freed space on a 256-row output buffer that holds the other
+// branch's output (TMA-loaded when an item starts, or written at the fused
+// layer's switch to its window branch); the epilogue mixes in place and
+// TMA-stores it.
 #pragma once
 
 #include "hs_common.cuh"
@@ -34,12 +37,22 @@
 namespace hs {
 namespace attn {
 
-constexpr int kThreads = 320;
-// The full layer with block scores adds two warps (10, 11) that reduce each
-// work item's spilled block maxima while the softmax warps move on.
+// Warps 0-7 softmax, 8 TMA producer, 9 UMMA issuer. The window-only gated
+// call and the fused sparse layer (short items, an epilogue each) give each
+// Q-tile its own issuer (warps 9, 10) so that one tile's wait never delays
+// the other's MMAs at item boundaries; with long items one issuer in the
+// order PV_0 QK_0 PV_1 QK_1 keeps the two softmax warpgroups out of phase,
+// which overlaps one's softmax with the other's MMAs (measured: the full and
+// plain sparse layers are faster with one issuer, these two with two). The
+// full layer with block scores adds warps 10-11, which reduce each work
+// item's spilled block maxima while the softmax warps move on.
+template <int MODE, int SB>
+constexpr bool two_issuers() {
+  return (MODE == 1 && SB == 0) || MODE == 2;
+}
 template <int MODE, int SB>
 constexpr int threads_for() {
-  return (MODE == 0 && SB > 0) ? 384 : 320;
+  return (MODE == 0 && SB > 0) ? 384 : two_issuers<MODE, SB>() ? 352 : 320;
 }
 constexpr int kStages = 5;
 constexpr int kSlabBytes = 128 * 128;  // 128 rows x 64 bf16
@@ -127,7 +140,7 @@ struct Ctl {
   uint64_t q_full, q_empty;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], p_full[2], o_ready[2], o_free[2];
-  uint64_t teardown;
+  uint64_t teardown[2];  // per UMMA issuer
   uint64_t wg_bar[2];   // per softmax warpgroup: bounded barrier of its 4 warps
   uint64_t g_full[2];   // per softmax warpgroup: other-branch output landed (gated call)
   uint64_t sc_ready;    // softmax warps: item's spill + lse2 written (count 8)
@@ -236,6 +249,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
   constexpr bool kFuse = (MODE == kFused);
   constexpr bool kBuf = kGate || kFuse;  // 256-row output buffer + gate epilogue
   constexpr bool kSp = (MODE != kFull);
+  constexpr int kIssuers = two_issuers<MODE, SB>() ? 2 : 1;
   using L = Layout<D, kBuf>;
   constexpr int kNS = L::kNStages;
   extern __shared__ uint8_t smem_raw[];
@@ -246,10 +260,10 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&c.q_full, 1);
-    mbar_init(&c.q_empty, 1);
+    mbar_init(&c.q_empty, kIssuers);  // released by every UMMA issuer
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&c.kv_full[s], 1);
-      mbar_init(&c.kv_empty[s], 1);
+      mbar_init(&c.kv_empty[s], kIssuers);
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&c.s_full[t], 1);
@@ -257,8 +271,8 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       mbar_init(&c.o_ready[t], 1);
       mbar_init(&c.o_free[t], 4);
     }
-    mbar_init(&c.teardown, 1);
     for (int t = 0; t < 2; ++t) {
+      mbar_init(&c.teardown[t], 1);
       mbar_init(&c.wg_bar[t], 4);
       mbar_init(&c.g_full[t], 1);
     }
@@ -388,18 +402,58 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kNS) & 1, p.wc, 90);
       if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 91);
     }
-  } else if (warp == 9) {
-    // ===================== UMMA issuer =====================
+  } else if (warp == 9 || (kIssuers == 2 && warp == 10)) {
+    // ===================== UMMA issuer(s) =====================
+    // One issuer walks both Q-tiles (t = 0, 1) or, with two issuers, warp
+    // 9 + t owns Q-tile t. Every issuer walks the same K/V ring and releases
+    // each stage and Q with its own commit (barrier count = issuers); an
+    // issuer whose Q-tile has no rows in an item only waits for the loads and
+    // arrives, so the ring phases stay in step.
+    const int t_lo = kIssuers == 2 ? warp - 9 : 0;
+    const int t_hi = kIssuers == 2 ? warp - 9 : 1;
     if (lane == 0) {
       constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, false, true);
       int ctr = 0, q_uses = 0;
-      int uses[2] = {0, 0};        // S/P/O phases per Q-tile
-      int items_t[2] = {0, 0};     // items in which tile t took part (o_free phase)
+      int uses[2] = {0, 0};     // S/P/O phases per Q-tile
+      int items_t[2] = {0, 0};  // items in which tile t took part (o_free phase)
       bool ok = true;
+      // Descriptors are built once; a K step only adds its byte offset / 16
+      // to the 14-bit start-address field (no carry: smem < 256 KB).
       const uint64_t q_desc0 = sdesc_sw128(smem_u32(smem + L::kOffQ), 16, 1024);
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(smem + L::kOffKV), 16, 1024);
       const uint64_t v_desc0 = sdesc_sw128(smem_u32(smem + L::kOffKV), kSlabBytes, 1024);
+      auto issue_qk = [&](int t, int stage) {
+        const uint32_t d_tmem = tmem + t * 256;
+        const uint64_t qd = q_desc0 + uint64_t((t * L::kTileBytes) >> 4);
+        const uint64_t kd = k_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
+          umma_bf16(d_tmem, qd + off, kd + off, kIdQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&c.s_full[t]);
+      };
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t d_tmem = tmem + t * 256 + 128;
+        const uint32_t pa = tmem + t * 256;  // P_t over the first 64 columns of S_t
+        const uint64_t vd = v_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
+        umma_bf16_ts(d_tmem, pa, vd, kIdPV, acc ? 1u : 0u);
+#pragma unroll
+        for (int kk = 1; kk < 8; ++kk) umma_bf16_ts(d_tmem, pa + kk * 8, vd + uint64_t(kk * (2048 >> 4)), kIdPV, 1u);
+        umma_commit(&c.o_ready[t]);
+      };
+      // release a K/V stage / Q: by commit after this issuer's MMAs, or at once
+      auto release = [&](uint64_t* bar, bool issued) {
+        if (issued) umma_commit(bar);
+        else mbar_arrive(bar);
+      };
+      auto wait_kv = [&](int site, int ctx) -> int {
+        const int s = ctr % kNS;
+        if (!mbar_wait(&c.kv_full[s], (ctr / kNS) & 1, abort_flag, p.wc, site, ctx)) return -1;
+        ++ctr;
+        return s;
+      };
       for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
         const Item it = get_item<MODE>(p, sc, wi);
         if (it.nq <= 0) continue;
@@ -407,47 +461,23 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         const int n = kp.total();
         if (n == 0) continue;
         const int n_qt = it.nq * p.G > 128 ? 2 : 1;
+        const int t_end = min(t_hi, n_qt - 1);  // last Q-tile of this issuer with rows in the item
+        const bool mine = t_lo <= t_end;
         if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 10, wi << 12)) { ok = false; break; }
         ++q_uses;
         tc_fence_after();
-        // Descriptors are built once; a K step only adds its byte offset / 16
-        // to the 14-bit start-address field (no carry: smem < 256 KB). Keeping
-        // the issuing thread's work per MMA to an add lets the tensor pipe run
-        // back to back (a 128x128x16 MMA takes 64 cycles).
-        auto issue_qk = [&](int t, int stage) {
-          const uint32_t d_tmem = tmem + t * 256;
-          const uint64_t qd = q_desc0 + uint64_t((t * L::kTileBytes) >> 4);
-          const uint64_t kd = k_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
-            umma_bf16(d_tmem, qd + off, kd + off, kIdQK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&c.s_full[t]);
-        };
-        auto issue_pv = [&](int t, int stage, bool acc) {
-          const uint32_t d_tmem = tmem + t * 256 + 128;
-          const uint32_t pa = tmem + t * 256;  // P_t over the first 64 columns of S_t
-          const uint64_t vd = v_desc0 + uint64_t((stage * L::kTileBytes) >> 4);
-          umma_bf16_ts(d_tmem, pa, vd, kIdPV, acc ? 1u : 0u);
-#pragma unroll
-          for (int kk = 1; kk < 8; ++kk) umma_bf16_ts(d_tmem, pa + kk * 8, vd + uint64_t(kk * (2048 >> 4)), kIdPV, 1u);
-          umma_commit(&c.o_ready[t]);
-        };
         // prologue: S_t(0)
-        int sk = ctr % kNS;
-        if (!mbar_wait(&c.kv_full[sk], (ctr / kNS) & 1, abort_flag, p.wc, 11, wi << 12)) { ok = false; break; }
-        ++ctr;
+        const int sk = wait_kv(11, wi << 12);
+        if (sk < 0) { ok = false; break; }
         tc_fence_after();
-        for (int t = 0; t < n_qt; ++t) issue_qk(t, sk);
-        umma_commit(&c.kv_empty[sk]);
-        if (n == 1) umma_commit(&c.q_empty);  // Q is only read by QK: free it early
+        for (int t = t_lo; t <= t_end; ++t) issue_qk(t, sk);
+        release(&c.kv_empty[sk], mine);
+        if (n == 1) release(&c.q_empty, mine);  // Q is only read by QK: free it early
         for (int i = 0; i < n && ok; ++i) {
-          const int sv = ctr % kNS;
-          if (!mbar_wait(&c.kv_full[sv], (ctr / kNS) & 1, abort_flag, p.wc, 12, (wi << 12) | i)) { ok = false; break; }
-          ++ctr;
+          const int sv = wait_kv(12, (wi << 12) | i);
+          if (sv < 0) { ok = false; break; }
           int sk_next = -1;
-          for (int t = 0; t < n_qt; ++t) {
+          for (int t = t_lo; t <= t_end; ++t) {
             if (!mbar_wait(&c.p_full[t], (uses[t] + i) & 1, abort_flag, p.wc, 13, (wi << 12) | i)) { ok = false; break; }
             if (i == 0 && items_t[t] > 0 &&
                 !mbar_wait(&c.o_free[t], (items_t[t] - 1) & 1, abort_flag, p.wc, 14)) { ok = false; break; }
@@ -455,28 +485,31 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
             issue_pv(t, sv, i > 0 && !(kFuse && i == kp.n1()));  // fused: the SWA branch starts a fresh O
             if (i + 1 < n) {
               if (sk_next < 0) {
-                sk_next = ctr % kNS;
-                if (!mbar_wait(&c.kv_full[sk_next], (ctr / kNS) & 1, abort_flag, p.wc, 15, (wi << 12) | i)) { ok = false; break; }
-                ++ctr;
+                sk_next = wait_kv(15, (wi << 12) | i);
+                if (sk_next < 0) { ok = false; break; }
                 tc_fence_after();
               }
               issue_qk(t, sk_next);
             }
           }
           if (!ok) break;
-          umma_commit(&c.kv_empty[sv]);
-          if (sk_next >= 0) umma_commit(&c.kv_empty[sk_next]);
-          if (i + 2 == n) umma_commit(&c.q_empty);  // last QK of the item issued
+          if (i + 1 < n && sk_next < 0) {  // an issuer without rows still takes the next K stage
+            sk_next = wait_kv(15, (wi << 12) | i);
+            if (sk_next < 0) { ok = false; break; }
+          }
+          release(&c.kv_empty[sv], mine);
+          if (sk_next >= 0) release(&c.kv_empty[sk_next], mine);
+          if (i + 2 == n) release(&c.q_empty, mine);  // last QK of the item issued
         }
         if (!ok) break;
-        for (int t = 0; t < n_qt; ++t) {
+        for (int t = t_lo; t <= t_end; ++t) {
           uses[t] += n;
           items_t[t] += 1;
         }
       }
-      // make sure no tensor-core op is still writing TMEM before teardown
-      umma_commit(&c.teardown);
-      mbar_wait_drain(&c.teardown, 0, p.wc, 92);
+      // make sure no tensor-core op of this issuer is still writing TMEM before teardown
+      umma_commit(&c.teardown[t_lo]);
+      mbar_wait_drain(&c.teardown[t_lo], 0, p.wc, 92);
     }
   } else if (warp < 8) {
     // ===================== softmax warpgroups =====================
@@ -834,7 +867,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       // (the fused layer reports the sparse branch's lse, written at its phase switch)
       if (!kFuse && valid && active && p.lse) p.lse[size_t(h) * p.Tq + qrow] = lse2 * 0.69314718055994531f;
       if (valid && n == 0 && p.lse) p.lse[size_t(h) * p.Tq + qrow] = -INFINITY;
-      // ---- hand the item's lse to the score warps (full mode, B > 1) ----
+      // ---- hand the item's lse to the score warp (full mode, B > 1) ----
       if constexpr (MODE == kFull && SB > 0) {
         if (sc_items >= 1 && ok &&
             !mbar_wait_warp(&c.lse_taken, (sc_items - 1) & 1, abort_flag, p.wc, 32, wi << 12))
@@ -858,8 +891,9 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     // score(t, g, b) = max over the tile's rows r of exp2(m_{r,b} - lse2_r):
     // the per-row block maxima m were spilled during the main loop; with the
     // final lse2 known they are reduced here, off the softmax critical path.
-    const int wq = warp - 10;                 // rows [128 wq, 128 wq + 128)
-    const int r0 = wq * 128 + lane * 4;       // this lane's 4 rows
+    // Warp 10 + wq owns the item's rows [128 wq, 128 wq + 128); lane l owns
+    // rows 4l..4l+3 of that half.
+    const int wq = warp - 10;
     int sc_items = 0;
     if constexpr (MODE == kFull && SB > 0)
     for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
@@ -870,31 +904,40 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       if (!mbar_wait_warp(&c.sc_ready, sc_items & 1, abort_flag, p.wc, 40, wi << 12)) break;
       float l2[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) l2[e] = c.lse2[r0 + e];
+      for (int e = 0; e < 4; ++e) l2[e] = c.lse2[wq * 128 + lane * 4 + e];
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.lse_taken);
       const int par = sc_items & 1;
       const int rows = it.nq * p.G;
-      const int w_lo = wq * 128, w_hi = min(rows, wq * 128 + 128);
-      if (w_lo < w_hi) {
-        const float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows;
-        const int nblk_item = min(p.nblk, (n * 128) / SB);
-        // selection tiles intersecting this warp's rows (row = query * G + head)
-        const int q_lo = w_lo / p.G, q_hi = (w_hi + p.G - 1) / p.G;
-        const int t_first = (it.qoff + q_lo) / p.T, t_last = (it.qoff + q_hi - 1) / p.T;
-        for (int b = 0; b < nblk_item; ++b) {
-          const float4 v4 = *reinterpret_cast<const float4*>(sp + size_t(b) * kMaxItemRows + r0);
-          const float vv[4] = {v4.x - l2[0], v4.y - l2[1], v4.z - l2[2], v4.w - l2[3]};
+      const float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows + wq * 128 + lane * 4;
+      const int nblk_item = min(p.nblk, (n * 128) / SB);
+      // selection tiles of the item's queries (row = query * G + head)
+      const int t_first = it.qoff / p.T, t_last = (it.qoff + it.nq - 1) / p.T;
+      // eight blocks per round, their loads in flight before any use
+      constexpr int kU = 8;
+      for (int b0 = 0; b0 < nblk_item; b0 += kU) {
+        float4 v4[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          v4[u] = *reinterpret_cast<const float4*>(sp + size_t(min(b0 + u, nblk_item - 1)) * kMaxItemRows);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int b = b0 + u;
+          if (b >= nblk_item) break;
+          const float vv[4] = {v4[u].x - l2[0], v4[u].y - l2[1], v4[u].z - l2[2], v4[u].w - l2[3]};
           for (int tt = t_first; tt <= t_last; ++tt) {
             // rows of tile tt inside the item: queries [tt*T - qoff, (tt+1)*T - qoff)
-            const int ra = max(w_lo, (tt * p.T - it.qoff) * p.G);
-            const int rb = min(w_hi, ((tt + 1) * p.T - it.qoff) * p.G);
+            const int ra = max(wq * 128, (tt * p.T - it.qoff) * p.G);
+            const int rb = min(min(rows, wq * 128 + 128), ((tt + 1) * p.T - it.qoff) * p.G);
+            if (ra >= rb) continue;  // the tile has no rows in this half
             const int tile_last = min(it.pos0 - it.qoff + (tt + 1) * p.T - 1, it.kv_len - 1);
             if (b * SB > tile_last) continue;  // not a candidate of this tile
             float v = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (r0 + e >= ra && r0 + e < rb) v = fmaxf(v, vv[e]);
+            for (int e = 0; e < 4; ++e) {
+              const int r = wq * 128 + lane * 4 + e;
+              if (r >= ra && r < rb) v = fmaxf(v, vv[e]);
+            }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
             if (lane == 0 && v > -INFINITY)
