@@ -85,8 +85,8 @@ struct Item {
 // Host-computed schedule, passed by value in the kernel parameters.
 // Items are enumerated sequence by sequence in `seq` order; the full layer
 // lists sequences longest first and each sequence's chunks last-to-first
-// (decreasing causal cost), so the round-robin over persistent CTAs starts
-// with the heaviest work.
+// (decreasing causal cost), so the persistent CTAs start with the heaviest
+// work (dealt in snake order, see snake_item).
 constexpr int kMaxSched = 256;
 struct Sched {
   int n_seq;
@@ -196,6 +196,15 @@ __device__ __forceinline__ Item get_item(const Params& p, const Sched& sc, int w
   it.tile0 = sc.tile_base[b] + qloc0 / p.T;
   it.qoff = qloc0 % p.T;
   return it;
+}
+
+// The k-th work item of this CTA. Items are listed heaviest first; dealing
+// them to the persistent CTAs in alternating direction each round (0..n-1,
+// then n-1..0) balances the per-CTA totals of a decreasing cost list far
+// better than plain round-robin (causal full layer at 32768 tokens: max/mean
+// 1.0005 instead of 1.035). Strictly increasing in k for every CTA.
+__device__ __forceinline__ int snake_item(int k) {
+  return k * int(gridDim.x) + ((k & 1) ? int(gridDim.x) - 1 - int(blockIdx.x) : int(blockIdx.x));
 }
 
 // Number of 128-key tiles an item iterates over, and the sparse-mode split.
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc, site, ctx) ? 1 : 0;
       return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
-    for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
+    for (int k = 0, wi = snake_item(0); wi < sc.n_items && ok; wi = snake_item(++k)) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
@@ -454,7 +463,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
         ++ctr;
         return s;
       };
-      for (int wi = blockIdx.x; wi < sc.n_items && ok; wi += gridDim.x) {
+      for (int k = 0, wi = snake_item(0); wi < sc.n_items && ok; wi = snake_item(++k)) {
         const Item it = get_item<MODE>(p, sc, wi);
         if (it.nq <= 0) continue;
         const KvPlan kp = kv_plan(p, it, MODE);
@@ -532,7 +541,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       ++wg_phase;
       return r;
     };
-    for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
+    for (int k = 0, wi = snake_item(0); wi < sc.n_items; wi = snake_item(++k)) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
@@ -896,7 +905,7 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
     const int wq = warp - 10;
     int sc_items = 0;
     if constexpr (MODE == kFull && SB > 0)
-    for (int wi = blockIdx.x; wi < sc.n_items; wi += gridDim.x) {
+    for (int k = 0, wi = snake_item(0); wi < sc.n_items; wi = snake_item(++k)) {
       const Item it = get_item<MODE>(p, sc, wi);
       if (it.nq <= 0) continue;
       const KvPlan kp = kv_plan(p, it, MODE);
