@@ -260,11 +260,46 @@ bool is_decode(const hs_varlen* vl, const hs_sel* sel) {
   return true;
 }
 
+// Resident CTAs of the full-layer decode pass 2 (the larger one) on this GPU.
+int full_decode_slots() {
+  static int slots = 0;
+  if (slots == 0) {
+    int per_sm = 0;
+    constexpr int bytes = dec::full_smem_bytes<true>();
+    if (set_smem(dec::full_decode_kernel<true>, bytes) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dec::full_decode_kernel<true>, dec::kThreads, bytes) ==
+            cudaSuccess &&
+        per_sm > 0)
+      slots = per_sm * num_sms();
+    else
+      slots = 2 * num_sms();
+  }
+  return slots;
+}
+
+// Key splits per (sequence, KV head): the grid (splits x sequences) should
+// fill whole waves of resident CTAs -- e.g. 10 splits x 64 sequences on 296
+// slots ran 3 waves for 2.16 waves of work. Take the fewest splits whose last
+// wave is at least 97 % full (else the best found), with at least one full
+// wave and one 64-key chunk per split.
 int full_decode_splits(const Shape& sh) {
   const int bg = sh.batch * sh.Hkv;
-  int n = (4 * num_sms() + bg - 1) / bg;
-  const int cap = std::max(1, (sh.max_kv + dec::kFullChunk - 1) / dec::kFullChunk);
-  return std::max(1, std::min(n, cap));
+  const int cap = std::max(1, std::min(256, (sh.max_kv + dec::kFullChunk - 1) / dec::kFullChunk));
+  const int slots = full_decode_slots();
+  int best = 1;
+  double best_eff = -1.0;
+  for (int ns = 1; ns <= cap; ++ns) {
+    const long long ctas = (long long)bg * ns;
+    if (ctas < slots && ns < cap) continue;
+    const long long waves = (ctas + slots - 1) / slots;
+    const double eff = double(ctas) / double(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = ns;
+    }
+    if (eff >= 0.97) break;
+  }
+  return best;
 }
 
 size_t full_decode_ws_bytes(const Shape& sh) {
