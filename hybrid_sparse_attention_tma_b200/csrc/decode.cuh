@@ -136,25 +136,6 @@ __device__ __forceinline__ void qk_bf16(const uint32_t (&qa)[8][4], const uint8_
 }
 
 // Same with FP8 keys: tile [NK][128 bytes], chunk c of 16 B at c ^ (r & 7).
-template <int NK>
-__device__ __forceinline__ void qk_fp8(const uint32_t (&qa)[8][4], const uint8_t* sk, float (&s)[NK / 8][4]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int nt = 0; nt < NK / 8; ++nt) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-    const int key = nt * 8 + (lane >> 2);
-    const uint8_t* row = sk + key * 128;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-      const int k0 = ks * 16 + 2 * (lane & 3);  // this thread's k pair, and k0 + 8
-      const int c0 = k0 >> 4, o0 = k0 & 15;
-      const uint16_t lo = *reinterpret_cast<const uint16_t*>(row + ((c0 ^ (key & 7)) << 4) + o0);
-      const uint16_t hi = *reinterpret_cast<const uint16_t*>(row + ((c0 ^ (key & 7)) << 4) + o0 + 8);
-      mma16816(s[nt], qa[ks], e4m3x2_to_bf16x2(lo), e4m3x2_to_bf16x2(hi));
-    }
-  }
-}
 
 // O[16 heads x 128] += P[16 x NK] . V[NK x 128], V bf16 swizzled.
 template <int NK>
@@ -174,31 +155,14 @@ __device__ __forceinline__ void pv_bf16(const uint32_t (&pa)[NK / 16][4], const 
   }
 }
 
-// FP8 V: B(k = key, n = d) pairs come from two rows; decode per element.
-template <int NK>
-__device__ __forceinline__ void pv_fp8(const uint32_t (&pa)[NK / 16][4], const uint8_t* sv, float (&o)[16][4]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int ks = 0; ks < NK / 16; ++ks) {
-    const int kr = ks * 16 + 2 * (lane & 3);  // keys kr, kr+1 (b0) and kr+8, kr+9 (b1)
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      const int dcol = nt * 8 + (lane >> 2);
-      const int c = dcol >> 4, off = dcol & 15;
-      auto at = [&](int key) -> uint8_t { return sv[key * 128 + ((c ^ (key & 7)) << 4) + off]; };
-      const uint16_t p0 = uint16_t(at(kr)) | (uint16_t(at(kr + 1)) << 8);
-      const uint16_t p1 = uint16_t(at(kr + 8)) | (uint16_t(at(kr + 9)) << 8);
-      mma16816(o[nt], pa[ks], e4m3x2_to_bf16x2(p0), e4m3x2_to_bf16x2(p1));
-    }
-  }
-}
-
 // ----------------------------------------------------------------------------
 // A6: sparse decode, one CTA per (sequence, KV head, 128-key chunk)
 // ----------------------------------------------------------------------------
+// Q | K, V tiles (bf16, swizzled; FP8 codes are gathered into their upper
+// halves and expanded in place) | scales, keys.
 template <bool FP8>
 constexpr int sparse_smem_bytes() {
-  return kHeads * 256 + 2 * kChunk * (FP8 ? 128 : 256) + 3 * kChunk * 4 + 1024;
+  return kHeads * 256 + 2 * kChunk * 256 + 3 * kChunk * 4 + 1024;
 }
 
 template <bool FP8>
@@ -207,9 +171,12 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sq = base;
-  uint8_t* sk = sq + kHeads * 256;
-  uint8_t* sv = sk + kChunk * kRowBytes;
-  float* sks = reinterpret_cast<float*>(sv + kChunk * kRowBytes);
+  uint8_t* sk = sq + kHeads * 256;   // bf16 tiles the MMAs read
+  uint8_t* sv = sk + kChunk * 256;
+  // gather target: the bf16 tiles, or (FP8) the upper half of each tile
+  uint8_t* gk = FP8 ? sk + kChunk * 128 : sk;
+  uint8_t* gv = FP8 ? sv + kChunk * 128 : sv;
+  float* sks = reinterpret_cast<float*>(sv + kChunk * 256);
   float* svs = sks + kChunk;
   int* skey = reinterpret_cast<int*>(svs + kChunk);
 
@@ -221,16 +188,23 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   const int pos = kv_len - 1;  // the new token is the sequence's last position
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
-  // visible set: selected tokens <= pos - w (a prefix of the ascending list), then the window
+  // visible set: selected tokens <= pos - w (a prefix of the ascending list),
+  // then the window; the prefix length is counted by all threads at once
   const int* idx = p.idx + size_t(bg) * p.topk;
   const int cnt = p.cnt ? __ldg(p.cnt + bg) : 0;
   const int lim = pos - p.w;
-  int lo = 0, hi = cnt;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(idx + mid) <= lim) lo = mid + 1; else hi = mid;
+  __shared__ int s_nsel[kThreads / 32];
+  {
+    int c = 0;
+    for (int i = threadIdx.x; i < cnt; i += kThreads) c += __ldg(idx + i) <= lim ? 1 : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+    if (lane == 0) s_nsel[warp] = c;
   }
-  const int n_sel = lo;
+  __syncthreads();
+  int n_sel = 0;
+#pragma unroll
+  for (int w = 0; w < kThreads / 32; ++w) n_sel += s_nsel[w];
   const int win_lo = max(0, pos - p.w + 1);
   const int total = n_sel + (pos - win_lo + 1) * (p.w > 0 ? 1 : 0);
   const int v0 = chunk * kChunk;
@@ -260,8 +234,8 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
     const uint8_t* ks = reinterpret_cast<const uint8_t*>(p.k) + row * kRowBytes + c * 16;
     const uint8_t* vs = reinterpret_cast<const uint8_t*>(p.v) + row * kRowBytes + c * 16;
     const uint32_t off = FP8 ? uint32_t(r * 128 + ((c ^ (r & 7)) << 4)) : swz(r, c);
-    cp_async16(smem_u32(sk) + off, ks, true);
-    cp_async16(smem_u32(sv) + off, vs, true);
+    cp_async16(smem_u32(gk) + off, ks, true);
+    cp_async16(smem_u32(gv) + off, vs, true);
   }
   if (FP8) {
     for (int i = threadIdx.x; i < kChunk; i += kThreads) {
@@ -274,12 +248,53 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   cp_async_commit();
   cp_async_wait<0>();
   __syncthreads();
+  if constexpr (FP8) {
+    // e4m3 -> bf16 is exact: expand both tiles in place into the swizzled
+    // bf16 layout, then the same ldmatrix / mma path as bf16 KV serves FP8.
+    // The codes of row r sit at byte 128 * (128 + r) of the tile; rows 0-63
+    // expand into bytes [0, 16 KB), below every code; rows 64-127 overwrite
+    // codes, so they are read into registers before anything is written.
+    constexpr int kItems = kChunk * 8;                    // (row, 16-code chunk) per tile
+    constexpr int kPer = kItems / kThreads;               // per thread and tile, per half
+    auto expand = [&](uint4 u, uint8_t* dst, int r, int c) {
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+      uint32_t b[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        b[2 * j] = e4m3x2_to_bf16x2(uint16_t(w4[j] & 0xFFFFu));
+        b[2 * j + 1] = e4m3x2_to_bf16x2(uint16_t(w4[j] >> 16));
+      }
+      *reinterpret_cast<uint4*>(dst + swz(r, 2 * c)) = make_uint4(b[0], b[1], b[2], b[3]);
+      *reinterpret_cast<uint4*>(dst + swz(r, 2 * c + 1)) = make_uint4(b[4], b[5], b[6], b[7]);
+    };
+    static_assert(kItems % (2 * kThreads) == 0, "even split of the expansion");
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint4 u[2][kPer / 2];
+#pragma unroll
+      for (int tv = 0; tv < 2; ++tv)
+#pragma unroll
+        for (int j = 0; j < kPer / 2; ++j) {
+          const int rc = half * (kItems / 2) + j * kThreads + threadIdx.x;
+          const int r = rc >> 3, c = rc & 7;
+          u[tv][j] = *reinterpret_cast<const uint4*>((tv ? gv : gk) + r * 128 + ((c ^ (r & 7)) << 4));
+        }
+      if (half == 1) __syncthreads();  // every code of rows 64-127 is in registers
+#pragma unroll
+      for (int tv = 0; tv < 2; ++tv)
+#pragma unroll
+        for (int j = 0; j < kPer / 2; ++j) {
+          const int rc = half * (kItems / 2) + j * kThreads + threadIdx.x;
+          expand(u[tv][j], tv ? sv : sk, rc >> 3, rc & 7);
+        }
+      __syncthreads();
+    }
+  }
 
   uint32_t qa[8][4];
   q_fragments(sq, qa);
   float s[kChunk / 8][4];
-  if constexpr (FP8) qk_fp8<kChunk>(qa, sk, s);
-  else qk_bf16<kChunk>(qa, sk, s);
+  qk_bf16<kChunk>(qa, sk, s);
 
   // softmax partial per head row (rows lane/4 and lane/4 + 8 of this warp)
   const float cs = p.scale_log2;
@@ -325,8 +340,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
-  if constexpr (FP8) pv_fp8<kChunk>(pa, sv, o);
-  else pv_bf16<kChunk>(pa, sv, o);
+  pv_bf16<kChunk>(pa, sv, o);
 
   // partials: unnormalised O and (m, l) per head
   float* po = p.part_o + (size_t(bg) * p.n_chunks + chunk) * kHeads * 128;
