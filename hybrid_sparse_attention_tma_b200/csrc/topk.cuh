@@ -9,10 +9,10 @@
 // Method: scores are >= 0, so their fp32 bit patterns order like the values.
 // A 4-pass MSB-first radix select (8 bits per pass, per-warp histograms in
 // shared memory) finds the k-th largest bit pattern tau and how many of the
-// k slots go to entries equal to tau. A final pass walks the row in index
-// order with a block-wide prefix scan and keeps every entry > tau plus the
-// first (k - #greater) entries == tau. Walking in index order both breaks
-// ties toward the lower index and emits the result already sorted.
+// k slots go to entries equal to tau. A final compaction over the row in
+// index order (each thread a contiguous segment, one block scan) keeps every
+// entry > tau plus the first (k - #greater) entries == tau. Index order both
+// breaks ties toward the lower index and emits the result already sorted.
 //
 // Two shapes of the same kernel: rows of up to kStageMax candidates are
 // staged once in shared memory by a 256-thread CTA (block-level selection,
@@ -157,20 +157,44 @@ __global__ void __launch_bounds__(THREADS)
   const int take_eq = krem;  // entries equal to tau to keep (lowest indices)
 
   // ---- ordered compaction ----
-  int out_base = 0, eq_base = 0;
-  for (int j0 = 0; j0 < n; j0 += THREADS) {
-    const int j = j0 + threadIdx.x;
-    const uint32_t key = j < n ? key_at(j) : 0u;
-    const int is_eq = (j < n && key == tau) ? 1 : 0;
-    int eq_total;
-    const int eq_rank = eq_base + block_excl_scan<THREADS>(is_eq, warp_sums, eq_total);
-    const int sel = (j < n) && (key > tau || (is_eq && eq_rank < take_eq));
-    int sel_total;
-    const int pos = out_base + block_excl_scan<THREADS>(sel, warp_sums, sel_total);
-    if (sel) out[pos] = j;
-    out_base += sel_total;
-    eq_base += eq_total;
+  // Thread t owns the contiguous segment [t*L, t*L + L) of the row: it counts
+  // its entries > tau and == tau, one pair of block scans gives every thread
+  // its output offset and the number of tau-entries before it, and a second
+  // walk writes the kept indices. Segments are in index order, so the output
+  // is ascending and ties go to the lowest indices.
+  const int L = (n + THREADS - 1) / THREADS;
+  const int j0 = min(n, threadIdx.x * L), j1 = min(n, j0 + L);
+  int gt = 0, eq = 0;
+  {
+    // counting may go in any order: start each lane at a different offset so
+    // staged (shared-memory) segments whose length is a multiple of 32 do not
+    // put a warp's accesses in one bank
+    const int len = j1 - j0;
+    int off = len > 0 ? lane % len : 0;
+    for (int c = 0; c < len; ++c) {
+      const uint32_t key = key_at(j0 + off);
+      gt += key > tau ? 1 : 0;
+      eq += key == tau ? 1 : 0;
+      off = off + 1 == len ? 0 : off + 1;
+    }
   }
+  int gt_total, eq_total;
+  const int gt_before = block_excl_scan<THREADS>(gt, warp_sums, gt_total);
+  const int eq_before = block_excl_scan<THREADS>(eq, warp_sums, eq_total);
+  int pos = gt_before + min(eq_before, take_eq);
+  int eq_seen = eq_before;
+  if (gt > 0 || (eq > 0 && eq_before < take_eq)) {
+    for (int j = j0; j < j1; ++j) {
+      const uint32_t key = key_at(j);
+      if (key > tau) {
+        out[pos++] = j;
+      } else if (key == tau) {
+        if (eq_seen < take_eq) out[pos++] = j;
+        ++eq_seen;
+      }
+    }
+  }
+  const int out_base = gt_total + min(eq_total, take_eq);
   for (int j = out_base + threadIdx.x; j < k; j += THREADS) out[j] = -1;
   if (threadIdx.x == 0) p.cnt[row] = out_base;
 }
