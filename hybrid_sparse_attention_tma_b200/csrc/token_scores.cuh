@@ -26,7 +26,9 @@ namespace tscore {
 
 constexpr int kThreads = 192;
 constexpr int kBlocks = 4;   // key blocks per item
-constexpr int kQStages = 3;
+constexpr int kQStagesMax = 3;
+template <int D>
+constexpr int q_stages() { return D == 128 ? 2 : 3; }  // 2 at d = 128 to fit the augmentation tiles
 constexpr int kSlabBytes = 128 * 128;
 
 struct Params {
@@ -38,18 +40,27 @@ struct Params {
   WaitCtl wc;
 };
 
+// The row's lse enters the MMA as one extra K step of 16 columns: K rows get
+// [1, 1, 0 ...], Q rows get [hi, lo, 0 ...] with hi + lo = -lse2 / c (bf16
+// pair, c = scale * log2 e > 0), so the accumulator holds s + (-lse2 / c) and
+// score = exp2(c * max) needs only a max per element from the reducers.
+// The augmentation tiles use the unswizzled K-major layout: 8-row x 16-byte
+// core matrices, the two K halves 128 bytes apart, 8-row groups 256 apart.
 template <int D>
 struct Layout {
   static constexpr int kTile = (D / 64) * kSlabBytes;  // 128 rows x D bf16
+  static constexpr int kQStages = q_stages<D>();
+  static constexpr int kAug = 128 * 16 * 2;            // 128 rows x 16 bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffQ = kBlocks * kTile;
-  static constexpr int kOffLse = kOffQ + kQStages * kTile;
-  static constexpr int kOffCtl = kOffLse + kQStages * 128 * 4;
+  static constexpr int kOffQa = kOffQ + kQStages * kTile;
+  static constexpr int kOffKa = kOffQa + kQStages * kAug;
+  static constexpr int kOffCtl = kOffKa + kAug;
 };
 
 struct Ctl {
   uint64_t k_full, k_empty;
-  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full[kBlocks], acc_free[kBlocks];
   uint64_t teardown;
   uint32_t tmem_base;
@@ -59,6 +70,21 @@ struct Ctl {
 template <int D>
 constexpr int smem_bytes() {
   return Layout<D>::kOffCtl + int(sizeof(Ctl)) + 1024;
+}
+static_assert(smem_bytes<128>() <= 232448 && smem_bytes<64>() <= 232448, "smem over 227 KB");
+
+// unswizzled K-major descriptor (layout type 0)
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= uint64_t((smem_addr >> 4) & 0x3FFF);
+  d |= uint64_t((lbo_bytes >> 4) & 0x3FFF) << 16;
+  d |= uint64_t((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= uint64_t(1) << 46;
+  return d;
+}
+// byte offset of 16-byte chunk `half` (K columns 8*half .. 8*half+7) of row r
+__device__ __forceinline__ uint32_t aug_off(int r, int half) {
+  return uint32_t((r >> 3) * 256 + half * 128 + (r & 7) * 16);
 }
 
 // item -> (tile, g, first key); items are enumerated tile by tile, KV head by
@@ -128,15 +154,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kOffCtl);
-  float* lse_s = reinterpret_cast<float*>(smem + L::kOffLse);
+  constexpr int kQStages = L::kQStages;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // constant K-side augmentation: every key row [1, 1, 0, ..., 0]
+  if (threadIdx.x < 128) {
+    *reinterpret_cast<uint4*>(smem + L::kOffKa + aug_off(threadIdx.x, 0)) = make_uint4(pack_bf16(1.f, 1.f), 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(smem + L::kOffKa + aug_off(threadIdx.x, 1)) = make_uint4(0u, 0u, 0u, 0u);
+  }
+  fence_proxy_async_smem();  // read by the tensor cores (async proxy)
 
   if (threadIdx.x == 0) {
     mbar_init(&c.k_full, 1);
     mbar_init(&c.k_empty, 1);
     for (int s = 0; s < kQStages; ++s) {
       mbar_init(&c.q_full[s], 1);
-      mbar_init(&c.q_empty[s], 1 + 4);  // MMA done with Q + each reducer warp done with lse
+      mbar_init(&c.q_empty[s], 1);  // MMA done with Q and its augmentation
     }
     for (int b = 0; b < kBlocks; ++b) {
       mbar_init(&c.acc_full[b], 1);
@@ -159,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 4) {
     // ===================== producer: K blocks, Q chunks + their lse =====================
     int qctr = 0, items = 0;
-    int last_q[kQStages] = {-1, -1, -1};
+    int last_q[kQStagesMax] = {-1, -1, -1};
     int k_loads = 0;
     bool ok = true;
     for (int wi = blockIdx.x; wi < p.n_items && ok; wi += gridDim.x) {
@@ -183,15 +215,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) okw = mbar_wait(&c.q_empty[s], ((qctr / kQStages) & 1) ^ 1, abort_flag, p.wc, 102, (wi << 12) | qc);
         okw = __shfl_sync(0xffffffffu, okw, 0);
         if (!okw) { ok = false; break; }
-        // lse of the chunk's 128 rows (row = query * G + head-in-group), log2 units
+        // augmentation of the chunk's 128 rows (row = query * G + head-in-group):
+        // [hi, lo] = -lse2 / c as a bf16 pair; rows past the tile get a huge
+        // negative hi so they never win a maximum
         const int qpc = 128 / p.G;
+        const float inv_c = 1.f / p.scale_log2;
         for (int rr = lane; rr < 128; rr += 32) {
           const int ql = qc * qpc + rr / p.G;
           const int h = it.g * p.G + rr % p.G;
-          float v = -INFINITY;
-          if (ql < it.ti.n) v = __ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) * 1.4426950408889634f;
-          lse_s[s * 128 + rr] = v;
+          uint32_t hl = pack_bf16(-3.0e38f, 0.f);
+          if (ql < it.ti.n) {
+            const float x = -(__ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) * 1.4426950408889634f) * inv_c;
+            const float hi = __bfloat162float(__float2bfloat16_rn(x));
+            hl = pack_bf16(hi, x - hi);
+          }
+          uint8_t* qa = smem + L::kOffQa + s * L::kAug;
+          *reinterpret_cast<uint4*>(qa + aug_off(rr, 0)) = make_uint4(hl, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(qa + aug_off(rr, 1)) = make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           mbar_expect_tx(&c.q_full[s], L::kTile);
@@ -218,6 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // descriptors built once; a K step adds its offset / 16 to the start field
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(smem + L::kOffK), 16, 1024);
       const uint64_t q_desc0 = sdesc_sw128(smem_u32(smem + L::kOffQ), 16, 1024);
+      const uint64_t ka_desc = sdesc_noswz(smem_u32(smem + L::kOffKa), 128, 256);
+      const uint64_t qa_desc0 = sdesc_noswz(smem_u32(smem + L::kOffQa), 128, 256);
       for (int wi = blockIdx.x; wi < p.n_items && ok; wi += gridDim.x) {
         const Item it = get_item(st, p, tile_items_prefix, wi);
         const int nb = (it.nkeys + 127) / 128;
@@ -239,6 +283,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
               umma_bf16(tmem + b * 128, ka + off, qb + off, kId, kk > 0 ? 1u : 0u);
             }
+            // + 1 * hi + 1 * lo = -lse2 / c per row
+            umma_bf16(tmem + b * 128, ka_desc, qa_desc0 + uint64_t((s * L::kAug) >> 4), kId, 1u);
             umma_commit(&c.acc_full[b]);
           }
           if (!ok) break;
@@ -266,12 +312,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int b = 0; b < kBlocks; ++b) best[b] = -INFINITY;
       for (int qc = 0; qc < it.nchunks && ok; ++qc) {
-        const int s = qctr % kQStages;
-        const float* ls = lse_s + s * 128;
-        // acquire the producer's lse writes directly (already complete once any
-        // accumulator of this chunk is ready; the stage cannot move on before
-        // this warp releases it)
-        if (!mbar_wait_warp(&c.q_full[s], (qctr / kQStages) & 1, abort_flag, p.wc, 121, (wi << 12) | qc)) { ok = false; break; }
         // valid columns of this chunk: rows of queries inside the tile
         const int c_max = min(128, (it.ti.n - qc * qpc) * p.G);
         const int pos_first = it.ti.pos0 + qc * qpc;  // position of the chunk's first query
@@ -286,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int c_min = max(0, (key - pos_first) * p.G);
           const bool full = (c_min == 0) && (c_max == 128);
           const uint32_t taddr = tmem + b * 128 + (uint32_t(warp * 32) << 16);
-          float m = best[b];
+          float m = best[b];  // max over rows of s - lse2 / c
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             uint32_t v[32];
@@ -294,19 +334,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             if (full) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                float a0, a1;
-                f2_split(f2_fma(f2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), f2(cs, cs),
-                                f2(-ls[ch * 32 + e], -ls[ch * 32 + e + 1])),
-                         a0, a1);
-                m = max3f(m, a0, a1);
-              }
+              for (int e = 0; e < 32; e += 2) m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
             } else {
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
                 const int col = ch * 32 + e;
-                const float a = fmaf(__uint_as_float(v[e]), cs, -ls[col]);
-                if (col >= c_min && col < c_max) m = fmaxf(m, a);
+                if (col >= c_min && col < c_max) m = fmaxf(m, __uint_as_float(v[e]));
               }
             }
           }
@@ -316,17 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) mbar_arrive(&c.acc_free[b]);
         }
         if (!ok) break;
-        // this warp is done with the chunk's lse
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.q_empty[s]);
-        ++qctr;
       }
       if (ok) {
         float* out = p.scores + (size_t(it.tile) * p.Hkv + it.g) * p.nblk;
 #pragma unroll
         for (int b = 0; b < kBlocks; ++b) {
           const int key = it.key0 + b * 128 + kl;
-          if (b < nb && key < it.key0 + it.nkeys) out[key] = best[b] > -INFINITY ? ex2(best[b]) : 0.f;
+          if (b < nb && key < it.key0 + it.nkeys) out[key] = best[b] > -1.0e30f ? ex2(best[b] * cs) : 0.f;
         }
       }
     }
