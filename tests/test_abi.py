@@ -84,5 +84,11 @@ def test_host_validation_errors(lib):
     assert _call_full(lib, _varlen([0, 600], [0, 512]), sel) == L.HS_ERR_INVALID_ARG
     assert lib.hs_swa_gated(ctypes.byref(vl), 0, 16, 16, 16, 16, 16, 16, 16, 1 << 20, None) == L.HS_ERR_INVALID_ARG
     assert lib.hs_topk_select(ctypes.byref(vl), ctypes.byref(sel), None, 16, 16, 16, 1 << 20, None) == L.HS_ERR_INVALID_ARG
+    # fused sparse layer: window, own cache and gate are required, pointers 16-byte aligned
+    fused = lambda win, ks, osp: lib.hs_sparse_swa_gated_prefill(
+        ctypes.byref(vl), ctypes.byref(sel), 16, 16, 16, 16, 16, win, ks, 16, 16, 16, osp, None, 16, 1 << 20, None)
+    assert fused(0, 16, None) == L.HS_ERR_INVALID_ARG
+    assert fused(128, None, None) == L.HS_ERR_INVALID_ARG
+    assert fused(128, 16, 24) == L.HS_ERR_INVALID_ARG
     assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG

@@ -136,6 +136,12 @@ VARIANTS = {
     # SWA + gate branch at small size
     "swa_gate": W.Workload("v7", ctx=(0, 100), new=(300, 200), n_q_heads=8, n_kv_heads=2, head_dim=128,
                            q_tile=64, block=64, topk=2, window=0, n_sparse=2, swa_window=128),
+    # a sequence with no new tokens inside the batch, fused layer with 16-token blocks
+    "empty_seq": W.Workload("v10", ctx=(0, 90, 40), new=(150, 0, 70), n_q_heads=4, n_kv_heads=1, head_dim=64,
+                            q_tile=16, block=16, topk=4, window=8, n_sparse=1, swa_window=32),
+    # token-level selection with the window branch and gate fused in (one launch per layer)
+    "swa_tok": W.Workload("v11", ctx=(0, 300), new=(260, 90), n_q_heads=16, n_kv_heads=1, head_dim=128,
+                          q_tile=16, block=1, topk=64, window=8, n_sparse=1, swa_window=32, needle_rate=0.02),
 }
 
 
