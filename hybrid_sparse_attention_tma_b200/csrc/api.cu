@@ -240,12 +240,17 @@ WaitCtl wait_ctl(void* ws) { return WaitCtl{reinterpret_cast<ErrWord*>(ws), g_ti
 size_t full_decode_ws_bytes(const Shape& sh);
 bool is_decode(const hs_varlen* vl, const hs_sel* sel);
 
+// Block-maximum spill of one CTA (double-buffered): per 128-key tile of the
+// longest sequence, 256 rows x (128 / B) blocks.
+size_t spill_floats_per_cta(int max_kv, int B) {
+  return 2 * size_t((max_kv + 127) / 128) * size_t(128 / B) * attn::kMaxItemRows;
+}
+
 size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
   if (is_decode(vl, sel) && sh.d == 128 && sh.G <= dec::kHeads) return full_decode_ws_bytes(sh);
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
-    const size_t nblk = (size_t(sh.max_kv) + sel->block - 1) / sel->block;
-    b += size_t(num_sms()) * 2 * nblk * attn::kMaxItemRows * sizeof(float);  // double-buffered spill
+    b += size_t(num_sms()) * spill_floats_per_cta(sh.max_kv, sel->block) * sizeof(float);
   } else {
     b += align_up(sizeof(int) * (size_t(n_tiles_of(vl, sel->q_tile)) + 1), 256);  // token-score item prefix
   }
@@ -541,6 +546,7 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   p.lse = lse;
   p.scores = scores;
   p.spill = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + kHeaderBytes);
+  p.spill_tiles = (sh.max_kv + 127) / 128;
   p.nblk = nblk;
   p.T = T;
   p.B = B;
@@ -846,9 +852,9 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   if (sel->block == 1) return HS_ERR_UNSUPPORTED;
   const int T = sel->q_tile, B = sel->block;
   const int nblk = (sh.max_kv + B - 1) / B;
-  // one CTA's spill is 2 x nblk x 256 floats (double-buffered); the fixed
-  // scratch bounds the grid
-  const size_t per_cta = 2 * size_t(nblk) * attn::kMaxItemRows * sizeof(float);
+  // one CTA's spill (double-buffered, whole 128-key tiles); the fixed scratch
+  // bounds the grid
+  const size_t per_cta = spill_floats_per_cta(sh.max_kv, B) * sizeof(float);
   const size_t cap = (kNoAllocScratchBytes - kHeaderBytes) / per_cta;
   if (cap < 1) return HS_ERR_WORKSPACE;  // sequence longer than the fixed scratch can serve
   cudaStream_t s = S(stream);
@@ -879,6 +885,7 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   p.lse = lse;
   p.scores = scores;
   p.spill = reinterpret_cast<float*>(reinterpret_cast<char*>(scratch) + kHeaderBytes);
+  p.spill_tiles = (sh.max_kv + 127) / 128;
   p.nblk = nblk;
   p.T = T;
   p.B = B;

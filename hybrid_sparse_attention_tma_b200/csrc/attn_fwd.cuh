@@ -105,7 +105,8 @@ struct Params {
   float* lse;  // [Hq, Tq] natural log, may be null
   // block-score by-product (full mode with SB = B > 1)
   float* scores;  // [n_tiles, Hkv, nblk]
-  float* spill;   // [gridDim.x][2][nblk][256] (double-buffered per CTA)
+  float* spill;   // [gridDim.x][2][spill_tiles][256 rows][128 / B] (double-buffered per CTA)
+  int spill_tiles;  // 128-key tiles of the longest sequence
   int nblk;
   int T, B;
   int chunks_per_tile;  // sparse mode: ceil(T*G / 256)
@@ -693,14 +694,23 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
           // ---- row max; block maxima for the scores ----
           float mt = -INFINITY;
           if constexpr (MODE == kFull && SB > 0) {
+            // this row's maxima of the tile's nb blocks, one vector store
+            // ([tile][row][block] layout; blocks past the sequence are never read)
             constexpr int nb = 128 / SB;
-            float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows + vr;
+            float* sp = p.spill + ((size_t(blockIdx.x) * 2 + par) * p.spill_tiles + i) * kMaxItemRows * nb +
+                        size_t(vr) * nb;
             float mb[nb];
 #pragma unroll
-            for (int b = 0; b < nb; ++b) {
-              mb[b] = max_n<SB>(x + b * SB);
-              const int gb = i * nb + b;
-              if (gb < p.nblk) sp[size_t(gb) * kMaxItemRows] = mb[b] * cs;  // log2 units
+            for (int b = 0; b < nb; ++b) mb[b] = max_n<SB>(x + b * SB);
+            if constexpr (nb == 1) {
+              sp[0] = mb[0] * cs;  // log2 units
+            } else if constexpr (nb == 2) {
+              *reinterpret_cast<float2*>(sp) = make_float2(mb[0] * cs, mb[1] * cs);
+            } else {
+#pragma unroll
+              for (int q4 = 0; q4 < nb / 4; ++q4)
+                reinterpret_cast<float4*>(sp)[q4] =
+                    make_float4(mb[4 * q4] * cs, mb[4 * q4 + 1] * cs, mb[4 * q4 + 2] * cs, mb[4 * q4 + 3] * cs);
             }
             mt = max_n<nb>(mb);
           } else {
@@ -918,40 +928,52 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
       if (lane == 0) mbar_arrive(&c.lse_taken);
       const int par = sc_items & 1;
       const int rows = it.nq * p.G;
-      const float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.nblk * kMaxItemRows + wq * 128 + lane * 4;
+      constexpr int nb = SB > 0 ? 128 / SB : 1;
+      // this lane's 4 rows of a tile: 4 * nb consecutive floats ([tile][row][block])
+      const float* sp = p.spill + (size_t(blockIdx.x) * 2 + par) * p.spill_tiles * kMaxItemRows * nb +
+                        size_t(wq * 128 + lane * 4) * nb;
       const int nblk_item = min(p.nblk, (n * 128) / SB);
+      const int ntile_item = (nblk_item + nb - 1) / nb;
       // selection tiles of the item's queries (row = query * G + head)
       const int t_first = it.qoff / p.T, t_last = (it.qoff + it.nq - 1) / p.T;
-      // eight blocks per round, their loads in flight before any use
-      constexpr int kU = 8;
-      for (int b0 = 0; b0 < nblk_item; b0 += kU) {
-        float4 v4[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-          v4[u] = *reinterpret_cast<const float4*>(sp + size_t(min(b0 + u, nblk_item - 1)) * kMaxItemRows);
+      // several tiles per round, their loads in flight before any use
+      constexpr int kU = nb >= 8 ? 1 : 8 / nb;
+      for (int i0 = 0; i0 < ntile_item; i0 += kU) {
+        float4 v4[kU][nb];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-          const int b = b0 + u;
-          if (b >= nblk_item) break;
-          const float vv[4] = {v4[u].x - l2[0], v4[u].y - l2[1], v4[u].z - l2[2], v4[u].w - l2[3]};
-          for (int tt = t_first; tt <= t_last; ++tt) {
-            // rows of tile tt inside the item: queries [tt*T - qoff, (tt+1)*T - qoff)
-            const int ra = max(wq * 128, (tt * p.T - it.qoff) * p.G);
-            const int rb = min(min(rows, wq * 128 + 128), ((tt + 1) * p.T - it.qoff) * p.G);
-            if (ra >= rb) continue;  // the tile has no rows in this half
-            const int tile_last = min(it.pos0 - it.qoff + (tt + 1) * p.T - 1, it.kv_len - 1);
-            if (b * SB > tile_last) continue;  // not a candidate of this tile
-            float v = -INFINITY;
+          const float4* src = reinterpret_cast<const float4*>(sp + size_t(min(i0 + u, ntile_item - 1)) * kMaxItemRows * nb);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int r = wq * 128 + lane * 4 + e;
-              if (r >= ra && r < rb) v = fmaxf(v, vv[e]);
+          for (int q = 0; q < nb; ++q) v4[u][q] = src[q];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          if (i0 + u >= ntile_item) break;
+          const float* f = reinterpret_cast<const float*>(&v4[u][0]);  // row e, block j at f[e * nb + j]
+#pragma unroll
+          for (int j = 0; j < nb; ++j) {
+            const int b = (i0 + u) * nb + j;
+            if (b >= nblk_item) break;
+            const float vv[4] = {f[j] - l2[0], f[nb + j] - l2[1], f[2 * nb + j] - l2[2], f[3 * nb + j] - l2[3]};
+            for (int tt = t_first; tt <= t_last; ++tt) {
+              // rows of tile tt inside the item: queries [tt*T - qoff, (tt+1)*T - qoff)
+              const int ra = max(wq * 128, (tt * p.T - it.qoff) * p.G);
+              const int rb = min(min(rows, wq * 128 + 128), ((tt + 1) * p.T - it.qoff) * p.G);
+              if (ra >= rb) continue;  // the tile has no rows in this half
+              const int tile_last = min(it.pos0 - it.qoff + (tt + 1) * p.T - 1, it.kv_len - 1);
+              if (b * SB > tile_last) continue;  // not a candidate of this tile
+              float v = -INFINITY;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int r = wq * 128 + lane * 4 + e;
+                if (r >= ra && r < rb) v = fmaxf(v, vv[e]);
+              }
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+              if (lane == 0 && v > -INFINITY)
+                atomicMax(reinterpret_cast<unsigned int*>(p.scores + (size_t(it.tile0 + tt) * p.Hkv + it.g) * p.nblk + b),
+                          __float_as_uint(ex2(v)));
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-            if (lane == 0 && v > -INFINITY)
-              atomicMax(reinterpret_cast<unsigned int*>(p.scores + (size_t(it.tile0 + tt) * p.Hkv + it.g) * p.nblk + b),
-                        __float_as_uint(ex2(v)));
           }
         }
       }

@@ -255,10 +255,10 @@ HS_API hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* 
  * Sharing: every call on a device uses the same array and leaves its contents
  * behind. Calls whose kernels overlap on the GPU (e.g. on two streams without
  * ordering) race on it and give wrong results; order them.
- * Limits: block-level selection only (B >= 8). The grid is capped so that
- * grid * 2 * ceil(max_kv / B) KB fits in the array; if a single CTA's share
- * (2 * ceil(max_kv / B) KB) does not fit -- more than 32767 blocks, i.e.
- * max_kv above ~2.1M tokens at B = 64 --
+ * Limits: block-level selection only (B >= 8). A CTA's share is
+ * 2 * ceil(max_kv / 128) * (128 / B) KB (whole 128-key tiles); the grid is
+ * capped so that grid shares fit in the array; if a single share does not
+ * fit -- more than ~32767 blocks, i.e. max_kv above ~2.1M tokens at B = 64 --
  * the call returns HS_ERR_WORKSPACE before launching. Smaller caps only mean
  * fewer CTAs, not different results.
  * check != 0: synchronise `stream` after the launch and return HS_ERR_TIMEOUT
