@@ -300,7 +300,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ===================== reducers: thread = key lane =====================
     const int kl = warp * 32 + lane;  // key within each 128-key block
-    int qctr = 0;
     int acc_cnt[kBlocks] = {0, 0, 0, 0};
     bool ok = true;
     const float cs = p.scale_log2;
