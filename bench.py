@@ -464,23 +464,36 @@ def oracle_threads():
         return os.cpu_count() or 1
 
 
-def time_oracle(w, n_tiles_sample=1, repeats=1):
-    """Time the oracle's block on `n_tiles_sample` middle tiles; tokens/s."""
+def time_oracle(w, n_tiles_sample=1, repeats=1, min_seconds=0.0, max_tiles=8):
+    """Time the oracle's whole block on middle selection tiles, one tile per
+    run: `repeats` runs of the first `n_tiles_sample` tiles, or (min_seconds >
+    0) successive tiles until that much oracle time or `max_tiles` tiles.
+    Returns (tokens per run, run times)."""
     import oracle as O
     from oracle.block import run_block
     inp = W.make_block_inputs(w, device="cpu")
     q, k, v, layers = oracle_sample(w, 0, inp)
     n_t = w.n_tiles()
-    mids = [n_t // 2 + i for i in range(n_tiles_sample)]
     tiles = O.make_tiles(w.cu_q(), w.cu_kv(), w.q_tile)
-    toks = sum(tiles[i].n for i in mids)
-    times = []
-    for _ in range(repeats):
+
+    def run(ids):
         t = time.perf_counter()
         run_block(q, k, v, layers, w.cu_q(), w.cu_kv(), w.n_kv_heads, w.q_tile, w.block, w.topk, w.window,
-                  w.swa_window, tile_ids=mids)
-        times.append(time.perf_counter() - t)
-    return toks, times
+                  w.swa_window, tile_ids=ids)
+        return time.perf_counter() - t
+
+    if min_seconds > 0:
+        toks, times = [], []
+        i = 0
+        while (sum(times) < min_seconds and i < max_tiles) or not times:
+            tid = min(n_t - 1, n_t // 2 + i)
+            times.append(run([tid]))
+            toks.append(tiles[tid].n)
+            i += 1
+        return toks, times
+    mids = [min(n_t - 1, n_t // 2 + i) for i in range(n_tiles_sample)]
+    toks = sum(tiles[i].n for i in mids)
+    return toks, [run(mids) for _ in range(repeats)]
 
 
 def bench_reference(args, world, rank):
@@ -521,10 +534,11 @@ def main():
     out = bench_ours(args, world, rank, local)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w = workload(args)
-        toks, times = time_oracle(w, 1, repeats=1)
-        out["cpu_baseline"] = {"value": round(toks / sum(times), 3), "unit": "tokens/s", "cores": oracle_threads(),
-                               "kind": "oracle",
-                               "sample": f"1 middle selection tile ({toks} queries), whole block, {sum(times):.1f} s"}
+        toks, times = time_oracle(w, min_seconds=10.0)
+        out["cpu_baseline"] = {"value": round(sum(toks) / sum(times), 3), "unit": "tokens/s",
+                               "cores": oracle_threads(), "kind": "oracle",
+                               "sample": f"{len(toks)} middle selection tiles ({sum(toks)} queries), whole block, "
+                                         f"{sum(times):.1f} s"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
