@@ -251,43 +251,65 @@ def bench_ours(args, world, rank, local):
     torch.cuda.synchronize()
     hs.check_error(blk.ws)
 
-    kinds = ["full", "topk", "sparse", "swa"]
-    ev = {kd: [] for kd in kinds}
+    kinds = ["full", "topk", "sparse"]
+    L0 = layers[0]
 
-    def rec(kind, fn):
+    def call(kind, st):
+        """One library call of `kind` on stream `st` (the first sparse layer's inputs)."""
+        sel, bufs = blk.sel, blk._bufs
+        if kind == "full":
+            full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"], bufs["scores"],
+                             ws=blk.ws, stream=st)
+        elif kind == "topk":
+            topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws, stream=st)
+        elif blk.decode:
+            if fp8_kv is not None:
+                sparse_attn_decode(vl, sel, L0.q, inp.k_fp8, inp.v_fp8, bufs["idx"], bufs["cnt"], inp.k_scale,
+                                   inp.v_scale, HS_KV_FP8_E4M3, o=bufs["o_sp0"], lse=bufs["lse_sp0"], ws=blk.ws,
+                                   stream=st)
+            else:
+                sparse_attn_decode(vl, sel, L0.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], kv_dtype=HS_KV_BF16,
+                                   o=bufs["o_sp0"], lse=bufs["lse_sp0"], ws=blk.ws, stream=st)
+        elif blk.swa_window > 0:
+            # the whole sparse layer: sparse branch, own-cache window, gate
+            sparse_swa_gated_prefill(vl, sel, L0.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], blk.swa_window, L0.k_swa,
+                                     L0.v_swa, L0.gamma, o=bufs["o_l0"], ws=blk.ws, stream=st)
+        else:
+            sparse_attn_prefill(vl, sel, L0.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["o_sp0"],
+                                bufs["lse_sp0"], ws=blk.ws, stream=st)
+
+    # Launch-bound steps (decode: dozens of microsecond kernels) would time the
+    # host's enqueue rate rather than the GPU, so the step and every kernel
+    # kind are captured once in CUDA graphs and replayed; the library enqueues
+    # only launches and memsets inside a call (its one-time set-up ran during
+    # warm-up), so capture is safe.
+    step_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(step_graph):
+        blk.forward(inp.q, inp.k, inp.v, layers, stream=torch.cuda.current_stream(), fp8_kv=fp8_kv,
+                    intermediates=False)
+    reps = 5
+    kind_graphs = {}
+    for kd in kinds:
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gk):
+            for _ in range(reps):
+                call(kd, torch.cuda.current_stream())
+        kind_graphs[kd] = gk
+    for _ in range(2):
+        step_graph.replay()
+        for gk in kind_graphs.values():
+            gk.replay()
+    torch.cuda.synchronize()
+    hs.check_error(blk.ws)
+
+    def timed(fn, n):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        fn()
+        for _ in range(n):
+            fn()
         b.record(stream)
-        ev[kind].append((a, b))
-
-    def step_instrumented():
-        sel, bufs = blk.sel, blk._bufs
-        rec("full", lambda: full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"],
-                                             bufs["scores"], ws=blk.ws, stream=stream))
-        rec("topk", lambda: topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws,
-                                        stream=stream))
-        for j, L in enumerate(layers):
-            tag = str(j % 2)
-            if blk.decode:
-                if fp8_kv is not None:
-                    rec("sparse", lambda: sparse_attn_decode(vl, sel, L.q, inp.k_fp8, inp.v_fp8, bufs["idx"],
-                                                             bufs["cnt"], inp.k_scale, inp.v_scale, HS_KV_FP8_E4M3,
-                                                             o=bufs["o_sp" + tag], lse=bufs["lse_sp" + tag],
-                                                             ws=blk.ws, stream=stream))
-                else:
-                    rec("sparse", lambda: sparse_attn_decode(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
-                                                             kv_dtype=HS_KV_BF16, o=bufs["o_sp" + tag],
-                                                             lse=bufs["lse_sp" + tag], ws=blk.ws, stream=stream))
-            elif blk.swa_window > 0:
-                # the whole sparse layer: sparse branch, own-cache window, gate
-                rec("sparse", lambda: sparse_swa_gated_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
-                                                               blk.swa_window, L.k_swa, L.v_swa, L.gamma,
-                                                               o=bufs["o_l" + tag], ws=blk.ws, stream=stream))
-            else:
-                rec("sparse", lambda: sparse_attn_prefill(vl, sel, L.q, inp.k, inp.v, bufs["idx"], bufs["cnt"],
-                                                          bufs["o_sp" + tag], bufs["lse_sp" + tag], ws=blk.ws,
-                                                          stream=stream))
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
 
     if world > 1:
         dist.barrier()
@@ -296,19 +318,13 @@ def bench_ours(args, world, rank, local):
                           if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
     clocks.start()
     time.sleep(0.3)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step_instrumented()
-    t1.record(stream)
-    torch.cuda.synchronize()
+    ms_total = timed(step_graph.replay, args.steps)
+    n_kind = max(2, args.steps // 4)
+    kms = {kd: timed(kind_graphs[kd].replay, n_kind) / (n_kind * reps) for kd in kinds}
     clk = clocks.stop()
     if world > 1:
         dist.barrier()
     hs.check_error(blk.ws)
-    ms_total = t0.elapsed_time(t1)
-    kms = {kd: (sum(a.elapsed_time(b) for a, b in ev[kd]) / len(ev[kd]) if ev[kd] else 0.0) for kd in kinds}
     vals = max_over_ranks([ms_total] + [kms[kd] for kd in kinds], device)
     ms_total = vals[0]
     kms = {kd: vals[i + 1] for i, kd in enumerate(kinds)}
@@ -352,7 +368,7 @@ def bench_ours(args, world, rank, local):
         swa_flop = 4.0 * d * hq * swa_pairs(w) if w.swa_window > 0 else 0.0
         entry("sparse", kms["sparse"], 4.0 * d * G * vis + swa_flop, "tensor")
     entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
-    per_step = {"full": 1, "topk": 1, "sparse": len(layers), "swa": len(layers) if w.swa_window else 0}
+    per_step = {"full": 1, "topk": 1, "sparse": len(layers)}
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])
