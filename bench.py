@@ -26,6 +26,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -109,7 +110,7 @@ def traffic_for(kernel: str, workload: str):
 class ClockSampler:
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"hs_clocks_bench_{os.getpid()}.csv")
         self.gpu = gpu_index
 
     def start(self):

@@ -261,8 +261,8 @@ def topk_select(scores, cu_q, cu_kv, T: int, B: int, k: int,
                 tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
     """Keep the k highest-scoring candidate blocks of each (tile, KV head).
 
-    Order: score descending, ties to the lower block index (north-star rule;
-    the pages only say "TopK"). The kept set is emitted in ascending index
+    Order: score descending, ties to the lower block index (the reading used
+    throughout; the pages only say "TopK"). The kept set is emitted in ascending index
     order and padded with -1; cnt = min(k, #candidates).
     Returns (idx int32 [n_tiles, H_kv, k], cnt int32 [n_tiles, H_kv]).
     """
