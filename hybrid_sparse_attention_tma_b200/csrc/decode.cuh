@@ -135,8 +135,6 @@ __device__ __forceinline__ void qk_bf16(const uint32_t (&qa)[8][4], const uint8_
   }
 }
 
-// Same with FP8 keys: tile [NK][128 bytes], chunk c of 16 B at c ^ (r & 7).
-
 // O[16 heads x 128] += P[16 x NK] . V[NK x 128], V bf16 swizzled.
 template <int NK>
 __device__ __forceinline__ void pv_bf16(const uint32_t (&pa)[NK / 16][4], const uint8_t* sv, float (&o)[16][4]) {
