@@ -38,17 +38,17 @@ namespace hs {
 namespace attn {
 
 // Warps 0-7 softmax, 8 TMA producer, 9 UMMA issuer. The window-only gated
-// call and the fused sparse layer (short items, an epilogue each) give each
-// Q-tile its own issuer (warps 9, 10) so that one tile's wait never delays
-// the other's MMAs at item boundaries; with long items one issuer in the
-// order PV_0 QK_0 PV_1 QK_1 keeps the two softmax warpgroups out of phase,
-// which overlaps one's softmax with the other's MMAs (measured: the full and
-// plain sparse layers are faster with one issuer, these two with two). The
-// full layer with block scores adds warps 10-11, which reduce each work
-// item's spilled block maxima while the softmax warps move on.
+// call (two tiles and an epilogue per item) gives each Q-tile its own issuer
+// (warps 9, 10) so that one tile's wait never delays the other's MMAs at item
+// boundaries; with longer items one issuer in the order PV_0 QK_0 PV_1 QK_1
+// keeps the two softmax warpgroups out of phase, which overlaps one's softmax
+// with the other's MMAs (measured: the full, plain sparse and fused sparse
+// layers are faster with one issuer, the window call with two). The full
+// layer with block scores adds warps 10-11, which reduce each work item's
+// spilled block maxima while the softmax warps move on.
 template <int MODE, int SB>
 constexpr bool two_issuers() {
-  return (MODE == 1 && SB == 0) || MODE == 2;
+  return MODE == 1 && SB == 0;
 }
 template <int MODE, int SB>
 constexpr int threads_for() {
