@@ -464,12 +464,12 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!q || !k || !v || !o || !scores) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
   if (!ws || ws_bytes < full_ws_bytes(vl, sh, sel)) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
-  if (sh.Tq == 0) return HS_OK;
   const int T = sel->q_tile, B = sel->block;
   const int n_tiles = n_tiles_of(vl, T);
   const int nblk = (sh.max_kv + B - 1) / B;
@@ -586,10 +586,10 @@ hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* sc
   hs_status st = check_varlen(vl, &sh, false);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!scores || !idx || !cnt) return HS_ERR_INVALID_ARG;
   if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
   if (vl->batch > kMaxSeq) return HS_ERR_UNSUPPORTED;
-  if (sh.Tq == 0) return HS_OK;
   SeqTable table;
   fill_seqtable(vl, sel->q_tile, &table);
   topk::Params p{};
@@ -626,6 +626,7 @@ static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!q || !k || !v || !o || (sel->topk > 0 && (!idx || !cnt))) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
   if (swa) {
@@ -636,7 +637,6 @@ static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void
   if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
-  if (sh.Tq == 0) return HS_OK;
   const int T = sel->q_tile, B = sel->block;
   Maps m;
   if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
@@ -792,6 +792,7 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
   Shape sh;
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (window < 1) return HS_ERR_INVALID_ARG;
   if (!q || !k_swa || !v_swa || !gamma || !o_sparse || !o) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_swa) || !aligned16(v_swa) || !aligned16(o) || !aligned16(o_sparse))
@@ -799,7 +800,6 @@ hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const
   if (!ws || ws_bytes < kHeaderBytes) return HS_ERR_WORKSPACE;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
-  if (sh.Tq == 0) return HS_OK;
   Maps m;
   if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
       !make_map_3d(&m.k, k_swa, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
@@ -845,6 +845,7 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!q || !k || !v || !o || !scores) return HS_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return HS_ERR_INVALID_ARG;
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
@@ -860,7 +861,6 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   cudaStream_t s = S(stream);
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch, s)) != HS_OK) return st;
-  if (sh.Tq == 0) return HS_OK;
   const int n_tiles = n_tiles_of(vl, T);
   if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
     return HS_ERR_CUDA;

@@ -221,6 +221,9 @@ DECODE = {
     # GQA group 8 (only 8 of the 64 MMA rows valid), several KV heads
     "dec_gqa8": W.Workload("d2", ctx=(700, 90), new=(1, 1), n_q_heads=32, n_kv_heads=4, head_dim=128,
                            q_tile=1, block=1, topk=40, window=16, n_sparse=1),
+    # k = 0: the sparse layer sees only the forced window (one context shorter than the window)
+    "dec_window_only": W.Workload("d3", ctx=(200, 45), new=(1, 1), n_q_heads=64, n_kv_heads=1, head_dim=128,
+                                  q_tile=1, block=1, topk=0, window=48, n_sparse=1),
 }
 
 
@@ -253,3 +256,17 @@ def test_bounded_wait_timeout_reports_and_context_survives():
     assert e.value.status == L.HS_ERR_TIMEOUT
     hs.check_error(ws)  # cleared
     run_and_check(VARIANTS["k0_window"], seed=1)
+
+
+def test_empty_batch_is_a_no_op():
+    """Every call accepts a batch without new tokens (empty tensors, null data
+    pointers) and returns without launching; the block runner passes through."""
+    w = W.Workload("e0", ctx=(64, 100), new=(0, 0), n_q_heads=8, n_kv_heads=2, head_dim=128, q_tile=64, block=64,
+                   topk=2, window=0, n_sparse=2, swa_window=128)
+    inp = W.make_block_inputs(w, device="cuda", seed=1)
+    assert inp.q.shape[0] == 0
+    res = GpuBlock(w, inp).run()
+    torch.cuda.synchronize()
+    assert res["o_full"].shape[0] == 0 and res["scores"].shape[0] == 0
+    for L in res["layers"]:
+        assert L["o"].shape[0] == 0
