@@ -92,3 +92,59 @@ def test_host_validation_errors(lib):
     assert fused(128, 16, 24) == L.HS_ERR_INVALID_ARG
     assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG
+
+
+def test_workspace_size_every_op_at_workload_shapes(lib):
+    """Every op sizes a workspace (header + scratch) for the benchmarked shapes."""
+    import workloads as W
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    ops = [L.HS_OP_FULL_ATTN_SELECT, L.HS_OP_TOPK_SELECT, L.HS_OP_SPARSE_ATTN_PREFILL, L.HS_OP_SPARSE_ATTN_DECODE,
+           L.HS_OP_SWA_GATED, L.HS_OP_SPARSE_SWA_GATED_PREFILL]
+    for name in ["tiny", "hys_block", "hys2_prefill", "decode", "agentic"]:
+        w = W.WORKLOADS[name]
+        vl = _varlen(w.cu_q(), w.cu_kv(), hq=w.n_q_heads, hkv=w.n_kv_heads, d=w.head_dim)
+        sel = L.HsSel(w.q_tile, w.block, w.topk, w.window)
+        for op in ops:
+            if op == L.HS_OP_SPARSE_ATTN_DECODE and name != "decode":
+                continue
+            n = lib.hs_workspace_size(op, ctypes.byref(vl), ctypes.byref(sel))
+            assert n >= 256 and n % 256 == 0, (name, op, n)
+        if name == "hys_block":  # the block-max spill: one double-buffered share per SM, whole 128-key tiles
+            n = lib.hs_workspace_size(L.HS_OP_FULL_ATTN_SELECT, ctypes.byref(vl), ctypes.byref(sel))
+            assert n >= 2 * (w.max_kv // 128) * (128 // w.block) * 256 * 4
+
+
+def test_bench_traffic_needs_matching_source_hash(tmp_path, monkeypatch):
+    import json
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    for f in bench.KERNEL_SOURCES:  # the hash is taken over the kernel sources under ROOT
+        dst = tmp_path / f
+        dst.parent.mkdir(parents=True, exist_ok=True)
+        dst.write_bytes(open(os.path.join(ROOT, f), "rb").read())
+    h = bench.src_hash()
+    (prof / "traffic.json").write_text(json.dumps({"attn_fwd_full:hys_block": {"src_hash": h,
+                                                                                "dram_bytes_per_launch": 123}}))
+    assert bench.traffic_for("attn_fwd_full", "hys_block") == 123
+    assert bench.traffic_for("attn_fwd_full", "decode") is None
+    (prof / "traffic.json").write_text(json.dumps({"attn_fwd_full:hys_block": {"src_hash": "stale",
+                                                                                "dram_bytes_per_launch": 123}}))
+    assert bench.traffic_for("attn_fwd_full", "hys_block") is None
+
+
+def test_cpu_baseline_samples_until_the_time_budget():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    w = W.WORKLOADS["tiny"]
+    toks, times = bench.time_oracle(w, min_seconds=1e-6, max_tiles=3)
+    assert len(toks) == 1 and toks[0] == w.q_tile  # one middle tile already exceeds a tiny budget
+    toks, times = bench.time_oracle(w, min_seconds=1e9, max_tiles=3)
+    assert len(toks) == 3 and all(t > 0 for t in times)  # capped by max_tiles
+    toks, times = bench.time_oracle(w, 2, repeats=2)
+    assert toks == 2 * w.q_tile and len(times) == 2
