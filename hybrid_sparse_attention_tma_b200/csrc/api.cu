@@ -507,7 +507,8 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
     }
     const dim3 grid(ns, bg);
     dec::full_decode_kernel<false><<<grid, dec::kThreads, dec::full_smem_bytes<false>(), s>>>(fp);
-    dec::lse_combine_kernel<<<bg, dec::kHeads, 0, s>>>(fp.part_ml, ns, fp.lse2);
+    dec::lse_combine_kernel<<<dim3(bg, dec::kHeads / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(
+        fp.part_ml, ns, fp.lse2);
     dec::full_decode_kernel<true><<<grid, dec::kThreads, dec::full_smem_bytes<true>(), s>>>(fp);
     dec::CombineParams cp{};
     cp.part_o = fp.part_o;
@@ -521,7 +522,7 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
     cp.lse2_in = fp.lse2;
     cp.o = reinterpret_cast<__nv_bfloat16*>(o);
     cp.lse = lse;
-    dec::combine_kernel<<<bg, 512, 0, s>>>(cp);
+    dec::combine_kernel<<<dim3(bg, (sh.G + dec::kCombineHeads - 1) / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(cp);
     return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
   }
 
@@ -726,6 +727,7 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!is_decode(vl, sel)) return HS_ERR_INVALID_ARG;  // one query per sequence, q_tile = block = 1
   if (sh.d != 128 || sh.G > dec::kHeads) return HS_ERR_UNSUPPORTED;
   if (kv_dtype != HS_KV_BF16 && kv_dtype != HS_KV_FP8_E4M3) return HS_ERR_INVALID_ARG;
@@ -782,7 +784,7 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   cp.normalised = false;
   cp.o = reinterpret_cast<__nv_bfloat16*>(o);
   cp.lse = lse;
-  dec::combine_kernel<<<bg, 512, 0, s>>>(cp);
+  dec::combine_kernel<<<dim3(bg, (sh.G + dec::kCombineHeads - 1) / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(cp);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 

@@ -181,70 +181,66 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   const int chunk = blockIdx.x;
   const int bg = blockIdx.y;  // sequence * Hkv + g
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int kv0 = __ldg(p.cu_kv + b);
-  const int kv_len = __ldg(p.cu_kv + b + 1) - kv0;
-  const int pos = kv_len - 1;  // the new token is the sequence's last position
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  static_assert(kChunk == kThreads, "one slot of the chunk per thread");
+  __shared__ uint32_t s_valid[kChunk / 32];
 
-  // visible set: selected tokens <= pos - w (a prefix of the ascending list),
-  // then the window; the prefix length is counted by all threads at once
-  const int* idx = p.idx + size_t(bg) * p.topk;
+  // Slot order of V_q: the window [pos-w+1, pos] first, then the selected
+  // tokens <= pos - w. The index list is ascending, so its visible part is a
+  // prefix and slot w + j holds idx[j] exactly when idx[j] <= pos - w: every
+  // slot decides its own membership from one index, loaded together with the
+  // sequence bounds, and no pass over the whole list precedes the gather.
+  const int slot = chunk * kChunk + threadIdx.x;
+  const int jsel = slot - p.w;  // position in the index list of a selected slot
+  const int kv0 = __ldg(p.cu_kv + b);
+  const int kv1 = __ldg(p.cu_kv + b + 1);
   const int cnt = p.cnt ? __ldg(p.cnt + bg) : 0;
-  const int lim = pos - p.w;
-  __shared__ int s_nsel[kThreads / 32];
-  {
-    int c = 0;
-    for (int i = threadIdx.x; i < cnt; i += kThreads) c += __ldg(idx + i) <= lim ? 1 : 0;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
-    if (lane == 0) s_nsel[warp] = c;
-  }
-  __syncthreads();
-  int n_sel = 0;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) n_sel += s_nsel[w];
+  const int cand = (jsel >= 0 && jsel < p.topk) ? __ldg(p.idx + size_t(bg) * p.topk + jsel) : -1;
+  const int pos = kv1 - kv0 - 1;  // the new token is the sequence's last position
   const int win_lo = max(0, pos - p.w + 1);
-  const int total = n_sel + (pos - win_lo + 1) * (p.w > 0 ? 1 : 0);
-  const int v0 = chunk * kChunk;
-  const int nk = max(0, min(kChunk, total - v0));
+  const int n_win = p.w > 0 ? pos - win_lo + 1 : 0;
+  int key = -1;
+  if (slot < n_win) key = win_lo + slot;
+  else if (jsel >= 0 && jsel < cnt && cand >= 0 && cand <= pos - p.w) key = cand;
+  skey[threadIdx.x] = key;
+  const uint32_t bal = __ballot_sync(0xffffffffu, key >= 0);
+  if (lane == 0) s_valid[warp] = bal;
+  __syncthreads();
+  uint32_t vmask[kChunk / 32];
+#pragma unroll
+  for (int w = 0; w < kChunk / 32; ++w) vmask[w] = s_valid[w];
   float* pml = p.part_ml + (size_t(bg) * p.n_chunks + chunk) * kHeads * 2;
-  if (nk == 0) {
+  if ((vmask[0] | vmask[1] | vmask[2] | vmask[3]) == 0) {
     if (threadIdx.x < kHeads) {
       pml[2 * threadIdx.x] = -INFINITY;
       pml[2 * threadIdx.x + 1] = 0.f;
     }
     return;
   }
-  for (int i = threadIdx.x; i < kChunk; i += kThreads) {
-    const int vi = v0 + i;
-    int key = -1;
-    if (i < nk) key = vi < n_sel ? __ldg(idx + vi) : win_lo + (vi - n_sel);
-    skey[i] = key;
-  }
-  __syncthreads();
-  // gather rows (invalid slots read row 0 of the sequence and are masked)
+  // gather: Q and K in one cp.async group, V in the next, so the QK product
+  // starts while V is still in flight; empty slots are zero-filled, not read
   load_q_tile(sq, p.q, b, g, p.Hq, p.G);
   constexpr int kChunks16 = kRowBytes / 16;
-  for (int i = threadIdx.x; i < kChunk * kChunks16; i += kThreads) {
-    const int r = i / kChunks16, c = i % kChunks16;
-    const int key = skey[r] >= 0 ? skey[r] : 0;
-    const size_t row = (size_t(kv0) + key) * p.Hkv + g;
-    const uint8_t* ks = reinterpret_cast<const uint8_t*>(p.k) + row * kRowBytes + c * 16;
-    const uint8_t* vs = reinterpret_cast<const uint8_t*>(p.v) + row * kRowBytes + c * 16;
-    const uint32_t off = FP8 ? uint32_t(r * 128 + ((c ^ (r & 7)) << 4)) : swz(r, c);
-    cp_async16(smem_u32(gk) + off, ks, true);
-    cp_async16(smem_u32(gv) + off, vs, true);
-  }
-  if (FP8) {
-    for (int i = threadIdx.x; i < kChunk; i += kThreads) {
-      const int key = skey[i] >= 0 ? skey[i] : 0;
-      const size_t row = (size_t(kv0) + key) * p.Hkv + g;
-      sks[i] = __ldg(p.k_scale + row);
-      svs[i] = __ldg(p.v_scale + row);
+  auto gather = [&](const void* src_base, uint8_t* dst) {
+    for (int i = threadIdx.x; i < kChunk * kChunks16; i += kThreads) {
+      const int r = i / kChunks16, c = i % kChunks16;
+      const int kr = skey[r];
+      const size_t row = (size_t(kv0) + (kr >= 0 ? kr : 0)) * p.Hkv + g;
+      const uint8_t* src = reinterpret_cast<const uint8_t*>(src_base) + row * kRowBytes + c * 16;
+      const uint32_t off = FP8 ? uint32_t(r * 128 + ((c ^ (r & 7)) << 4)) : swz(r, c);
+      cp_async16(smem_u32(dst) + off, src, kr >= 0);
     }
+    cp_async_commit();
+  };
+  gather(p.k, gk);
+  gather(p.v, gv);
+  if (FP8) {
+    const size_t row = (size_t(kv0) + (key >= 0 ? key : 0)) * p.Hkv + g;
+    sks[threadIdx.x] = key >= 0 ? __ldg(p.k_scale + row) : 0.f;
+    svs[threadIdx.x] = key >= 0 ? __ldg(p.v_scale + row) : 0.f;
   }
-  cp_async_commit();
-  cp_async_wait<0>();
+  if constexpr (FP8) cp_async_wait<0>();
+  else cp_async_wait<1>();
   __syncthreads();
   if constexpr (FP8) {
     // e4m3 -> bf16 is exact: expand both tiles in place into the swizzled
@@ -304,7 +300,7 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
       const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
       float x = s[nt][e] * cs;
       if (FP8) x *= sks[col];
-      if (col >= nk) x = -INFINITY;
+      if (!((vmask[nt >> 2] >> (col & 31)) & 1u)) x = -INFINITY;
       s[nt][e] = x;
       m[e >> 1] = fmaxf(m[e >> 1], x);
     }
@@ -338,6 +334,10 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+  if constexpr (!FP8) {
+    cp_async_wait<0>();  // V
+    __syncthreads();
+  }
   pv_bf16<kChunk>(pa, sv, o);
 
   // partials: unnormalised O and (m, l) per head
@@ -357,7 +357,14 @@ __global__ void __launch_bounds__(kThreads) sparse_decode_kernel(const SparsePar
   }
 }
 
-// Merge chunk partials: one CTA per (sequence, KV head), thread = (head, 16 dims).
+// Merge the chunk partials of one (sequence, KV head) by log-sum-exp. CTA
+// (bg, quarter) covers 16 heads: one warp per head, each lane 4 of the 128
+// dims. The lanes read the (m, l) of up to 32 chunks at once and the partial-O
+// loads of 8 chunks are issued before any of them is used (empty chunks are
+// not read), so the merge takes a few memory round trips however many chunks
+// there are.
+constexpr int kCombineHeads = 16;
+
 struct CombineParams {
   const float* part_o;
   const float* part_ml;
@@ -368,46 +375,72 @@ struct CombineParams {
   float* lse;             // [Hq, Tq] natural log
 };
 
-__global__ void __launch_bounds__(512) combine_kernel(const CombineParams p) {
+__global__ void __launch_bounds__(32 * kCombineHeads) combine_kernel(const CombineParams p) {
   const int bg = blockIdx.x;
   const int b = bg / p.Hkv, g = bg % p.Hkv;
-  const int h = threadIdx.x >> 3;     // 0..63
-  const int d0 = (threadIdx.x & 7) * 16;
-  if (h >= p.G) return;
-  const float* ml = p.part_ml + size_t(bg) * p.n_chunks * kHeads * 2;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 5);
+  if (h >= p.G) return;  // whole warps
+  const int n = p.n_chunks;
+  const float* ml = p.part_ml + size_t(bg) * n * kHeads * 2;
+  // this lane's float4 of chunk c: po[c * kHeads * 32]
+  const float4* po = reinterpret_cast<const float4*>(p.part_o) + (size_t(bg) * n * kHeads + h) * 32 + lane;
   float M = -INFINITY;
-  if (!p.normalised)
-    for (int c = 0; c < p.n_chunks; ++c) M = fmaxf(M, ml[(size_t(c) * kHeads + h) * 2]);
-  float acc[16];
+  if (!p.normalised) {
+    for (int c = lane; c < n; c += 32) M = fmaxf(M, ml[(size_t(c) * kHeads + h) * 2]);
 #pragma unroll
-  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-  float L = 0.f;
-  for (int c = 0; c < p.n_chunks; ++c) {
-    float wgt = 1.f;
-    if (!p.normalised) {
-      const float mc = ml[(size_t(c) * kHeads + h) * 2];
-      if (mc == -INFINITY) continue;
-      wgt = ex2(mc - M);
-      L += wgt * ml[(size_t(c) * kHeads + h) * 2 + 1];
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+  }
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float L = 0.f;  // this lane's chunks
+  auto add = [&](float wk, const float4& v) {
+    // a chunk without keys has weight 0 and an unwritten partial: skip it
+    if (wk != 0.f) {
+      acc.x = fmaf(wk, v.x, acc.x);
+      acc.y = fmaf(wk, v.y, acc.y);
+      acc.z = fmaf(wk, v.z, acc.z);
+      acc.w = fmaf(wk, v.w, acc.w);
     }
-    const float4* src = reinterpret_cast<const float4*>(p.part_o + ((size_t(bg) * p.n_chunks + c) * kHeads + h) * 128 + d0);
+  };
+  for (int c0 = 0; c0 < n; c0 += 32) {
+    float wl = 1.f;  // weight of chunk c0 + lane
+    if (!p.normalised) {
+      wl = 0.f;
+      const int c = c0 + lane;
+      if (c < n) {
+        const float mc = ml[(size_t(c) * kHeads + h) * 2];
+        if (mc != -INFINITY) {
+          wl = ex2(mc - M);
+          L += wl * ml[(size_t(c) * kHeads + h) * 2 + 1];
+        }
+      }
+    }
+    const int nc = min(32, n - c0);
+    int k = 0;
+    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (; k + 8 <= nc; k += 8) {
+      float wk[8];
+      float4 v[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float4 v4 = src[e];
-      acc[4 * e + 0] += wgt * v4.x;
-      acc[4 * e + 1] += wgt * v4.y;
-      acc[4 * e + 2] += wgt * v4.z;
-      acc[4 * e + 3] += wgt * v4.w;
+      for (int u = 0; u < 8; ++u) {
+        wk[u] = __shfl_sync(0xffffffffu, wl, k + u);
+        v[u] = wk[u] != 0.f ? po[size_t(c0 + k + u) * kHeads * 32] : zero;  // empty chunks are not read
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) add(wk[u], v[u]);
+    }
+    for (; k < nc; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, wl, k);
+      if (wk != 0.f) add(wk, po[size_t(c0 + k) * kHeads * 32]);
     }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
   const float inv = p.normalised ? 1.f : (L > 0.f ? 1.f / L : 0.f);
   const int hq = g * p.G + h;
-  uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(b) * p.Hq + hq) * 128 + d0);
-  dst[0] = make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
-                      pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
-  dst[1] = make_uint4(pack_bf16(acc[8] * inv, acc[9] * inv), pack_bf16(acc[10] * inv, acc[11] * inv),
-                      pack_bf16(acc[12] * inv, acc[13] * inv), pack_bf16(acc[14] * inv, acc[15] * inv));
-  if (d0 == 0 && p.lse) {
+  *reinterpret_cast<uint2*>(p.o + (size_t(b) * p.Hq + hq) * 128 + lane * 4) =
+      make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+  if (lane == 0 && p.lse) {
     float lse2;
     if (p.normalised) lse2 = p.lse2_in[size_t(bg) * kHeads + h];
     else lse2 = L > 0.f ? M + __log2f(L) : -INFINITY;
@@ -598,18 +631,25 @@ __global__ void __launch_bounds__(kThreads) full_decode_kernel(const FullParams 
   }
 }
 
-// lse2 per (sequence, KV head, head) from the pass-1 partials
-__global__ void __launch_bounds__(64) lse_combine_kernel(const float* part_ml, int n_split, float* lse2) {
-  const int bg = blockIdx.x, h = threadIdx.x;
+// lse2 per (sequence, KV head, head) from the pass-1 partials: CTA (bg,
+// quarter), one warp per head, the lanes strided over the splits.
+__global__ void __launch_bounds__(32 * kCombineHeads) lse_combine_kernel(const float* part_ml, int n_split,
+                                                                         float* lse2) {
+  const int bg = blockIdx.x, lane = threadIdx.x & 31;
+  const int h = blockIdx.y * kCombineHeads + (threadIdx.x >> 5);
   const float* ml = part_ml + size_t(bg) * n_split * kHeads * 2;
   float M = -INFINITY;
-  for (int s = 0; s < n_split; ++s) M = fmaxf(M, ml[(size_t(s) * kHeads + h) * 2]);
+  for (int s = lane; s < n_split; s += 32) M = fmaxf(M, ml[(size_t(s) * kHeads + h) * 2]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   float L = 0.f;
-  for (int s = 0; s < n_split; ++s) {
+  for (int s = lane; s < n_split; s += 32) {
     const float m = ml[(size_t(s) * kHeads + h) * 2];
     if (m > -INFINITY) L += ex2(m - M) * ml[(size_t(s) * kHeads + h) * 2 + 1];
   }
-  lse2[size_t(bg) * kHeads + h] = L > 0.f ? M + __log2f(L) : -INFINITY;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+  if (lane == 0) lse2[size_t(bg) * kHeads + h] = L > 0.f ? M + __log2f(L) : -INFINITY;
 }
 
 }  // namespace dec

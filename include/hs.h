@@ -182,7 +182,12 @@ HS_API hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel,
  * FP8 e4m3 (the HySparse2 key-data table sizes an FP8 KV cache); FP8 values
  * decode as x = scale[token, kv_head] * e4m3(code), with separate fp32 scale
  * arrays for K and V ([T_kv, H_kv]; NULL for bf16).
- * split_k: number of key chunks per sequence (0 = automatic).
+ * The visible set of each (sequence, KV head) is cut into 128-key chunks, one
+ * CTA each, and the chunks' partials are merged by log-sum-exp.
+ * split_k: 0 = one chunk per 128 keys of k + w (automatic); a positive value
+ * below that count is HS_ERR_UNSUPPORTED, a larger one is accepted and the
+ * automatic count is used. Negative values are rejected.
+ * An empty batch (T_q = 0) returns HS_OK without touching any pointer.
  * Requires n_b = 1 for every sequence and sel->q_tile = 1.
  */
 HS_API hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel,

@@ -94,6 +94,27 @@ def test_host_validation_errors(lib):
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG
 
 
+def test_batch_without_new_tokens_returns_before_touching_pointers(lib):
+    """Sequences with no new tokens: every call returns HS_OK on the host with
+    null data, index and workspace pointers (nothing is launched)."""
+    from hybrid_sparse_attention_tma_b200 import _lib as L
+    vl = _varlen([0, 0, 0], [0, 64, 164], hq=64, hkv=1, d=128)
+    dec = L.HsSel(1, 1, 16, 8)
+    blk = L.HsSel(64, 64, 2, 0)
+    n = None
+    assert lib.hs_full_attn_select(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, n, n, 0, n) == L.HS_OK
+    assert lib.hs_topk_select(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, 0, n) == L.HS_OK
+    assert lib.hs_sparse_attn_prefill(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, n, n, n, 0, n) == L.HS_OK
+    assert lib.hs_sparse_swa_gated_prefill(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, 128, n, n, n, n, n,
+                                           n, n, 0, n) == L.HS_OK
+    assert lib.hs_swa_gated(ctypes.byref(vl), 128, n, n, n, n, n, n, n, 0, n) == L.HS_OK
+    assert lib.hs_sparse_attn_decode(ctypes.byref(vl), ctypes.byref(dec), n, L.HS_KV_BF16, n, n, n, n, n, n, 0, n, n,
+                                     n, 0, n) == L.HS_OK
+    # a batch of no sequences at all is malformed
+    assert lib.hs_sparse_attn_decode(ctypes.byref(_varlen([0], [0], hq=64, hkv=1, d=128)), ctypes.byref(dec), n,
+                                     L.HS_KV_BF16, n, n, n, n, n, n, 0, n, n, n, 0, n) == L.HS_ERR_INVALID_ARG
+
+
 def test_workspace_size_every_op_at_workload_shapes(lib):
     """Every op sizes a workspace (header + scratch) for the benchmarked shapes."""
     import workloads as W

@@ -260,7 +260,8 @@ def test_bounded_wait_timeout_reports_and_context_survives():
 
 def test_empty_batch_is_a_no_op():
     """Every call accepts a batch without new tokens (empty tensors, null data
-    pointers) and returns without launching; the block runner passes through."""
+    pointers) and returns without launching; the block runner passes through.
+    The decode entry point likewise accepts a batch of no sequences."""
     w = W.Workload("e0", ctx=(64, 100), new=(0, 0), n_q_heads=8, n_kv_heads=2, head_dim=128, q_tile=64, block=64,
                    topk=2, window=0, n_sparse=2, swa_window=128)
     inp = W.make_block_inputs(w, device="cuda", seed=1)
