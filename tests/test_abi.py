@@ -3,6 +3,7 @@ rejects bad arguments on the host before any launch (no GPU needed)."""
 import ctypes
 import os
 import re
+import sys
 
 import pytest
 
@@ -169,3 +170,39 @@ def test_cpu_baseline_samples_until_the_time_budget():
     assert len(toks) == 3 and all(t > 0 for t in times)  # capped by max_tiles
     toks, times = bench.time_oracle(w, 2, repeats=2)
     assert toks == 2 * w.q_tile and len(times) == 2
+
+
+def test_clock_summary_median_max_and_reasons():
+    sys.path.insert(0, ROOT)
+    import bench
+    lines = ["0, 1965, 1965, 610.2, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+             "0, 1755, 1965, 998.7, 0x4, Not Active, Not Active, Not Active, Active\n",
+             "0, 1740, 1965, 1001.0, 0x4, Not Active, Not Active, Not Active, Active\n",
+             "0, [N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active\n",
+             "garbage\n"]
+    c = bench.summarize_clocks(lines)
+    assert c == {"sm_mhz": 1755.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c = bench.summarize_clocks(["0, 1200, 1965, 700, 0x8, Active, Not Active, Active, Not Active\n"])
+    assert c["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert bench.summarize_clocks([]) is None
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference: the oracle on the host cores, one JSON line
+    with the keys the driver reads (tiny workload, so it runs in seconds)."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload",
+                          "tiny", "--steps", "2", "--warmup", "3"], capture_output=True, text=True, timeout=600,
+                         cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ["impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"]:
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
