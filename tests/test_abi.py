@@ -18,7 +18,8 @@ def lib():
 
 
 def header_functions():
-    src = open(os.path.join(ROOT, "include", "hs.h")).read()
+    with open(os.path.join(ROOT, "include", "hs.h")) as f:
+        src = f.read()
     return sorted(set(re.findall(r"HS_API\s+[\w\s\*]+?\b(hs_\w+)\s*\(", src)))
 
 
@@ -147,7 +148,8 @@ def test_bench_traffic_needs_matching_source_hash(tmp_path, monkeypatch):
     for f in bench.KERNEL_SOURCES:  # the hash is taken over the kernel sources under ROOT
         dst = tmp_path / f
         dst.parent.mkdir(parents=True, exist_ok=True)
-        dst.write_bytes(open(os.path.join(ROOT, f), "rb").read())
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            dst.write_bytes(fh.read())
     h = bench.src_hash()
     (prof / "traffic.json").write_text(json.dumps({"attn_fwd_full:hys_block": {"src_hash": h,
                                                                                 "dram_bytes_per_launch": 123}}))

@@ -22,6 +22,7 @@ RNG = np.random.default_rng(7)
 
 # ---------------------------------------------------------------- number formats
 
+@pytest.mark.filterwarnings("ignore:invalid value encountered in cast:RuntimeWarning")  # NaN patterns
 def test_bf16_decode_matches_torch_for_all_patterns():
     bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     ours = O.bf16_to_f64(bits)
