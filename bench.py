@@ -1,20 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of one hybrid block (1 full layer + N sparse layers) on B200.
 
-Workload (default): HySparse block-level prefill, 1 x 32768 tokens, 32 query
-heads / 8 KV heads, d = 128, 64-token blocks, top-16, separate SWA window 128
-+ sigmoid gate, 1 full layer feeding 3 sparse layers; seeded synthetic bf16
-N(0,1) inputs with 1 % planted keys. A "step" is one pass of the whole block:
-hs_full_attn_select -> hs_topk_select -> 3 x hs_sparse_swa_gated_prefill (the
-sparse branch, the own-cache window branch and the gate of one layer in one
-launch). The per-step working set (~2 GB) is larger than the 126 MB L2.
+Workload (default, the largest single-GPU configuration): agentic ragged
+chunked prefill -- 4 sequences with cached contexts {262144, 131072, 65536,
+16384} and new chunks {8192, 4096, 8192, 2048} queries, 64 query heads / 1 KV
+head, d = 128, token-level top-1024 + forced recent 128, tile 64, 1 full layer
+feeding 11 sparse layers; seeded synthetic bf16 N(0,1) inputs with 0.5 %
+planted keys. A "step" is one pass of the whole block: hs_full_attn_select
+(forward + token-score pass) -> hs_topk_select -> 11 x hs_sparse_attn_prefill.
+The per-step working set (~5 GB) is larger than the 126 MB L2. On one GPU the
+same line also carries a shorter measurement of every other configuration
+("workloads"): the block-level HySparse prefill (with its own-cache window
+branch and gate fused into each sparse layer), the token-level HySparse2
+prefill, decode with bf16 and FP8 KV, and the tiny case.
 
 Multi-GPU (torchrun): every rank runs its own independent block (its own
 sequences); no data-path collective. value = tokens of all ranks / max-over-
 ranks time ("weak" scaling).
 
 --impl reference: the fp64 CPU oracle on host cores, timed on a bounded
-sample of the same workload (one selection tile of 64 queries per step).
+sample of the same workload (one selection tile of 64 queries of the
+shortest-context sequence per step).
 """
 from __future__ import annotations
 
@@ -49,7 +55,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="hys_block", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default="agentic", choices=list(W.WORKLOADS))
+    ap.add_argument("--no-extra", action="store_true",
+                    help="measure only --workload (skip the other configurations' short runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8-kv", action="store_true", help="decode: sparse layers read an FP8-e4m3 KV cache")
@@ -234,6 +242,38 @@ def visible_counts(w, idx, cnt):
     return float(total)
 
 
+def needle_recall(w, inp, idx, cnt):
+    """Share of planted keys that the sparse layers see from the query they
+    were aimed at: the key lies in that query's forced window, or its block is
+    in the top-k set of the query's tile and KV head. Reported overall and for
+    keys outside the window (where only the selection can find them)."""
+    if not inp.needles:
+        return None
+    import numpy as np
+    last = {}
+    for (b, j, p, h) in inp.needles:  # a key planted twice keeps its last aim (as the generator does)
+        last[(b, j, h // w.group)] = p
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    tile_base, tb = [], 0
+    for n in w.new:
+        tile_base.append(tb)
+        tb += -(-n // w.q_tile)
+    n_all = hit_all = n_out = hit_out = 0
+    for (b, j, g), p in last.items():
+        c_b = w.kv_lens[b] - w.new[b]
+        t = tile_base[b] + (p - c_b) // w.q_tile
+        in_win = w.window > 0 and j > p - w.window
+        sel = idx_h[t, g, :cnt_h[t, g]]
+        in_sel = bool(np.isin(j // w.block, sel))
+        n_all += 1
+        hit_all += int(in_win or in_sel)
+        if not in_win:
+            n_out += 1
+            hit_out += int(in_sel)
+    return {"needles": n_all, "recall": round(hit_all / n_all, 4), "outside_window": n_out,
+            "recall_outside_window": round(hit_out / n_out, 4) if n_out else None}
+
+
 def swa_pairs(w):
     tot = 0
     for c, n in zip(w.ctx, w.new):
@@ -242,7 +282,7 @@ def swa_pairs(w):
     return tot
 
 
-def bench_ours(args, world, rank, local):
+def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=None, workload_name=None):
     import torch.distributed as dist
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
@@ -250,17 +290,21 @@ def bench_ours(args, world, rank, local):
                                                   HS_KV_FP8_E4M3)
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
-    w = workload(args)
-    if args.fp8_kv:
+    w = workload(args) if w is None else w
+    steps = args.steps if steps is None else steps
+    fp8 = args.fp8_kv if fp8 is None else fp8
+    workload_name = args.workload if workload_name is None else workload_name
+    if fp8:
         w = w.with_(fp8_kv=True)
     inp, vl, blk, layers = make_runner(w, device, seed=rank_seed(w, rank))
     stream = torch.cuda.current_stream()
-    fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if args.fp8_kv else None
+    fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if fp8 else None
 
     for _ in range(max(3, args.warmup)):
         blk.forward(inp.q, inp.k, inp.v, layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
     torch.cuda.synchronize()
     hs.check_error(blk.ws)
+    recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"])
 
     kinds = ["full", "topk", "sparse"]
     L0 = layers[0]
@@ -340,8 +384,8 @@ def bench_ours(args, world, rank, local):
                           if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
     clocks.start()
     time.sleep(0.3)
-    ms_total = timed(step_graph.replay, args.steps)
-    n_kind = max(4, args.steps // 4)
+    ms_total = timed(step_graph.replay, steps)
+    n_kind = max(4, steps // 4)
     ms_flush = timed(flush_graph.replay, n_kind)
     kms = {kd: max(0.0, timed(kind_graphs[kd].replay, n_kind) - ms_flush) / (n_kind * reps) for kd in kinds}
     clk = clocks.stop()
@@ -351,7 +395,7 @@ def bench_ours(args, world, rank, local):
     vals = max_over_ranks([ms_total] + [kms[kd] for kd in kinds], device)
     ms_total = vals[0]
     kms = {kd: vals[i + 1] for i, kd in enumerate(kinds)}
-    ms_step = ms_total / args.steps
+    ms_step = ms_total / steps
     tokens = w.total_q
     value = whole_job_rate(world, tokens, ms_step)
 
@@ -382,7 +426,7 @@ def bench_ours(args, world, rank, local):
     if blk.decode:
         # full-layer decode: every K/V row once, Q, O, lse and the token scores
         entry("full", kms["full"], kv_bytes * 2 + q_bytes * 2 + n_tiles * hkv * nblk * 4, "hbm")
-        row = d * (1 if args.fp8_kv else 2) + (4 if args.fp8_kv else 0)
+        row = d * (1 if fp8 else 2) + (4 if fp8 else 0)
         entry("sparse", kms["sparse"], vis * 2 * row + q_bytes * 2, "hbm")
     else:
         entry("full", kms["full"], full_flops(w), "tensor")
@@ -397,28 +441,49 @@ def bench_ours(args, world, rank, local):
     dom = dict(kernels["full"])
     dom["kernel"] = ("full-layer decode (two split-K passes + combines)" if blk.decode
                      else "attn_fwd_kernel<d, full, B> (+ token-score pass when B = 1)")
-    dom["traffic"] = traffic_for("attn_fwd_full", args.workload)
+    dom["traffic"] = traffic_for("attn_fwd_full", workload_name)
     dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
 
     # ---- e2e through the public API with host buffers ----
     e2e = None
-    if not args.no_e2e:
+    if with_e2e and not args.no_e2e:
         e2e = bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv)
 
     kind = ("decode" if blk.decode else ("HySparse block-level prefill" if w.block > 1 else "HySparse2 token-level prefill"))
     desc = (f"{w.name}: {kind}, {w.batch}x ctx {list(w.ctx)[:4]} + new {list(w.new)[:4]} tokens, "
             f"{hq}/{hkv} heads, d={d}, B={w.block}, k={w.topk}, w={w.window}"
             + (f", SWA {w.swa_window}+gate" if w.swa_window else "")
-            + f", 1 full + {w.n_sparse} sparse" + (", FP8-e4m3 KV in the sparse layers" if args.fp8_kv else ""))
+            + f", 1 full + {w.n_sparse} sparse" + (", FP8-e4m3 KV in the sparse layers" if fp8 else ""))
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+           "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded N(0,1) bf16" + (", planted keys)" if w.needle_rate else ")"),
            "config": {"workload": desc, "tokens_per_step_per_gpu": tokens,
                       "l2": "step: inputs larger than L2; per-kernel times: L2 flushed before every call", "parallelism": f"independent blocks x{world}"},
            "roofline": dom, "kernels": kernels,
-           "gpu_launches": blk.launches_per_forward(len(layers)) * args.steps,
-           "clocks": clk, "e2e": e2e}
+           "gpu_launches": blk.launches_per_forward(len(layers)) * steps,
+           "needle_recall": recall, "clocks": clk, "e2e": e2e}
+    del step_graph, flush_graph, kind_graphs, flush, inp, blk, layers
+    torch.cuda.empty_cache()
+    return out
+
+
+EXTRA = [("hys_block", False), ("hys2_prefill", False), ("decode", False), ("decode", True), ("tiny", False)]
+
+
+def bench_extra(args, world, rank, local, headline):
+    """Short measurements of the other configurations (one GPU only): the
+    step rate, the per-kernel roofline entries and the needle recall of each."""
+    out = {}
+    for name, fp8 in EXTRA:
+        if name == headline and not fp8:
+            continue
+        r = bench_ours(args, world, rank, local, w=W.WORKLOADS[name], steps=max(4, min(args.steps, 10)),
+                       with_e2e=False, fp8=fp8, workload_name=name)
+        key = name + ("_fp8" if fp8 else "")
+        out[key] = {k: r[k] for k in ["value", "unit", "ms_per_step", "steps", "kernels", "needle_recall",
+                                      "clocks", "gpu_launches"]}
+        out[key]["workload"] = r["config"]["workload"]
     return out
 
 
@@ -476,22 +541,67 @@ def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
 
 # ---------------------------------------------------------------- oracle side
 
-def oracle_sample(w, tile_id, inp_cpu):
-    """Run the oracle's whole block on one selection tile; returns tokens."""
-    import numpy as np
-    import oracle as O
-    from oracle.block import run_block
-    q = O.bf16_to_f64(W.bf16_bits(inp_cpu.q))
-    k = O.bf16_to_f64(W.bf16_bits(inp_cpu.k))
-    v = O.bf16_to_f64(W.bf16_bits(inp_cpu.v))
+class _LazyF64:
+    """float64 view of a bf16 CPU tensor: only the slices the oracle reads are
+    decoded (a whole C5 block in fp64 would take ~18 GB of host memory)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, idx):
+        import numpy as np
+        import oracle as O
+        conv = (lambda i: torch.from_numpy(i.astype(np.int64)) if isinstance(i, np.ndarray) else i)
+        idx = tuple(conv(i) for i in idx) if isinstance(idx, tuple) else conv(idx)
+        return O.bf16_to_f64(W.bf16_bits(self.t[idx]))
+
+
+def oracle_inputs(inp_cpu):
+    """The block's inputs as the oracle reads them (float64 values of the bf16 data)."""
     layers = []
     for L in inp_cpu.layers:
-        d = {"q": O.bf16_to_f64(W.bf16_bits(L.q))}
+        d = {"q": _LazyF64(L.q)}
         if L.k_swa is not None:
-            d.update(k_swa=O.bf16_to_f64(W.bf16_bits(L.k_swa)), v_swa=O.bf16_to_f64(W.bf16_bits(L.v_swa)),
-                     gamma=L.gamma.double().numpy())
+            d.update(k_swa=_LazyF64(L.k_swa), v_swa=_LazyF64(L.v_swa), gamma=L.gamma.double().numpy())
         layers.append(d)
-    return q, k, v, layers
+    return _LazyF64(inp_cpu.q), _LazyF64(inp_cpu.k), _LazyF64(inp_cpu.v), layers
+
+
+def sample_tiles(w):
+    """Selection tiles the oracle is timed on: from the middle outwards of the
+    sequence with the shortest context (the oracle's cost per query grows with
+    the keys it sees, so its rate on these tiles is an upper bound of its rate
+    on the whole workload)."""
+    import oracle as O
+    tiles = O.make_tiles(w.cu_q(), w.cu_kv(), w.q_tile)
+    b = min(range(w.batch), key=lambda i: (w.kv_lens[i] if w.new[i] > 0 else 1 << 62))
+    own = [t.index for t in tiles if t.seq == b]
+    mid = len(own) // 2
+    order = [own[mid]]
+    for d in range(1, len(own)):
+        for j in (mid + d, mid - d):
+            if 0 <= j < len(own):
+                order.append(own[j])
+    return order, tiles
+
+
+def host_description():
+    """CPU model and the number of cores this process may use."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except Exception:
+        nproc = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": nproc}
 
 
 def oracle_threads():
@@ -504,35 +614,33 @@ def oracle_threads():
 
 
 def time_oracle(w, n_tiles_sample=1, repeats=1, min_seconds=0.0, max_tiles=8):
-    """Time the oracle's whole block on middle selection tiles, one tile per
-    run: `repeats` runs of the first `n_tiles_sample` tiles, or (min_seconds >
-    0) successive tiles until that much oracle time or `max_tiles` tiles.
-    Returns (tokens per run, run times)."""
-    import oracle as O
+    """Time the oracle's whole block on selection tiles of sample_tiles(w), one
+    tile per run: `repeats` runs of the first `n_tiles_sample` tiles, or
+    (min_seconds > 0) successive tiles until that much oracle time or
+    `max_tiles` tiles. Returns (tokens per run, run times)."""
     from oracle.block import run_block
     inp = W.make_block_inputs(w, device="cpu")
-    q, k, v, layers = oracle_sample(w, 0, inp)
-    n_t = w.n_tiles()
-    tiles = O.make_tiles(w.cu_q(), w.cu_kv(), w.q_tile)
+    q, k, v, layers = oracle_inputs(inp)
+    order, tiles = sample_tiles(w)
 
     def run(ids):
         t = time.perf_counter()
         run_block(q, k, v, layers, w.cu_q(), w.cu_kv(), w.n_kv_heads, w.q_tile, w.block, w.topk, w.window,
-                  w.swa_window, tile_ids=ids)
+                  w.swa_window, tile_ids=ids, compact=True)
         return time.perf_counter() - t
 
     if min_seconds > 0:
         toks, times = [], []
         i = 0
-        while (sum(times) < min_seconds and i < max_tiles) or not times:
-            tid = min(n_t - 1, n_t // 2 + i)
+        while (sum(times) < min_seconds and i < max_tiles and i < len(order)) or not times:
+            tid = order[i % len(order)]
             times.append(run([tid]))
             toks.append(tiles[tid].n)
             i += 1
         return toks, times
-    mids = [min(n_t - 1, n_t // 2 + i) for i in range(n_tiles_sample)]
-    toks = sum(tiles[i].n for i in mids)
-    return toks, [run(mids) for _ in range(repeats)]
+    ids = order[:n_tiles_sample]
+    toks = sum(tiles[i].n for i in ids)
+    return toks, [run(ids) for _ in range(repeats)]
 
 
 def bench_reference(args, world, rank):
@@ -545,14 +653,17 @@ def bench_reference(args, world, rank):
     s = sum(timed) / len(timed)
     value = toks / s
     cores = oracle_threads()
-    sample = f"selection tile {w.n_tiles() // 2} ({toks} queries, all layers of the block) per step"
+    order, tiles = sample_tiles(w)
+    t0 = tiles[order[0]]
+    sample = (f"selection tile {t0.index} of sequence {t0.seq} (its shortest context; {toks} queries at positions "
+              f"{t0.pos0}..{t0.last_pos}, all layers of the block) per step; tokens/s extrapolated from it")
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(s * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded N(0,1) bf16, 1% planted keys)",
+            "data": "synthetic (seeded N(0,1) bf16" + (", planted keys)" if w.needle_rate else ")"),
             "config": {"workload": w.name, "tokens_per_step": toks},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "extrapolated": True, **host_description()},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
 
@@ -571,13 +682,18 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     out = bench_ours(args, world, rank, local)
+    if world == 1 and not args.no_extra and not args.tokens:
+        out["workloads"] = bench_extra(args, world, rank, local, args.workload)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w = workload(args)
         toks, times = time_oracle(w, min_seconds=10.0)
         out["cpu_baseline"] = {"value": round(sum(toks) / sum(times), 3), "unit": "tokens/s",
-                               "cores": oracle_threads(), "kind": "oracle",
-                               "sample": f"{len(toks)} middle selection tiles ({sum(toks)} queries), whole block, "
-                                         f"{sum(times):.1f} s"}
+                               "cores": oracle_threads(), "kind": "oracle", "extrapolated": True,
+                               **host_description(),
+                               "sample": f"{len(toks)} selection tiles of the shortest-context sequence "
+                                         f"({sum(toks)} queries), whole block, {sum(times):.1f} s; tokens/s "
+                                         f"extrapolated from those tiles (an upper bound: longer contexts cost "
+                                         f"the oracle more per query)"}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

@@ -194,6 +194,27 @@ cudaError_t set_smem(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
+// A kernel's dynamic shared-memory limit is a per-device attribute: each call
+// site keeps one of these and raises the limit once on every device it
+// launches on (devices beyond the mask get the call on every launch).
+struct PerDeviceOnce {
+  std::mutex mu;
+  uint64_t done[2] = {0, 0};  // devices 0..127
+};
+
+template <typename K>
+cudaError_t set_smem_once(PerDeviceOnce& once, K kernel, int bytes) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  if (dev < 0 || dev >= 128) return set_smem(kernel, bytes);
+  std::lock_guard<std::mutex> lock(once.mu);
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (once.done[dev >> 6] & bit) return cudaSuccess;
+  const cudaError_t e = set_smem(kernel, bytes);
+  if (e == cudaSuccess) once.done[dev >> 6] |= bit;
+  return e;
+}
+
 // Tensor maps of one attention launch. g / o (the other branch's output and
 // this call's output, boxes of 64 rows = 64/G queries x G heads) are used by
 // the gated sliding-window call only; the other calls pass copies of q.
@@ -207,11 +228,8 @@ hs_status launch_attn(const Maps& m, const attn::Params& p, const attn::Sched& s
   auto kern = attn::attn_fwd_kernel<D, MODE, SB>;
   constexpr int need = attn::smem_bytes<D, (MODE == attn::kSparse && SB == 0) || MODE == attn::kFused>();
   constexpr int smem = need > 116 * 1024 ? need : 116 * 1024;
-  static bool configured = false;
-  if (!configured) {
-    if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
-    configured = true;
-  }
+  static PerDeviceOnce once;
+  if (set_smem_once(once, kern, smem) != cudaSuccess) return HS_ERR_CUDA;
   kern<<<grid, attn::threads_for<MODE, SB>(), smem, st>>>(m.q, m.k, m.v, m.kb, m.vb, m.g, m.o, m.ks, m.vs, p, sc);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
@@ -267,7 +285,10 @@ bool is_decode(const hs_varlen* vl, const hs_sel* sel) {
 
 // Resident CTAs of the full-layer decode pass 2 (the larger one) on this GPU.
 int full_decode_slots() {
-  static int slots = 0;
+  static int slots_of[129] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) dev = 128;
+  int& slots = slots_of[dev];
   if (slots == 0) {
     int per_sm = 0;
     constexpr int bytes = dec::full_smem_bytes<true>();
@@ -353,16 +374,25 @@ __global__ void debug_wait_kernel(WaitCtl wc) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, wc, 99);
 }
 
+// 2^x on the FMA pipe, as the softmax uses it, over an array (self test).
+__global__ void debug_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long stride = 2LL * gridDim.x * blockDim.x;
+  for (long long i = 2LL * (blockIdx.x * (long long)blockDim.x + threadIdx.x); i < n; i += stride) {
+    const bool two = i + 1 < n;
+    float a, b;
+    exp2_poly_pair(x[i], two ? x[i + 1] : 0.f, a, b);
+    y[i] = a;
+    if (two) y[i + 1] = b;
+  }
+}
+
 template <int D>
 hs_status launch_token_scores(const Maps& m, const tscore::Params& p, const SeqTable& st, const int* prefix,
                               int grid, cudaStream_t s) {
   auto kern = tscore::token_scores_kernel<D>;
   constexpr int smem = tscore::smem_bytes<D>() > 116 * 1024 ? tscore::smem_bytes<D>() : 116 * 1024;
-  static bool configured = false;
-  if (!configured) {
-    if (set_smem(kern, smem) != cudaSuccess) return HS_ERR_CUDA;
-    configured = true;
-  }
+  static PerDeviceOnce once;
+  if (set_smem_once(once, kern, smem) != cudaSuccess) return HS_ERR_CUDA;
   kern<<<grid, tscore::kThreads, smem, s>>>(m.q, m.k, p, st, prefix);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
@@ -385,16 +415,14 @@ void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
 
 // Device address of the scratch array on the current device. In host code the
 // array's name is only a host-side stand-in, so the address is looked up once
-// per device (with that device current) and cached; the error header is
-// zeroed at that point.
-hs_status noalloc_scratch(void** out, cudaStream_t s) {
+// per device (with that device current) and cached.
+hs_status noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return HS_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   if (!g_noalloc_ptr[dev]) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return HS_ERR_CUDA;
-    if (cudaMemsetAsync(ptr, 0, kHeaderBytes, s) != cudaSuccess) return HS_ERR_CUDA;
     g_noalloc_ptr[dev] = ptr;
   }
   *out = g_noalloc_ptr[dev];
@@ -498,13 +526,10 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
     fp.part_o = reinterpret_cast<float*>(after_ml + align_up(size_t(bg) * dec::kHeads * 4, 256));
     fp.scores = scores;
     fp.nblk = nblk;
-    static bool configured = false;
-    if (!configured) {
-      if (set_smem(dec::full_decode_kernel<false>, dec::full_smem_bytes<false>()) != cudaSuccess ||
-          set_smem(dec::full_decode_kernel<true>, dec::full_smem_bytes<true>()) != cudaSuccess)
-        return HS_ERR_CUDA;
-      configured = true;
-    }
+    static PerDeviceOnce once1, once2;
+    if (set_smem_once(once1, dec::full_decode_kernel<false>, dec::full_smem_bytes<false>()) != cudaSuccess ||
+        set_smem_once(once2, dec::full_decode_kernel<true>, dec::full_smem_bytes<true>()) != cudaSuccess)
+      return HS_ERR_CUDA;
     const dim3 grid(ns, bg);
     dec::full_decode_kernel<false><<<grid, dec::kThreads, dec::full_smem_bytes<false>(), s>>>(fp);
     dec::lse_combine_kernel<<<dim3(bg, dec::kHeads / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(
@@ -761,13 +786,10 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   char* w = reinterpret_cast<char*>(ws);
   p.part_o = reinterpret_cast<float*>(w + kHeaderBytes);
   p.part_ml = reinterpret_cast<float*>(w + align_up(kHeaderBytes + size_t(bg) * nc * dec::kHeads * 128 * 4, 256));
-  static bool configured = false;
-  if (!configured) {
-    if (set_smem(dec::sparse_decode_kernel<false>, dec::sparse_smem_bytes<false>()) != cudaSuccess ||
-        set_smem(dec::sparse_decode_kernel<true>, dec::sparse_smem_bytes<true>()) != cudaSuccess)
-      return HS_ERR_CUDA;
-    configured = true;
-  }
+  static PerDeviceOnce once1, once2;
+  if (set_smem_once(once1, dec::sparse_decode_kernel<false>, dec::sparse_smem_bytes<false>()) != cudaSuccess ||
+      set_smem_once(once2, dec::sparse_decode_kernel<true>, dec::sparse_smem_bytes<true>()) != cudaSuccess)
+    return HS_ERR_CUDA;
   const dim3 grid(nc, bg);
   if (fp8)
     dec::sparse_decode_kernel<true><<<grid, dec::kThreads, dec::sparse_smem_bytes<true>(), s>>>(p);
@@ -862,7 +884,10 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
   if (cap < 1) return HS_ERR_WORKSPACE;  // sequence longer than the fixed scratch can serve
   cudaStream_t s = S(stream);
   void* scratch = nullptr;
-  if ((st = noalloc_scratch(&scratch, s)) != HS_OK) return st;
+  if ((st = noalloc_scratch(&scratch)) != HS_OK) return st;
+  // every call starts from a clear error header (stream-ordered), so a wait
+  // that gave up in an earlier unchecked call is not reported by this one
+  if (cudaMemsetAsync(scratch, 0, kHeaderBytes, s) != cudaSuccess) return HS_ERR_CUDA;
   const int n_tiles = n_tiles_of(vl, T);
   if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
     return HS_ERR_CUDA;
@@ -901,7 +926,6 @@ hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* sel, co
     if (cudaMemcpy(&e, scratch, sizeof(e), cudaMemcpyDeviceToHost) != cudaSuccess) return HS_ERR_CUDA;
     if (e.flag != 0) {
       last_err = e;
-      if (cudaMemset(scratch, 0, sizeof(ErrWord)) != cudaSuccess) return HS_ERR_CUDA;
       return HS_ERR_TIMEOUT;
     }
   }
@@ -921,6 +945,17 @@ hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, 
   if (timeout_ns == 0 || timeout_ns > 2000000000ull) return HS_ERR_INVALID_ARG;
   WaitCtl wc{reinterpret_cast<ErrWord*>(ws), timeout_ns};
   debug_wait_kernel<<<1, 32, 0, S(stream)>>>(wc);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_debug_exp2_poly(const float* x, float* y, int64_t n, hs_stream_t stream) {
+  if (n < 0) return HS_ERR_INVALID_ARG;
+  if (n == 0) return HS_OK;
+  if (!x || !y || (reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(y) & 3))
+    return HS_ERR_INVALID_ARG;
+  const long long pairs = (n + 1) / 2;
+  const int grid = int(std::min<long long>(4LL * num_sms(), (pairs + 255) / 256));
+  debug_exp2_poly_kernel<<<grid, 256, 0, S(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 

@@ -35,6 +35,12 @@
  * Errors: each call validates its arguments on the host before launching
  *   anything and returns a status. Device-side failures (a bounded wait that
  *   gave up) are recorded in the workspace and reported by hs_check_error().
+ * Limits: at most 256 sequences per call (batch <= 256); a larger batch is
+ *   HS_ERR_UNSUPPORTED (split it into several calls). Per call the packed
+ *   token axes hold at most 2^31 - 1 rows.
+ * Devices: calls may target any device; each kernel's shared-memory limit is
+ *   raised once per device it runs on. Calls on one device that share a
+ *   workspace must be ordered (one stream, or events between streams).
  */
 #ifndef HS_H_
 #define HS_H_
@@ -255,8 +261,12 @@ HS_API hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* 
  * and outputs exactly as for hs_full_attn_select. No call allocates or frees
  * memory (no cudaMalloc/cudaFree or allocating library routine).
  * First call per device: looks up the array's device address with the device
- * current and zeroes its error header (an async memset on `stream`); make that
- * first call before any stream capture on that device.
+ * current (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture on that device.
+ * Every call first zeroes the array's 256-byte error header with an async
+ * memset on `stream`, so a bounded wait that gave up during an earlier call
+ * made with check = 0 is never reported by a later call; such a failure is
+ * visible only to a check != 0 call on the same launch.
  * Sharing: every call on a device uses the same array and leaves its contents
  * behind. Calls whose kernels overlap on the GPU (e.g. on two streams without
  * ordering) race on it and give wrong results; order them.
@@ -283,6 +293,17 @@ HS_API hs_status hs_full_attn_select_noalloc(const hs_varlen* vl, const hs_sel* 
  * This is the same bounded wait every pipelined kernel uses.
  */
 HS_API hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, hs_stream_t stream);
+
+/*
+ * hs_debug_exp2_poly -- self test of the softmax's FMA-pipe exponential (no
+ * counterpart on the pages). Writes y[i] = 2^x[i] as the attention kernels
+ * compute one in four of their exponentials: a Cody-Waite split 2^x = 2^j * 2^f
+ * (j = nearest integer, |f| <= 1/2) with a degree-3 minimax polynomial for
+ * 2^f (relative error 7.5e-5), inputs clamped to >= -125 (so x < -125 gives
+ * about 2^-125). x, y: device arrays of n fp32 values (4-byte aligned); n = 0
+ * is a no-op; n < 0 or a null / misaligned pointer is HS_ERR_INVALID_ARG.
+ */
+HS_API hs_status hs_debug_exp2_poly(const float* x, float* y, int64_t n, hs_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -25,30 +25,35 @@ def tile_rows(cu_q, cu_kv, T, tile_ids):
 
 
 def run_block(q, k, v, layers, cu_q, cu_kv, n_kv_heads, T, B, topk, w, swa_window=0,
-              tile_ids: Optional[Sequence[int]] = None, idx_override=None, cnt_override=None):
+              tile_ids: Optional[Sequence[int]] = None, idx_override=None, cnt_override=None,
+              compact: bool = False):
     """layers: list of dicts with 'q' and optionally 'k_swa', 'v_swa', 'gamma'.
 
     Returns a dict with o_full, lse_full, scores, idx, cnt and per-layer outputs.
     When idx_override/cnt_override are given, the sparse layers use those
     indices (used to check outputs independently of legitimate tie-band
-    differences in the selection).
+    differences in the selection). With ``compact`` (and tile_ids) every
+    output holds only the sampled tiles' rows, tile after tile, instead of
+    full-size arrays with the other rows left NaN / 0.
     """
+    compact = compact and tile_ids is not None
     o_full, lse_full = O.full_attention(q, k, v, cu_q, cu_kv, n_kv_heads, tiles_T=T,
-                                        tile_ids=tile_ids)
+                                        tile_ids=tile_ids, compact=compact)
     scores = O.importance_scores(q, k, lse_full, cu_q, cu_kv, n_kv_heads, T, B,
-                                 tile_ids=tile_ids)
-    idx, cnt = O.topk_select(scores, cu_q, cu_kv, T, B, topk, tile_ids=tile_ids)
+                                 tile_ids=tile_ids, compact=compact)
+    idx, cnt = O.topk_select(scores, cu_q, cu_kv, T, B, topk, tile_ids=tile_ids, compact=compact)
     use_idx = idx if idx_override is None else idx_override
     use_cnt = cnt if cnt_override is None else cnt_override
     outs = []
     rows = None if tile_ids is None else tile_rows(cu_q, cu_kv, T, tile_ids)
     for L in layers:
         o_sp, lse_sp = O.sparse_attention(L["q"], k, v, use_idx, use_cnt, cu_q, cu_kv, T, B, w,
-                                          tile_ids=tile_ids)
+                                          tile_ids=tile_ids, compact=compact)
         if swa_window > 0:
             o_swa, _ = O.swa_attention(L["q"], L["k_swa"], L["v_swa"], cu_q, cu_kv, swa_window,
-                                       row_ids=rows)
-            o = O.gated_merge(L["gamma"], o_sp, o_swa)
+                                       row_ids=rows, compact=compact)
+            gamma = L["gamma"][rows] if compact else L["gamma"]
+            o = O.gated_merge(gamma, o_sp, o_swa)
         else:
             o = o_sp
         outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o})

@@ -94,6 +94,11 @@ def test_host_validation_errors(lib):
     assert fused(128, 16, 24) == L.HS_ERR_INVALID_ARG
     assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG
+    # exp2 self test: empty is a no-op, null / misaligned / negative sizes are rejected before launch
+    assert lib.hs_debug_exp2_poly(None, None, 0, None) == L.HS_OK
+    assert lib.hs_debug_exp2_poly(None, None, 4, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_debug_exp2_poly(16, 18, 4, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_debug_exp2_poly(16, 32, -1, None) == L.HS_ERR_INVALID_ARG
 
 
 def test_batch_without_new_tokens_returns_before_touching_pointers(lib):
