@@ -14,9 +14,12 @@ same line also carries a shorter measurement of every other configuration
 branch and gate fused into each sparse layer), the token-level HySparse2
 prefill, decode with bf16 and FP8 KV, and the tiny case.
 
-Multi-GPU (torchrun): every rank runs its own independent block (its own
-sequences); no data-path collective. value = tokens of all ranks / max-over-
-ranks time ("weak" scaling).
+Multi-GPU (torchrun): one block is partitioned over the ranks
+(hybrid_sparse_attention_tma_b200.shard): decode by sequences, GQA prefill by
+KV heads (neither has a data-path collective), MQA prefill by contiguous
+ranges of selection tiles whose K / V come from one all-gather of every
+rank's token shard inside each timed step. value = the block's tokens / the
+slowest rank's step time ("strong" scaling: the total work is fixed).
 
 --impl reference: the fp64 CPU oracle on host cores, timed on a bounded
 sample of the same workload (one selection tile of 64 queries of the
@@ -61,8 +64,12 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--fp8-kv", action="store_true", help="decode: sparse layers read an FP8-e4m3 KV cache")
+    ap.add_argument("--exclusive", action="store_true",
+                    help="window-exclusive top-k: k global tokens drawn before the last query's forced window")
     ap.add_argument("--tokens", type=int, default=0,
                     help="scale a single-sequence workload to this many new tokens (profiling cases)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="decode: keep this many of the workload's sequences (profiling cases)")
     return ap.parse_args()
 
 
@@ -70,6 +77,10 @@ def workload(args) -> W.Workload:
     w = W.WORKLOADS[args.workload]
     if args.tokens and w.batch == 1:
         w = W.scaled(w, ctx=(0,), new=(args.tokens,))
+    if args.batch and args.batch < w.batch:
+        w = W.scaled(w, ctx=w.ctx[:args.batch], new=w.new[:args.batch])
+    if args.exclusive:
+        w = w.with_(exclusive=True)
     return w
 
 
@@ -181,9 +192,53 @@ def dist_setup():
     return world, rank, local
 
 
-def rank_seed(w, rank: int) -> int:
-    """Seed of the independent block rank `rank` processes (distinct per rank)."""
-    return 1000 + w.config_index + 7919 * rank
+def block_seed(w) -> int:
+    """Seed of the block's synthetic inputs (the same on every rank)."""
+    return 1000 + w.config_index
+
+
+def rank_problem(w, world: int, rank: int, device, fp8: bool = False):
+    """This rank's part of one block (shard.plan): the whole block's inputs are
+    drawn from one seed on every rank and sliced. Returns (w_r, inputs_r,
+    kv_own): kv_own = (k_shard, v_shard, total_rows, kv_row0, kv_rows) for a
+    query-tile shard, whose K / V arrive by all-gather in each step; else
+    None. Needles are kept only on one rank."""
+    from hybrid_sparse_attention_tma_b200 import shard as S
+    full = W.make_block_inputs(w, device=device, seed=block_seed(w))
+    if fp8 and full.k_fp8 is None:
+        full.k_fp8, full.k_scale = W.quantize_e4m3_per_token(full.k)
+        full.v_fp8, full.v_scale = W.quantize_e4m3_per_token(full.v)
+    if world == 1:
+        return w, full, None
+    sh = S.plan(w.ctx, w.new, w.n_q_heads, w.n_kv_heads, w.q_tile, world, w.topk, w.block, w.window,
+                w.n_sparse)[rank]
+    opt = lambda t, f: None if t is None else f(t).contiguous()  # noqa: E731
+    if sh.kind == "kv_heads":
+        G = w.group
+        hq = slice(sh.kv_head0 * G, (sh.kv_head0 + sh.n_kv_heads) * G)
+        hk = slice(sh.kv_head0, sh.kv_head0 + sh.n_kv_heads)
+        w_r = w.with_(n_q_heads=sh.n_q_heads, n_kv_heads=sh.n_kv_heads)
+        cq, ck = (lambda t: t[:, hq]), (lambda t: t[:, hk])
+        layers = [W.LayerInputs(opt(L.q, cq), opt(L.k_swa, ck), opt(L.v_swa, ck), opt(L.gamma, cq))
+                  for L in full.layers]
+        inp = W.BlockInputs(w_r, opt(full.q, cq), opt(full.k, ck), opt(full.v, ck), layers, full.cu_q, full.cu_kv,
+                            [], opt(full.k_fp8, ck), opt(full.v_fp8, ck), opt(full.k_scale, ck),
+                            opt(full.v_scale, ck))
+        return w_r, inp, None
+    w_r = W.scaled(w, ctx=sh.ctx, new=sh.new)
+    qs = slice(sh.q_row0, sh.q_row0 + w_r.total_q)
+    ks = slice(sh.kv_row0, sh.kv_row0 + sh.kv_rows)
+    cq, ck = (lambda t: t[qs]), (lambda t: t[ks])
+    layers = [W.LayerInputs(opt(L.q, cq), opt(L.k_swa, ck), opt(L.v_swa, ck), opt(L.gamma, cq)) for L in full.layers]
+    cu_q = torch.tensor(w_r.cu_q(), dtype=torch.int32, device=device)
+    cu_kv = torch.tensor(w_r.cu_kv(), dtype=torch.int32, device=device)
+    inp = W.BlockInputs(w_r, opt(full.q, cq), opt(full.k, ck), opt(full.v, ck), layers, cu_q, cu_kv, [],
+                        opt(full.k_fp8, ck), opt(full.v_fp8, ck), opt(full.k_scale, ck), opt(full.v_scale, ck))
+    if sh.kind == "batch":
+        return w_r, inp, None
+    lo, hi = S.token_shard(w.total_kv, rank, world)
+    kv_own = (full.k[lo:hi].contiguous(), full.v[lo:hi].contiguous(), w.total_kv, sh.kv_row0, sh.kv_rows)
+    return w_r, inp, kv_own
 
 
 def max_over_ranks(values, device):
@@ -196,19 +251,20 @@ def max_over_ranks(values, device):
     return t.tolist()
 
 
-def whole_job_rate(world: int, tokens_per_rank: int, ms_per_step: float) -> float:
-    """Tokens/s of the whole job: every rank's tokens over the slowest rank's step time."""
-    return world * tokens_per_rank / (ms_per_step / 1e3)
+def whole_job_rate(block_tokens: int, ms_per_step: float) -> float:
+    """Tokens/s of the whole job: the block's new tokens (all ranks together)
+    over the slowest rank's step time."""
+    return block_tokens / (ms_per_step / 1e3)
 
 
-def make_runner(w, device, seed):
+def make_runner(w_r, inp, device):
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200.block import HybridBlock, SparseLayerIn
-    inp = W.make_block_inputs(w, device=device, seed=seed)
-    vl = hs.Varlen(w.cu_q(), w.cu_kv(), w.n_q_heads, w.n_kv_heads, w.head_dim, device=device)
-    blk = HybridBlock(vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device)
+    vl = hs.Varlen(w_r.cu_q(), w_r.cu_kv(), w_r.n_q_heads, w_r.n_kv_heads, w_r.head_dim, device=device)
+    blk = HybridBlock(vl, w_r.q_tile, w_r.block, w_r.topk, w_r.window, w_r.swa_window, device=device,
+                      exclusive=w_r.exclusive)
     layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
-    return inp, vl, blk, layers
+    return vl, blk, layers
 
 
 def visible_counts(w, idx, cnt):
@@ -296,15 +352,27 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     workload_name = args.workload if workload_name is None else workload_name
     if fp8:
         w = w.with_(fp8_kv=True)
-    inp, vl, blk, layers = make_runner(w, device, seed=rank_seed(w, rank))
+    w_block = w
+    w, inp, kv_own = rank_problem(w_block, world, rank, device, fp8)
+    vl, blk, layers = make_runner(w, inp, device)
     stream = torch.cuda.current_stream()
     fp8_kv = (inp.k_fp8, inp.v_fp8, inp.k_scale, inp.v_scale) if fp8 else None
+    if kv_own is not None:
+        # query-tile shard: every step all-gathers the ranks' K / V token shards
+        from hybrid_sparse_attention_tma_b200 import shard as S
+        k_own, v_own, kv_total, kv_r0, kv_n = kv_own
+
+        def gather_kv():
+            kf = S.all_gather_kv(k_own, kv_total)
+            vf = S.all_gather_kv(v_own, kv_total)
+            return kf[kv_r0:kv_r0 + kv_n], vf[kv_r0:kv_r0 + kv_n]
+        inp.k, inp.v = gather_kv()
 
     for _ in range(max(3, args.warmup)):
         blk.forward(inp.q, inp.k, inp.v, layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
     torch.cuda.synchronize()
     hs.check_error(blk.ws)
-    recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"])
+    recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"]) if world == 1 else None
 
     kinds = ["full", "topk", "sparse"]
     L0 = layers[0]
@@ -338,10 +406,19 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     # kind are captured once in CUDA graphs and replayed; the library enqueues
     # only launches and memsets inside a call (its one-time set-up ran during
     # warm-up), so capture is safe.
-    step_graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(step_graph):
-        blk.forward(inp.q, inp.k, inp.v, layers, stream=torch.cuda.current_stream(), fp8_kv=fp8_kv,
-                    intermediates=False)
+    # (a step that holds the K / V all-gather runs eagerly: no collective
+    # inside a captured graph, and such prefill steps are long)
+    step_graph = None
+    if kv_own is None:
+        step_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(step_graph):
+            blk.forward(inp.q, inp.k, inp.v, layers, stream=torch.cuda.current_stream(), fp8_kv=fp8_kv,
+                        intermediates=False)
+
+    def eager_step():
+        kk, vv = gather_kv()
+        blk.forward(inp.q, kk, vv, layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
+    run_step = step_graph.replay if step_graph is not None else eager_step
     # Per-kernel times with a cold L2: every call is preceded by a write of
     # twice the L2 size, and the same flushes alone are timed and subtracted
     # (the sparse decode's gathered rows, ~40 MB, would otherwise stay in L2
@@ -361,7 +438,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                 call(kd, torch.cuda.current_stream())
         kind_graphs[kd] = gk
     for _ in range(2):
-        step_graph.replay()
+        run_step()
         flush_graph.replay()
         for gk in kind_graphs.values():
             gk.replay()
@@ -384,7 +461,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                           if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
     clocks.start()
     time.sleep(0.3)
-    ms_total = timed(step_graph.replay, steps)
+    ms_total = timed(run_step, steps)
     n_kind = max(4, steps // 4)
     ms_flush = timed(flush_graph.replay, n_kind)
     kms = {kd: max(0.0, timed(kind_graphs[kd].replay, n_kind) - ms_flush) / (n_kind * reps) for kd in kinds}
@@ -397,7 +474,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     kms = {kd: vals[i + 1] for i, kd in enumerate(kinds)}
     ms_step = ms_total / steps
     tokens = w.total_q
-    value = whole_job_rate(world, tokens, ms_step)
+    value = whole_job_rate(w_block.total_q, ms_step)
 
     # ---- algorithmic work of each kernel launch ----
     hbm, tf_burst, tf_sust, src = peaks()
@@ -439,7 +516,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])
-    dom["kernel"] = ("full-layer decode (two split-K passes + combines)" if blk.decode
+    dom["kernel"] = ("full_decode_tc_kernel (both exact passes, one persistent launch)" if blk.decode
                      else "attn_fwd_kernel<d, full, B> (+ token-score pass when B = 1)")
     dom["traffic"] = traffic_for("attn_fwd_full", workload_name)
     dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
@@ -447,25 +524,33 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     # ---- e2e through the public API with host buffers ----
     e2e = None
     if with_e2e and not args.no_e2e:
-        e2e = bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv)
+        e2e = bench_e2e(args, w, inp, vl, blk, layers, device, w_block.total_q, fp8_kv)
 
-    kind = ("decode" if blk.decode else ("HySparse block-level prefill" if w.block > 1 else "HySparse2 token-level prefill"))
-    desc = (f"{w.name}: {kind}, {w.batch}x ctx {list(w.ctx)[:4]} + new {list(w.new)[:4]} tokens, "
-            f"{hq}/{hkv} heads, d={d}, B={w.block}, k={w.topk}, w={w.window}"
-            + (f", SWA {w.swa_window}+gate" if w.swa_window else "")
-            + f", 1 full + {w.n_sparse} sparse" + (", FP8-e4m3 KV in the sparse layers" if fp8 else ""))
+    kind = ("decode" if blk.decode else ("HySparse block-level prefill" if w_block.block > 1 else "HySparse2 token-level prefill"))
+    desc = (f"{w_block.name}: {kind}, {w_block.batch}x ctx {list(w_block.ctx)[:4]} + new {list(w_block.new)[:4]} tokens, "
+            f"{w_block.n_q_heads}/{w_block.n_kv_heads} heads, d={d}, B={w_block.block}, k={w_block.topk}, w={w_block.window}"
+            + (f", SWA {w_block.swa_window}+gate" if w_block.swa_window else "")
+            + f", 1 full + {w_block.n_sparse} sparse" + (", FP8-e4m3 KV in the sparse layers" if fp8 else ""))
     out = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
            "steps": steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
            "data": "synthetic (seeded N(0,1) bf16" + (", planted keys)" if w.needle_rate else ")"),
-           "config": {"workload": desc, "tokens_per_step_per_gpu": tokens,
-                      "l2": "step: inputs larger than L2; per-kernel times: L2 flushed before every call", "parallelism": f"independent blocks x{world}"},
+           "config": {"workload": desc, "tokens_per_step": w_block.total_q, "tokens_this_rank": tokens,
+                      "l2": "step: inputs larger than L2; per-kernel times: L2 flushed before every call", "parallelism": (f"one block over {world} GPUs: {shard_kind(w_block, world)}" if world > 1
+                                      else "one block, one GPU")},
            "roofline": dom, "kernels": kernels,
            "gpu_launches": blk.launches_per_forward(len(layers)) * steps,
            "needle_recall": recall, "clocks": clk, "e2e": e2e}
-    del step_graph, flush_graph, kind_graphs, flush, inp, blk, layers
+    del step_graph, flush_graph, kind_graphs, flush, inp, blk, layers, kv_own
     torch.cuda.empty_cache()
     return out
+
+
+def shard_kind(w, world):
+    from hybrid_sparse_attention_tma_b200 import shard as S
+    sh = S.plan(w.ctx, w.new, w.n_q_heads, w.n_kv_heads, w.q_tile, world, w.topk, w.block, w.window, w.n_sparse)
+    return {"batch": "sequences per rank", "kv_heads": "KV heads per rank",
+            "q_tiles": "selection tiles per rank + K/V all-gather"}[sh[0].kind]
 
 
 EXTRA = [("hys_block", False), ("hys2_prefill", False), ("decode", False), ("decode", True), ("tiny", False)]
@@ -487,7 +572,7 @@ def bench_extra(args, world, rank, local, headline):
     return out
 
 
-def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
+def bench_e2e(args, w, inp, vl, blk, layers, device, block_tokens, fp8_kv=None):
     """Same metric through HybridBlock.forward with the step's inputs copied
     from pinned host memory each step and the last layer's output read back."""
     from hybrid_sparse_attention_tma_b200.block import SparseLayerIn
@@ -535,7 +620,7 @@ def bench_e2e(args, w, inp, vl, blk, layers, device, world, fp8_kv=None):
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
     ms = max_over_ranks([ms], device)[0]
-    return {"value": round(whole_job_rate(world, w.total_q, ms), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+    return {"value": round(whole_job_rate(block_tokens, ms), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
@@ -682,7 +767,7 @@ def main():
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     out = bench_ours(args, world, rank, local)
-    if world == 1 and not args.no_extra and not args.tokens:
+    if world == 1 and not args.no_extra and not args.tokens and not args.batch:
         out["workloads"] = bench_extra(args, world, rank, local, args.workload)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         w = workload(args)

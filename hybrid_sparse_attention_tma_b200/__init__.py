@@ -63,8 +63,10 @@ class Varlen:
         return sum((b - a + T - 1) // T for a, b in zip(self.cu_q_list, self.cu_q_list[1:]))
 
 
-def Sel(q_tile: int, block: int, topk: int, window: int) -> L.HsSel:
-    return L.HsSel(q_tile, block, topk, window)
+def Sel(q_tile: int, block: int, topk: int, window: int, exclusive: bool = False) -> L.HsSel:
+    """Selection parameters; exclusive=True draws the top-k only from blocks
+    that end before the forced window of the tile's last query."""
+    return L.HsSel(q_tile, block, topk, window, L.HS_SEL_WINDOW_EXCLUSIVE if exclusive else 0)
 
 
 def workspace_size(op: int, vl: Varlen, sel: Optional[L.HsSel] = None) -> int:

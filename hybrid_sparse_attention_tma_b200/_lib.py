@@ -33,7 +33,10 @@ class HsVarlen(ctypes.Structure):
 
 class HsSel(ctypes.Structure):
     _fields_ = [("q_tile", ctypes.c_int32), ("block", ctypes.c_int32), ("topk", ctypes.c_int32),
-                ("window", ctypes.c_int32)]
+                ("window", ctypes.c_int32), ("flags", ctypes.c_int32)]
+
+
+HS_SEL_WINDOW_EXCLUSIVE = 1
 
 
 class HsError(RuntimeError):

@@ -26,9 +26,9 @@ class SparseLayerIn:
 
 class HybridBlock:
     def __init__(self, vl: Varlen, q_tile: int, block: int, topk: int, window: int, swa_window: int = 0,
-                 device="cuda", fused: bool = True):
+                 device="cuda", fused: bool = True, exclusive: bool = False):
         self.vl = vl
-        self.sel = Sel(q_tile, block, topk, window)
+        self.sel = Sel(q_tile, block, topk, window, exclusive)
         self.swa_window = swa_window
         # prefill layers with a window branch run as one fused launch
         # (hs_sparse_swa_gated_prefill) unless fused=False (two launches)

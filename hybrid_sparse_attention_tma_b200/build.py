@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhs.so")
 SOURCES = ["api.cu"]
-HEADERS = ["hs_common.cuh", "attn_fwd.cuh", "topk.cuh", "seqtable.cuh", "token_scores.cuh", "decode.cuh"]
+HEADERS = ["hs_common.cuh", "attn_fwd.cuh", "topk.cuh", "seqtable.cuh", "token_scores.cuh",
+           "decode_tc.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

@@ -13,7 +13,7 @@
 #include "attn_fwd.cuh"
 #include "hs_common.cuh"
 #include "seqtable.cuh"
-#include "decode.cuh"
+#include "decode_tc.cuh"
 #include "token_scores.cuh"
 #include "topk.cuh"
 
@@ -124,6 +124,7 @@ hs_status check_sel(const hs_sel* sel) {
   if (sel->q_tile < 1 || sel->block < 1 || sel->topk < 0 || sel->window < 0) return HS_ERR_INVALID_ARG;
   if (sel->topk > 4096) return HS_ERR_UNSUPPORTED;
   if (!is_pow2(sel->block) || sel->block > 128 || (sel->block > 1 && sel->block < 8)) return HS_ERR_UNSUPPORTED;
+  if (sel->flags & ~HS_SEL_WINDOW_EXCLUSIVE) return HS_ERR_INVALID_ARG;
   return HS_OK;
 }
 
@@ -255,7 +256,7 @@ hs_status dispatch_full(int d, int B, const Maps& m, const attn::Params& p, cons
 
 WaitCtl wait_ctl(void* ws) { return WaitCtl{reinterpret_cast<ErrWord*>(ws), g_timeout_ns}; }
 
-size_t full_decode_ws_bytes(const Shape& sh);
+size_t full_decode_ws_bytes(const hs_varlen* vl, const Shape& sh);
 bool is_decode(const hs_varlen* vl, const hs_sel* sel);
 
 // Block-maximum spill of one CTA (double-buffered): per 128-key tile of the
@@ -265,7 +266,7 @@ size_t spill_floats_per_cta(int max_kv, int B) {
 }
 
 size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
-  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= dec::kHeads) return full_decode_ws_bytes(sh);
+  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= 64) return full_decode_ws_bytes(vl, sh);
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
     b += size_t(num_sms()) * spill_floats_per_cta(sh.max_kv, sel->block) * sizeof(float);
@@ -283,66 +284,87 @@ bool is_decode(const hs_varlen* vl, const hs_sel* sel) {
   return true;
 }
 
-// Resident CTAs of the full-layer decode pass 2 (the larger one) on this GPU.
-int full_decode_slots() {
-  static int slots_of[129] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) dev = 128;
-  int& slots = slots_of[dev];
-  if (slots == 0) {
-    int per_sm = 0;
-    constexpr int bytes = dec::full_smem_bytes<true>();
-    if (set_smem(dec::full_decode_kernel<true>, bytes) == cudaSuccess &&
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, dec::full_decode_kernel<true>, dec::kThreads, bytes) ==
-            cudaSuccess &&
-        per_sm > 0)
-      slots = per_sm * num_sms();
-    else
-      slots = 2 * num_sms();
+// Full-layer decode on the tensor cores (decode_tc.cuh): keys per work item.
+// Pass 2 re-reads a unit's K about D = (one unit's chunks + two grids of
+// items) pass-1 items after pass 1 read it. Each item costs a few
+// microseconds of hand-offs besides its tiles, so items are long (up to 32
+// tiles of 128 keys, as long as every CTA gets two items per pass); an L2
+// budget (HS_DEC_L2_BUDGET_MB, off by default) can shorten them so that K
+// stays in L2 between the passes. Measured at 64 x 131072 keys: 1.28 ms with
+// 32-tile items against 1.62 / 2.04 ms with 8 / 4 tiles.
+#ifndef HS_DEC_MAX_TILES
+#define HS_DEC_MAX_TILES 32
+#endif
+#ifndef HS_DEC_L2_BUDGET_MB
+#define HS_DEC_L2_BUDGET_MB (1LL << 40)
+#endif
+#ifndef HS_DEC_DELAY_GRIDS
+#define HS_DEC_DELAY_GRIDS 2
+#endif
+int full_decode_chunk_keys(const hs_varlen* vl, const Shape& sh) {
+  long long tiles = 0, unit_tiles = 0;
+  for (int b = 0; b < vl->batch; ++b) {
+    const long long t = (vl->cu_kv_host[b + 1] - vl->cu_kv_host[b] + 127) / 128;
+    tiles += t;
+    unit_tiles = std::max(unit_tiles, t);
   }
-  return slots;
+  tiles *= sh.Hkv;
+  const long long grid = num_sms();
+  long long T = HS_DEC_MAX_TILES;
+  while (T > 1 && (2 * T * grid + unit_tiles) * 32768LL > (HS_DEC_L2_BUDGET_MB << 20)) --T;
+  while (T > 1 && tiles / T < 2 * grid) --T;
+  return int(T) * 128;
 }
 
-// Key splits per (sequence, KV head): the grid (splits x sequences) should
-// fill whole waves of resident CTAs -- e.g. 10 splits x 64 sequences on 296
-// slots ran 3 waves for 2.16 waves of work. Take the fewest splits whose last
-// wave is at least 97 % full (else the best found), with at least one full
-// wave and one 64-key chunk per split.
-int full_decode_splits(const Shape& sh) {
-  const int bg = sh.batch * sh.Hkv;
-  const int cap = std::max(1, std::min(256, (sh.max_kv + dec::kFullChunk - 1) / dec::kFullChunk));
-  const int slots = full_decode_slots();
-  int best = 1;
-  double best_eff = -1.0;
-  for (int ns = 1; ns <= cap; ++ns) {
-    const long long ctas = (long long)bg * ns;
-    if (ctas < slots && ns < cap) continue;
-    const long long waves = (ctas + slots - 1) / slots;
-    const double eff = double(ctas) / double(waves * slots);
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = ns;
-    }
-    if (eff >= 0.97) break;
-  }
-  return best;
+// Workspace: header | sync words (work counter + 3 per unit) | O accumulators
+// [units][64][128] fp32 | pass-1 fp64 totals [units][64] (these three are
+// zeroed together before each launch) | lse2 [units][64].
+struct FullDecodeWs {
+  size_t sync, o_acc, unit_l, lse2, total;
+};
+
+FullDecodeWs full_decode_layout(const hs_varlen* vl, const Shape& sh) {
+  (void)vl;
+  const size_t U = size_t(sh.batch) * sh.Hkv;
+  FullDecodeWs w;
+  w.sync = kHeaderBytes;
+  w.o_acc = align_up(w.sync + (1 + 3 * U) * sizeof(int), 256);
+  w.unit_l = align_up(w.o_acc + U * 64 * 128 * sizeof(float), 256);
+  w.lse2 = align_up(w.unit_l + U * 64 * sizeof(double), 256);
+  w.total = align_up(w.lse2 + U * 64 * sizeof(float), 256);
+  return w;
 }
 
-size_t full_decode_ws_bytes(const Shape& sh) {
-  const size_t bg = size_t(sh.batch) * sh.Hkv;
-  const size_t ns = full_decode_splits(sh);
-  return align_up(kHeaderBytes + bg * ns * dec::kHeads * 2 * 4, 256) + align_up(bg * dec::kHeads * 4, 256) +
-         align_up(bg * ns * dec::kHeads * 128 * 4, 256);
+size_t full_decode_ws_bytes(const hs_varlen* vl, const Shape& sh) { return full_decode_layout(vl, sh).total; }
+
+// Sparse decode on the tensor cores (decode_tc.cuh, namespace sdec): each
+// (sequence, KV head) unit's slot space (window w + k selected tokens) is cut
+// into 128-slot tiles and those into `nsplit` ranges, one work item each.
+struct SparseDecodePlan {
+  int unit_tiles, nsplit, tiles_per_split, n_items;
+};
+
+SparseDecodePlan sparse_decode_plan(const Shape& sh, const hs_sel* sel, int split_k) {
+  SparseDecodePlan pl;
+  const int U = sh.batch * sh.Hkv;
+  pl.unit_tiles = std::max(1, (sel->topk + sel->window + 127) / 128);
+  int want = split_k > 0 ? split_k : std::max(1, num_sms() / std::max(1, U));
+  want = std::min(want, pl.unit_tiles);
+  pl.tiles_per_split = (pl.unit_tiles + want - 1) / want;
+  pl.nsplit = (pl.unit_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;  // no empty range
+  pl.n_items = U * pl.nsplit;
+  return pl;
 }
 
-int sparse_decode_chunks(const hs_sel* sel) {
-  return std::max(1, (sel->topk + sel->window + dec::kChunk - 1) / dec::kChunk);
-}
-
+// Workspace: header | per-unit item counters | partial (m, l) [items][64] |
+// partial O [items][64][128] fp32 (used when a unit has more than one range).
+// Sized for the automatic split or any split_k up to the unit's tile count
+// (the largest split is one tile per item).
 size_t sparse_decode_ws_bytes(const Shape& sh, const hs_sel* sel) {
-  const size_t bg = size_t(sh.batch) * sh.Hkv;
-  const size_t nc = sparse_decode_chunks(sel);
-  return align_up(kHeaderBytes + bg * nc * dec::kHeads * 128 * 4, 256) + align_up(bg * nc * dec::kHeads * 2 * 4, 256);
+  const size_t U = size_t(sh.batch) * sh.Hkv;
+  const size_t items = U * size_t(std::max(1, (sel->topk + sel->window + 127) / 128));
+  return align_up(kHeaderBytes + U * sizeof(int), 256) + align_up(items * 64 * 2 * sizeof(float), 256) +
+         align_up(items * 64 * 128 * sizeof(float), 256);
 }
 
 // Token-level scores: items are (tile, KV head, 512-key range) up to the
@@ -504,50 +526,58 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   cudaStream_t s = S(stream);
   if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
     return HS_ERR_CUDA;
-  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= dec::kHeads) {
-    // one query per sequence: exact two-pass split-K over each sequence's keys
-    const int bg = sh.batch * sh.Hkv;
-    const int ns = full_decode_splits(sh);
-    dec::FullParams fp{};
-    fp.q = reinterpret_cast<const __nv_bfloat16*>(q);
-    fp.k = reinterpret_cast<const __nv_bfloat16*>(k);
-    fp.v = reinterpret_cast<const __nv_bfloat16*>(v);
-    fp.cu_kv = vl->cu_kv;
-    fp.Hq = sh.Hq;
-    fp.Hkv = sh.Hkv;
-    fp.G = sh.G;
-    fp.n_split = ns;
-    fp.max_kv = sh.max_kv;
-    fp.scale_log2 = sh.scale * 1.4426950408889634f;
+  if (is_decode(vl, sel) && sh.d == 128 && sh.G <= 64) {
+    // one query per sequence: both exact passes in one persistent tcgen05 kernel
+    const int U = sh.batch * sh.Hkv;
+    if (U > dtc::kMaxUnits) return HS_ERR_UNSUPPORTED;
+    static dtc::Sched dsc;  // large; filled under the lock
+    static std::mutex dmu;
+    std::lock_guard<std::mutex> lock(dmu);
+    const int chunk_keys = full_decode_chunk_keys(vl, sh);
+    dsc.n_units = U;
+    dsc.Hkv = sh.Hkv;
+    dsc.chunk_keys = chunk_keys;
+    for (int b = 0; b <= sh.batch; ++b) dsc.cu_kv[b] = vl->cu_kv_host[b];
+    std::vector<int> nch(U);
+    dsc.chunk_base[0] = 0;
+    for (int u = 0; u < U; ++u) {
+      const int b = u / sh.Hkv;
+      nch[u] = (vl->cu_kv_host[b + 1] - vl->cu_kv_host[b] + chunk_keys - 1) / chunk_keys;
+      dsc.chunk_base[u + 1] = dsc.chunk_base[u] + nch[u];
+    }
+    // pass-2 items trail the pass-1 stream by D items (see decode_tc.cuh)
+    int s_max = 0;
+    for (int u = 0; u < U; ++u) s_max = std::max(s_max, nch[u]);
+    dsc.n1 = dsc.chunk_base[U];
+    dsc.delay = std::min(dsc.n1, s_max + HS_DEC_DELAY_GRIDS * num_sms());
+    dsc.n_items = 2 * dsc.n1;
+    const FullDecodeWs lay = full_decode_layout(vl, sh);
     char* w = reinterpret_cast<char*>(ws);
-    fp.part_ml = reinterpret_cast<float*>(w + kHeaderBytes);
-    char* after_ml = w + align_up(kHeaderBytes + size_t(bg) * ns * dec::kHeads * 2 * 4, 256);
-    fp.lse2 = reinterpret_cast<float*>(after_ml);
-    fp.part_o = reinterpret_cast<float*>(after_ml + align_up(size_t(bg) * dec::kHeads * 4, 256));
-    fp.scores = scores;
-    fp.nblk = nblk;
-    static PerDeviceOnce once1, once2;
-    if (set_smem_once(once1, dec::full_decode_kernel<false>, dec::full_smem_bytes<false>()) != cudaSuccess ||
-        set_smem_once(once2, dec::full_decode_kernel<true>, dec::full_smem_bytes<true>()) != cudaSuccess)
+    dtc::Params dp{};
+    dp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+    dp.G = sh.G;
+    dp.Hq = sh.Hq;
+    dp.Hkv = sh.Hkv;
+    dp.Tq = int(sh.Tq);
+    dp.nblk = nblk;
+    dp.scale_log2 = sh.scale * 1.4426950408889634f;
+    dp.sync = reinterpret_cast<int*>(w + lay.sync);
+    dp.o_acc = reinterpret_cast<float*>(w + lay.o_acc);
+    dp.lse2 = reinterpret_cast<float*>(w + lay.lse2);
+    dp.unit_l = reinterpret_cast<double*>(w + lay.unit_l);
+    dp.scores = scores;
+    dp.o = reinterpret_cast<__nv_bfloat16*>(o);
+    dp.lse = lse;
+    dp.wc = wait_ctl(ws);
+    if (cudaMemsetAsync(w + lay.sync, 0, lay.lse2 - lay.sync, s) != cudaSuccess) return HS_ERR_CUDA;
+    Maps m;
+    if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 1) || !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) ||
+        !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128))
       return HS_ERR_CUDA;
-    const dim3 grid(ns, bg);
-    dec::full_decode_kernel<false><<<grid, dec::kThreads, dec::full_smem_bytes<false>(), s>>>(fp);
-    dec::lse_combine_kernel<<<dim3(bg, dec::kHeads / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(
-        fp.part_ml, ns, fp.lse2);
-    dec::full_decode_kernel<true><<<grid, dec::kThreads, dec::full_smem_bytes<true>(), s>>>(fp);
-    dec::CombineParams cp{};
-    cp.part_o = fp.part_o;
-    cp.part_ml = fp.part_ml;
-    cp.n_chunks = ns;
-    cp.Hq = sh.Hq;
-    cp.Hkv = sh.Hkv;
-    cp.G = sh.G;
-    cp.Tq = int(sh.Tq);
-    cp.normalised = true;
-    cp.lse2_in = fp.lse2;
-    cp.o = reinterpret_cast<__nv_bfloat16*>(o);
-    cp.lse = lse;
-    dec::combine_kernel<<<dim3(bg, (sh.G + dec::kCombineHeads - 1) / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(cp);
+    static PerDeviceOnce once;
+    if (set_smem_once(once, dtc::full_decode_tc_kernel, dtc::smem_bytes()) != cudaSuccess) return HS_ERR_CUDA;
+    const int grid = std::min(num_sms(), std::max(1, dsc.n_items));
+    dtc::full_decode_tc_kernel<<<grid, dtc::kThreads, dtc::smem_bytes(), s>>>(m.q, m.k, m.v, dp, dsc);
     return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
   }
 
@@ -626,6 +656,8 @@ hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* sc
   p.nblk = (sh.max_kv + sel->block - 1) / sel->block;
   p.B = sel->block;
   p.k = sel->topk;
+  p.w = sel->window;
+  p.exclusive = (sel->flags & HS_SEL_WINDOW_EXCLUSIVE) ? 1 : 0;
   const long long rows = (long long)table.n_tiles * sh.Hkv;
   if (rows > (1LL << 31) - 1) return HS_ERR_UNSUPPORTED;
   if (p.nblk <= topk::kStageMax)
@@ -754,7 +786,7 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   if ((st = check_sel(sel)) != HS_OK) return st;
   if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
   if (!is_decode(vl, sel)) return HS_ERR_INVALID_ARG;  // one query per sequence, q_tile = block = 1
-  if (sh.d != 128 || sh.G > dec::kHeads) return HS_ERR_UNSUPPORTED;
+  if (sh.d != 128 || sh.G > 64) return HS_ERR_UNSUPPORTED;
   if (kv_dtype != HS_KV_BF16 && kv_dtype != HS_KV_FP8_E4M3) return HS_ERR_INVALID_ARG;
   const bool fp8 = kv_dtype == HS_KV_FP8_E4M3;
   if (!q || !k || !v || !o || (sel->topk > 0 && (!idx || !cnt)) || (fp8 && (!k_scale || !v_scale)))
@@ -763,50 +795,56 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   if (split_k < 0) return HS_ERR_INVALID_ARG;
   if (sel->topk + sel->window == 0) return HS_ERR_INVALID_ARG;  // empty visible set
   if (!ws || ws_bytes < sparse_decode_ws_bytes(sh, sel)) return HS_ERR_WORKSPACE;
-  const int bg = sh.batch * sh.Hkv;
-  const int nc = sparse_decode_chunks(sel);  // 128 keys per chunk; split_k only caps it
-  if (split_k > 0 && split_k < nc) return HS_ERR_UNSUPPORTED;
+  const int U = sh.batch * sh.Hkv;
+  if (U > dtc::sdec::kMaxUnits) return HS_ERR_UNSUPPORTED;
+  const SparseDecodePlan pl = sparse_decode_plan(sh, sel, split_k);
   cudaStream_t s = S(stream);
-  dec::SparseParams p{};
-  p.q = reinterpret_cast<const __nv_bfloat16*>(q);
-  p.k = k;
-  p.v = v;
-  p.k_scale = k_scale;
-  p.v_scale = v_scale;
+  char* w = reinterpret_cast<char*>(ws);
+  const size_t off_ml = align_up(kHeaderBytes + size_t(U) * sizeof(int), 256);
+  const size_t off_o = off_ml + align_up(size_t(pl.n_items) * 64 * 2 * sizeof(float), 256);
+  dtc::sdec::Params p{};
   p.idx = idx;
   p.cnt = sel->topk > 0 ? cnt : nullptr;
   p.cu_kv = vl->cu_kv;
+  p.k8 = reinterpret_cast<const uint8_t*>(k);
+  p.v8 = reinterpret_cast<const uint8_t*>(v);
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
   p.topk = sel->topk;
   p.w = sel->window;
+  p.G = sh.G;
   p.Hq = sh.Hq;
   p.Hkv = sh.Hkv;
-  p.G = sh.G;
-  p.n_chunks = nc;
+  p.Tq = int(sh.Tq);
+  p.n_units = U;
+  p.nsplit = pl.nsplit;
+  p.tiles_per_split = pl.tiles_per_split;
+  p.unit_tiles = pl.unit_tiles;
+  p.n_items = pl.n_items;
   p.scale_log2 = sh.scale * 1.4426950408889634f;
-  char* w = reinterpret_cast<char*>(ws);
-  p.part_o = reinterpret_cast<float*>(w + kHeaderBytes);
-  p.part_ml = reinterpret_cast<float*>(w + align_up(kHeaderBytes + size_t(bg) * nc * dec::kHeads * 128 * 4, 256));
-  static PerDeviceOnce once1, once2;
-  if (set_smem_once(once1, dec::sparse_decode_kernel<false>, dec::sparse_smem_bytes<false>()) != cudaSuccess ||
-      set_smem_once(once2, dec::sparse_decode_kernel<true>, dec::sparse_smem_bytes<true>()) != cudaSuccess)
+  p.done = reinterpret_cast<int*>(w + kHeaderBytes);
+  p.part_ml = reinterpret_cast<float*>(w + off_ml);
+  p.part_o = reinterpret_cast<float*>(w + off_o);
+  p.o = reinterpret_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.wc = wait_ctl(ws);
+  if (cudaMemsetAsync(p.done, 0, size_t(U) * sizeof(int), s) != cudaSuccess) return HS_ERR_CUDA;
+  Maps m;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 1)) return HS_ERR_CUDA;
+  m.k = m.v = m.q;
+  if (!fp8 && (!make_map_rows(&m.k, k, sh.d, sh.Tkv * sh.Hkv) || !make_map_rows(&m.v, v, sh.d, sh.Tkv * sh.Hkv)))
     return HS_ERR_CUDA;
-  const dim3 grid(nc, bg);
-  if (fp8)
-    dec::sparse_decode_kernel<true><<<grid, dec::kThreads, dec::sparse_smem_bytes<true>(), s>>>(p);
-  else
-    dec::sparse_decode_kernel<false><<<grid, dec::kThreads, dec::sparse_smem_bytes<false>(), s>>>(p);
-  dec::CombineParams cp{};
-  cp.part_o = p.part_o;
-  cp.part_ml = p.part_ml;
-  cp.n_chunks = nc;
-  cp.Hq = sh.Hq;
-  cp.Hkv = sh.Hkv;
-  cp.G = sh.G;
-  cp.Tq = int(sh.Tq);
-  cp.normalised = false;
-  cp.o = reinterpret_cast<__nv_bfloat16*>(o);
-  cp.lse = lse;
-  dec::combine_kernel<<<dim3(bg, (sh.G + dec::kCombineHeads - 1) / dec::kCombineHeads), 32 * dec::kCombineHeads, 0, s>>>(cp);
+  const int grid = std::min(num_sms(), pl.n_items);
+  constexpr int smem = dtc::sdec::smem_bytes();
+  if (fp8) {
+    static PerDeviceOnce once;
+    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<true>, smem) != cudaSuccess) return HS_ERR_CUDA;
+    dtc::sdec::sparse_decode_tc_kernel<true><<<grid, dtc::sdec::threads<true>(), smem, s>>>(m.q, m.k, m.v, p);
+  } else {
+    static PerDeviceOnce once;
+    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<false>, smem) != cudaSuccess) return HS_ERR_CUDA;
+    dtc::sdec::sparse_decode_tc_kernel<false><<<grid, dtc::sdec::threads<false>(), smem, s>>>(m.q, m.k, m.v, p);
+  }
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 

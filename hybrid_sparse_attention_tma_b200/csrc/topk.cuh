@@ -3,8 +3,10 @@
 // TopK over the full layer's block scores (HySparse explainer, techwalker.com)
 // or token scores with k = 1024 (HySparse2 release note; demingchina
 // commentary section 03). Candidates of a tile are the blocks b with
-// b*B <= last query position of the tile. Rule: score descending, ties to the
-// lower index; the kept set is written in ascending index order, padded -1.
+// b*B <= last query position of the tile, or (window-exclusive reading) only
+// those starting before the last query's forced window, b*B <= last - w.
+// Rule: score descending, ties to the lower index; the kept set is written in
+// ascending index order, padded -1.
 //
 // Method: scores are >= 0, so their fp32 bit patterns order like the values.
 // A 4-pass MSB-first radix select (8 bits per pass, per-warp histograms in
@@ -33,6 +35,7 @@ struct Params {
   int* idx;             // [n_tiles, Hkv, k]
   int* cnt;             // [n_tiles, Hkv]
   int Hkv, nblk, B, k;
+  int w, exclusive;  // forced window; 1 = candidates stop before the last query's window
 };
 
 // Block-wide exclusive scan of one int per thread; returns the total.
@@ -78,7 +81,8 @@ __global__ void __launch_bounds__(THREADS)
   const int tile = row / p.Hkv;
   const TileInfo ti = tile_info(st, tile);
   const int last_pos = ti.pos0 + ti.n - 1;
-  const int n = min(p.nblk, last_pos / p.B + 1);
+  const int lim = p.exclusive ? last_pos - p.w : last_pos;  // candidates: b * B <= lim
+  const int n = lim < 0 ? 0 : min(p.nblk, lim / p.B + 1);
   const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
   int* out = p.idx + size_t(row) * p.k;
   const int k = p.k;

@@ -86,7 +86,22 @@ typedef struct {
   int32_t block;   /* B: keys per selectable block; 1 = token-level selection */
   int32_t topk;    /* k: blocks kept per (tile, KV head); 0 <= k <= 4096 */
   int32_t window;  /* w: forced recent window (tokens) unioned into the sparse set */
+  int32_t flags;   /* 0, or HS_SEL_WINDOW_EXCLUSIVE (zero-initialise the struct) */
 } hs_sel;
+
+/* hs_sel.flags: which blocks compete for the top-k (used by hs_topk_select).
+ * 0 (union reading): every causal block, b * B <= last query position of the
+ *   tile; the forced window is then added per query and may overlap the kept
+ *   blocks (HySparse2 release note on airebao.com: the latest tokens are
+ *   forced into the selected set).
+ * HS_SEL_WINDOW_EXCLUSIVE: only blocks that start before the forced window of
+ *   the tile's last query, b * B <= last_pos - w, so the k kept blocks are
+ *   "global" and the w recent tokens come on top (demingchina
+ *   commentary on HySparse2, section 03: 1024 global tokens plus the latest
+ *   128). Identical to the union reading when w = 0. The sparse-attention
+ *   calls need no flag: their visible set is the same rule for both readings.
+ * Other bits are HS_ERR_INVALID_ARG. */
+#define HS_SEL_WINDOW_EXCLUSIVE 1
 
 typedef enum { HS_KV_BF16 = 0, HS_KV_FP8_E4M3 = 1 } hs_kv_dtype;
 
@@ -152,8 +167,10 @@ HS_API hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel,
  * token-level selection of 1024 tokens. Candidates of tile t are blocks
  * b <= floor(last_pos(t) / B). Order: score descending, ties to the lower
  * index. Output idx ascending, padded with -1; cnt = min(k, #candidates).
- * The forced recent window is not applied here: the sparse attention calls
- * union it per query.
+ * With sel->flags = HS_SEL_WINDOW_EXCLUSIVE the candidates stop before the
+ * forced window of the tile's last query: b * B <= last_pos(t) - w.
+ * The forced recent window itself is not applied here: the sparse attention
+ * calls union it per query.
  * In: scores [n_tiles,H_kv,n_blk] fp32 (>= 0). Out: idx [n_tiles,H_kv,k], cnt.
  */
 HS_API hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* scores,
@@ -188,11 +205,12 @@ HS_API hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel,
  * FP8 e4m3 (the HySparse2 key-data table sizes an FP8 KV cache); FP8 values
  * decode as x = scale[token, kv_head] * e4m3(code), with separate fp32 scale
  * arrays for K and V ([T_kv, H_kv]; NULL for bf16).
- * The visible set of each (sequence, KV head) is cut into 128-key chunks, one
- * CTA each, and the chunks' partials are merged by log-sum-exp.
- * split_k: 0 = one chunk per 128 keys of k + w (automatic); a positive value
- * below that count is HS_ERR_UNSUPPORTED, a larger one is accepted and the
- * automatic count is used. Negative values are rejected.
+ * The slots of each (sequence, KV head) -- the window, then the selected
+ * tokens -- form ceil((k + w) / 128) tiles of 128 keys, cut into split_k
+ * contiguous ranges of whole tiles, one tensor-core work item each; the
+ * ranges' partial results are merged by log-sum-exp inside the same launch.
+ * split_k: 0 = automatic (about one range per SM over all units); a value
+ * above the tile count is clamped to it; negative values are rejected.
  * An empty batch (T_q = 0) returns HS_OK without touching any pointer.
  * Requires n_b = 1 for every sequence and sel->q_tile = 1.
  */

@@ -26,13 +26,14 @@ def tile_rows(cu_q, cu_kv, T, tile_ids):
 
 def run_block(q, k, v, layers, cu_q, cu_kv, n_kv_heads, T, B, topk, w, swa_window=0,
               tile_ids: Optional[Sequence[int]] = None, idx_override=None, cnt_override=None,
-              compact: bool = False):
+              compact: bool = False, exclusive: bool = False):
     """layers: list of dicts with 'q' and optionally 'k_swa', 'v_swa', 'gamma'.
 
     Returns a dict with o_full, lse_full, scores, idx, cnt and per-layer outputs.
     When idx_override/cnt_override are given, the sparse layers use those
     indices (used to check outputs independently of legitimate tie-band
-    differences in the selection). With ``compact`` (and tile_ids) every
+    differences in the selection). ``exclusive`` selects the window-exclusive
+    reading of the top-k candidates. With ``compact`` (and tile_ids) every
     output holds only the sampled tiles' rows, tile after tile, instead of
     full-size arrays with the other rows left NaN / 0.
     """
@@ -41,7 +42,8 @@ def run_block(q, k, v, layers, cu_q, cu_kv, n_kv_heads, T, B, topk, w, swa_windo
                                         tile_ids=tile_ids, compact=compact)
     scores = O.importance_scores(q, k, lse_full, cu_q, cu_kv, n_kv_heads, T, B,
                                  tile_ids=tile_ids, compact=compact)
-    idx, cnt = O.topk_select(scores, cu_q, cu_kv, T, B, topk, tile_ids=tile_ids, compact=compact)
+    idx, cnt = O.topk_select(scores, cu_q, cu_kv, T, B, topk, tile_ids=tile_ids, compact=compact, w=w,
+                             exclusive=exclusive)
     use_idx = idx if idx_override is None else idx_override
     use_cnt = cnt if cnt_override is None else cnt_override
     outs = []

@@ -252,18 +252,35 @@ def importance_scores(q, k, lse, cu_q, cu_kv, n_kv_heads: int, T: int, B: int, s
 # A3  top-k selection
 # ----------------------------------------------------------------------------
 
-def n_candidates(t: Tile, B: int) -> int:
-    """Causal candidates of a tile: blocks b with b*B <= last query position."""
-    return t.last_pos // B + 1
+def n_candidates(t: Tile, B: int, w: int = 0, exclusive: bool = False) -> int:
+    """Candidate blocks of a tile.
+
+    Union reading (default): every causal block, b*B <= last query position;
+    the forced window is added per query afterwards, so a selected block may
+    overlap it [airebao-HySparse2: the latest tokens are forced into the
+    selected set].
+    Exclusive reading: only blocks that start before the forced window of the
+    tile's last query, b*B <= last_pos - w, compete, so the k selected blocks
+    are "global" tokens and the w recent ones come on top
+    [demingchina-HySparse2 s.03: 1024 global tokens plus the latest 128].
+    With w = 0 the two readings coincide.
+    """
+    if not exclusive:
+        return t.last_pos // B + 1
+    lim = t.last_pos - w
+    return 0 if lim < 0 else lim // B + 1
 
 
 def topk_select(scores, cu_q, cu_kv, T: int, B: int, k: int,
-                tile_ids: Optional[Sequence[int]] = None, compact: bool = False):
+                tile_ids: Optional[Sequence[int]] = None, compact: bool = False,
+                w: int = 0, exclusive: bool = False):
     """Keep the k highest-scoring candidate blocks of each (tile, KV head).
 
-    Order: score descending, ties to the lower block index (the reading used
-    throughout; the pages only say "TopK"). The kept set is emitted in ascending index
-    order and padded with -1; cnt = min(k, #candidates).
+    Candidates per n_candidates (union or exclusive reading of the forced
+    window). Order: score descending, ties to the lower block index (the
+    reading used throughout; the pages only say "TopK"). The kept set is
+    emitted in ascending index order and padded with -1;
+    cnt = min(k, #candidates).
     Returns (idx int32 [n_tiles, H_kv, k], cnt int32 [n_tiles, H_kv]).
     """
     n_rows, Hkv, _ = scores.shape
@@ -273,7 +290,7 @@ def topk_select(scores, cu_q, cu_kv, T: int, B: int, k: int,
     sel = tiles if tile_ids is None else [tiles[i] for i in tile_ids]
     for si, t in enumerate(sel):
         r = si if compact else t.index   # compact: scores/idx rows follow tile_ids
-        nc = n_candidates(t, B)
+        nc = n_candidates(t, B, w, exclusive)
         ids = np.arange(nc)
         for g in range(Hkv):
             s = scores[r, g, :nc]

@@ -101,9 +101,9 @@ class GpuBlock:
         self.w = w
         self.inp = inp
         self.vl = hs.Varlen(w.cu_q(), w.cu_kv(), w.n_q_heads, w.n_kv_heads, w.head_dim, device=device)
-        self.sel = hs.Sel(w.q_tile, w.block, w.topk, w.window)
+        self.sel = hs.Sel(w.q_tile, w.block, w.topk, w.window, w.exclusive)
         self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device,
-                                 fused=fused)
+                                 fused=fused, exclusive=w.exclusive)
         self.layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
 
     def run(self, stream=None, fp8=False, intermediates=True):

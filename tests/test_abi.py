@@ -94,6 +94,9 @@ def test_host_validation_errors(lib):
     assert fused(128, 16, 24) == L.HS_ERR_INVALID_ARG
     assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG
+    # unknown selection flags are rejected
+    bad = L.HsSel(16, 16, 8, 32, 2)
+    assert _call_full(lib, vl, bad) == L.HS_ERR_INVALID_ARG
     # exp2 self test: empty is a no-op, null / misaligned / negative sizes are rejected before launch
     assert lib.hs_debug_exp2_poly(None, None, 0, None) == L.HS_OK
     assert lib.hs_debug_exp2_poly(None, None, 4, None) == L.HS_ERR_INVALID_ARG

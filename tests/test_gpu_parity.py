@@ -59,10 +59,12 @@ def check_block(w, inp, res, tile_ids=None, fp8=False):
     # A3: top-k -- exact on the GPU's own scores, tie band against the oracle's
     idx_g = res["idx"][tids_t].cpu().numpy()[:, :, :w.topk]
     cnt_g = res["cnt"][tids_t].cpu().numpy()
-    idx_x, cnt_x = O.topk_select(sc_g, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True)
+    idx_x, cnt_x = O.topk_select(sc_g, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True, w=w.window,
+                                 exclusive=w.exclusive)
     assert (cnt_g == cnt_x).all(), "cnt of GPU scores differs"
     assert (idx_g == idx_x).all(), "top-k of GPU scores differs"
-    idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True)
+    idx_o, cnt_o = O.topk_select(sc_o, cu_q, cu_kv, T, B, w.topk, tile_ids=tids, compact=True, w=w.window,
+                                 exclusive=w.exclusive)
     assert_indices_match(idx_g, cnt_g, sc_o, idx_o, cnt_o, range(len(tids)), max(w.topk, 1))
     # A4 / A5 / A6: sparse layers, fed the GPU's (checked) indices
     kd, vd = (_Dequant(inp.k_fp8, inp.k_scale), _Dequant(inp.v_fp8, inp.v_scale)) if fp8 else (k, v)
@@ -139,6 +141,12 @@ VARIANTS = {
     # a sequence with no new tokens inside the batch, fused layer with 16-token blocks
     "empty_seq": W.Workload("v10", ctx=(0, 90, 40), new=(150, 0, 70), n_q_heads=4, n_kv_heads=1, head_dim=64,
                             q_tile=16, block=16, topk=4, window=8, n_sparse=1, swa_window=32),
+    # window-exclusive top-k (k global tokens + the latest w), token level, chunked + ragged
+    "tok_exclusive": W.Workload("v12", ctx=(0, 500), new=(300, 150), n_q_heads=32, n_kv_heads=1, head_dim=128,
+                                q_tile=16, block=1, topk=96, window=32, n_sparse=1, needle_rate=0.02, exclusive=True),
+    # window-exclusive top-k at block level, GQA
+    "blk_exclusive": W.Workload("v13", ctx=(64, 0), new=(260, 200), n_q_heads=8, n_kv_heads=2, head_dim=64,
+                                q_tile=32, block=16, topk=4, window=24, n_sparse=1, exclusive=True),
     # token-level selection with the window branch and gate fused in (one launch per layer)
     "swa_tok": W.Workload("v11", ctx=(0, 300), new=(260, 90), n_q_heads=16, n_kv_heads=1, head_dim=128,
                           q_tile=16, block=1, topk=64, window=8, n_sparse=1, swa_window=32, needle_rate=0.02),
@@ -201,6 +209,14 @@ def test_hys2_token_full_size_sampled_tiles():
     run_and_check(w, tile_ids=tiles)
 
 
+def test_hys2_token_full_size_exclusive_sampled_tiles():
+    """HySparse2 token-level prefill at full size with the window-exclusive
+    reading (top-1024 global tokens + the latest 128), sampled tiles."""
+    w = W.WORKLOADS["hys2_prefill"].with_(exclusive=True, n_sparse=2)
+    n_t = w.n_tiles()
+    run_and_check(w, tile_ids=[0, n_t // 3, n_t - 1])
+
+
 def test_agentic_chunked_full_size_sampled_tiles():
     """Agentic ragged chunked prefill at full size (contexts 262144/131072/65536/
     16384 + chunks 8192/4096/8192/2048, 64/1 heads, top-1024 + forced 128),
@@ -221,6 +237,9 @@ DECODE = {
     # GQA group 8 (only 8 of the 64 MMA rows valid), several KV heads
     "dec_gqa8": W.Workload("d2", ctx=(700, 90), new=(1, 1), n_q_heads=32, n_kv_heads=4, head_dim=128,
                            q_tile=1, block=1, topk=40, window=16, n_sparse=1),
+    # window-exclusive decode: 1024-style global tokens plus the latest w, disjoint
+    "dec_exclusive": W.Workload("d4", ctx=(900, 130, 2000), new=(1, 1, 1), n_q_heads=64, n_kv_heads=1,
+                                head_dim=128, q_tile=1, block=1, topk=80, window=48, n_sparse=1, exclusive=True),
     # k = 0: the sparse layer sees only the forced window (one context shorter than the window)
     "dec_window_only": W.Workload("d3", ctx=(200, 45), new=(1, 1), n_q_heads=64, n_kv_heads=1, head_dim=128,
                                   q_tile=1, block=1, topk=0, window=48, n_sparse=1),
@@ -232,6 +251,37 @@ DECODE = {
 def test_decode_whole(name, fp8):
     w = DECODE[name].with_(fp8_kv=True)
     run_and_check(w, seed=5, fp8=fp8)
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_decode_split_counts_agree_with_the_oracle(fp8):
+    """Every way of cutting a unit's slots into key ranges (one range, the
+    automatic count, one tile per range, more ranges than tiles) gives the
+    oracle's sparse-layer output; the ranges are merged by log-sum-exp."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    w = W.Workload("dsplit", ctx=(1500, 700, 300), new=(1, 1, 1), n_q_heads=64, n_kv_heads=1, head_dim=128,
+                   q_tile=1, block=1, topk=500, window=40, n_sparse=1, fp8_kv=True)
+    inp = W.make_block_inputs(w, device="cuda", seed=17)
+    blk = GpuBlock(w, inp)
+    res = blk.run(fp8=fp8)
+    torch.cuda.synchronize()
+    idx, cnt = res["idx"], res["cnt"]
+    L0 = inp.layers[0]
+    kd, vd = (_Dequant(inp.k_fp8, inp.k_scale), _Dequant(inp.v_fp8, inp.v_scale)) if fp8 else (LazyF64(inp.k),
+                                                                                                   LazyF64(inp.v))
+    cu_q, cu_kv = w.cu_q(), w.cu_kv()
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    o_ref, lse_ref = O.sparse_attention(LazyF64(L0.q), kd, vd, idx_h, cnt_h, cu_q, cu_kv, 1, 1, w.window)
+    tiles = (w.topk + w.window + 127) // 128
+    for split in [1, 2, tiles, tiles + 5]:
+        if fp8:
+            o, lse = hs.sparse_attn_decode(blk.vl, blk.sel, L0.q, inp.k_fp8, inp.v_fp8, idx, cnt, inp.k_scale,
+                                           inp.v_scale, hs.HS_KV_FP8_E4M3, split_k=split)
+        else:
+            o, lse = hs.sparse_attn_decode(blk.vl, blk.sel, L0.q, inp.k, inp.v, idx, cnt, split_k=split)
+        torch.cuda.synchronize()
+        assert_close_out(f64(o), o_ref, what=f"split {split} o")
+        assert_close_lse(f64(lse), lse_ref, what=f"split {split} lse")
 
 
 @pytest.mark.parametrize("fp8", [False, True])

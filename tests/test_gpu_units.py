@@ -40,29 +40,34 @@ TOPK_CASES = {
     "streamed_decode_b64": ((131072,) * 64, (1,) * 64, 1, 1, 1, 1024, [0.1, 0.2, 0.4, 0.8]),
     # token level, one long sequence, tiles of 64, streamed
     "streamed_token_b1": ((131008,), (128,), 1, 64, 1, 1024, [0.5, 0.75, 1.0]),
+    # window-exclusive candidates (start before the last query's window of 128), staged and streamed
+    "excl_token_staged": ((4000, 100), (64, 64), 1, 64, 1, 1024, [0.25, 0.5, 1.0], 128),
+    "excl_decode_streamed": ((131072,) * 8, (1,) * 8, 1, 1, 1, 1024, [0.1, 0.2, 0.4, 0.8], 128),
+    "excl_block": ((0,), (4096,), 2, 64, 64, 8, [0.25, 0.5], 100),
 }
 
 
 @pytest.mark.parametrize("name", list(TOPK_CASES))
 def test_topk_exact_ties_bit_exact(name):
     import hybrid_sparse_attention_tma_b200 as hs
-    ctx, new, Hkv, T, B, k, levels = TOPK_CASES[name]
+    ctx, new, Hkv, T, B, k, levels = TOPK_CASES[name][:7]
+    win = TOPK_CASES[name][7] if len(TOPK_CASES[name]) > 7 else 0  # window-exclusive cases
     kv = [c + n for c, n in zip(ctx, new)]
     cu_q = [0] + np.cumsum(new).tolist()
     cu_kv = [0] + np.cumsum(kv).tolist()
     vl = hs.Varlen(cu_q, cu_kv, Hkv, Hkv, 128, device="cuda")
-    sel = hs.Sel(T, B, k, 0)
+    sel = hs.Sel(T, B, k, win, exclusive=win > 0)
     nblk = (max(kv) + B - 1) // B
     scores = _level_scores((vl.n_tiles(T), Hkv, nblk), levels, seed=len(name))
     idx, cnt = hs.topk_select(vl, sel, scores)
     torch.cuda.synchronize()
     sc = scores.cpu().double().numpy()
-    idx_o, cnt_o = O.topk_select(sc, cu_q, cu_kv, T, B, k)
+    idx_o, cnt_o = O.topk_select(sc, cu_q, cu_kv, T, B, k, w=win, exclusive=win > 0)
     assert np.array_equal(cnt.cpu().numpy(), cnt_o)
     assert np.array_equal(idx.cpu().numpy(), idx_o)
     # the case really exercises ties at the k-th place
     t0 = O.make_tiles(cu_q, cu_kv, T)[0]
-    nc = O.n_candidates(t0, B)
+    nc = O.n_candidates(t0, B, win, win > 0)
     if nc > k:
         row = np.sort(sc[0, 0, :nc])[::-1]
         assert row[k - 1] == row[k], "no tie straddles the k-th place"

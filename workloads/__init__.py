@@ -58,6 +58,7 @@ class Workload:
     needle_rate: float = 0.0
     fp8_kv: bool = False  # decode only: KV cache given as e4m3 codes + scales
     config_index: int = 0
+    exclusive: bool = False  # top-k drawn only from blocks before the last query's forced window
 
     @property
     def batch(self) -> int:
