@@ -63,7 +63,8 @@ def parse():
                     help="measure only --workload (skip the other configurations' short runs)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--fp8-kv", action="store_true", help="decode: sparse layers read an FP8-e4m3 KV cache")
+    ap.add_argument("--fp8-kv", action="store_true",
+                    help="FP8-e4m3 KV cache: decode sparse layers read it directly; prefill expands it once per block")
     ap.add_argument("--exclusive", action="store_true",
                     help="window-exclusive top-k: k global tokens drawn before the last query's forced window")
     ap.add_argument("--tokens", type=int, default=0,
@@ -539,7 +540,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                       "l2": "step: inputs larger than L2; per-kernel times: L2 flushed before every call", "parallelism": (f"one block over {world} GPUs: {shard_kind(w_block, world)}" if world > 1
                                       else "one block, one GPU")},
            "roofline": dom, "kernels": kernels,
-           "gpu_launches": blk.launches_per_forward(len(layers)) * steps,
+           "gpu_launches": blk.launches_per_forward(len(layers), fp8_prefill=bool(fp8) and not blk.decode) * steps,
            "needle_recall": recall, "clocks": clk, "e2e": e2e}
     del step_graph, flush_graph, kind_graphs, flush, inp, blk, layers, kv_own
     torch.cuda.empty_cache()

@@ -17,8 +17,8 @@ from . import _lib as L
 from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
 
 __all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
-           "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "workspace_size", "check_error",
-           "HsError"]
+           "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "kv_dequantize", "workspace_size",
+           "check_error", "HsError"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -193,6 +193,15 @@ def sparse_attn_decode(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, k_scale=None
         _ptr(v_scale), _ptr(idx), _ptr(cnt), split_k, _ptr(o), _ptr(lse), _ptr(buf), buf.numel(),
         _stream(stream)))
     return o, lse
+
+
+def kv_dequantize(codes, scale, out=None, stream=None):
+    """FP8-e4m3 KV codes [T, H, d] uint8 with scales [T, H] fp32 -> bf16 [T, H, d]."""
+    lib = L.load()
+    T, H, d = codes.shape
+    out = torch.empty((T, H, d), dtype=torch.bfloat16, device=codes.device) if out is None else out
+    L.check("hs_kv_dequantize", lib.hs_kv_dequantize(_ptr(codes), _ptr(scale), T * H, d, _ptr(out), _stream(stream)))
+    return out
 
 
 def swa_gated(vl: Varlen, window: int, q, k_swa, v_swa, gamma, o_sparse, o=None,

@@ -17,7 +17,7 @@ EXPORTS = [
     "hs_workspace_size", "hs_workspace_init", "hs_check_error", "hs_status_string",
     "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
     "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
-    "hs_full_attn_select_noalloc", "hs_sparse_swa_gated_prefill", "hs_debug_exp2_poly",
+    "hs_full_attn_select_noalloc", "hs_sparse_swa_gated_prefill", "hs_debug_exp2_poly", "hs_kv_dequantize",
 ]
 
 
@@ -86,6 +86,8 @@ def load():
     lib.hs_debug_wait_timeout.argtypes = [vp, sz, ctypes.c_uint64, vp]
     lib.hs_debug_exp2_poly.restype = i32
     lib.hs_debug_exp2_poly.argtypes = [vp, vp, ctypes.c_int64, vp]
+    lib.hs_kv_dequantize.restype = i32
+    lib.hs_kv_dequantize.argtypes = [vp, vp, ctypes.c_int64, i32, vp, vp]
     _lib = lib
     return lib
 

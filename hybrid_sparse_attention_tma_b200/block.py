@@ -13,7 +13,7 @@ from typing import List, Optional
 import torch
 
 from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
-               swa_gated, sparse_swa_gated_prefill, HS_KV_BF16, HS_KV_FP8_E4M3)
+               swa_gated, sparse_swa_gated_prefill, kv_dequantize, HS_KV_BF16, HS_KV_FP8_E4M3)
 
 
 @dataclass
@@ -55,7 +55,10 @@ class HybridBlock:
         With keep_all=False, output buffers are reused across calls (no
         allocation in steady state) and only the last layer's tensors are
         guaranteed distinct. fp8_kv = (k_codes, v_codes, k_scale, v_scale) makes the
-        sparse decode layers read an FP8-e4m3 copy of the KV cache. With
+        sparse decode layers read an FP8-e4m3 copy of the KV cache; in prefill
+        the block reads that FP8 cache everywhere: it is expanded to bf16 once
+        (hs_kv_dequantize) and the full and sparse layers use the expansion
+        (k and v may then be None). With
         intermediates=False a fused layer does not write o_sparse / lse_sparse
         (they are returned as None)."""
         vl, sel = self.vl, self.sel
@@ -67,6 +70,10 @@ class HybridBlock:
         scores = self._buf("scores", (nt, vl.n_kv_heads, nblk), torch.float32)
         idx = self._buf("idx", (nt, vl.n_kv_heads, max(sel.topk, 1)), torch.int32)
         cnt = self._buf("cnt", (nt, vl.n_kv_heads), torch.int32)
+        if fp8_kv is not None and not self.decode:
+            kq, vq, ks, vs = fp8_kv
+            k = kv_dequantize(kq, ks, self._buf("k_deq", tuple(kq.shape), torch.bfloat16), stream=stream)
+            v = kv_dequantize(vq, vs, self._buf("v_deq", tuple(vq.shape), torch.bfloat16), stream=stream)
         full_attn_select(vl, sel, q, k, v, o, lse, scores, ws=self.ws, stream=stream)
         topk_select(vl, sel, scores, idx, cnt, ws=self.ws, stream=stream)
         outs = []
@@ -101,17 +108,17 @@ class HybridBlock:
             outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
         return {"o_full": o, "lse_full": lse, "scores": scores, "idx": idx, "cnt": cnt, "layers": outs}
 
-    def launches_per_forward(self, n_layers: int) -> int:
+    def launches_per_forward(self, n_layers: int, fp8_prefill: bool = False) -> int:
         """Kernels of this library launched by one forward (memsets excluded):
         full layer 1 (block scores) / 3 (token scores: forward, item prefix,
-        score pass) / 4 (decode: two passes and two combines); top-k 1; each
-        sparse layer 1 (prefill, with its window branch and gate when fused)
-        or 2 (decode: partials + combine), plus 1 for an unfused gated SWA
-        branch."""
+        score pass) / 1 (decode: both passes in one launch); top-k 1; each
+        sparse layer 1 (prefill, with its window branch and gate when fused;
+        decode, with its key ranges merged in the same launch), plus 1 for an
+        unfused gated SWA branch; an FP8 prefill adds the two expansions."""
         if self.decode:
-            full = 4
+            full = 1
         else:
             full = 1 if self.sel.block > 1 else 3
-        sparse = 2 if self.decode else 1
+        sparse = 1
         swa = 1 if (self.swa_window > 0 and not (self.fused and not self.decode)) else 0
-        return full + 1 + n_layers * (sparse + swa)
+        return full + 1 + n_layers * (sparse + swa) + (2 if fp8_prefill else 0)

@@ -396,6 +396,32 @@ __global__ void debug_wait_kernel(WaitCtl wc) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, wc, 99);
 }
 
+// FP8-e4m3 KV rows -> bf16: thread = 16 codes of one row (one 16-byte load,
+// two 16-byte stores); exact e4m3 -> f16 conversion, fp32 product with the
+// row's scale, bf16 round-to-nearest-even. HBM-bound: 3 bytes per element.
+__global__ void __launch_bounds__(256) kv_dequant_kernel(const uint4* __restrict__ codes, const float* __restrict__ scale,
+                                                         uint4* __restrict__ out, long long rows, int chunks_per_row) {
+  const long long n = rows * chunks_per_row;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += (long long)gridDim.x * blockDim.x) {
+    const float sc = __ldg(scale + i / chunks_per_row);
+    const uint4 c = __ldg(codes + i);
+    const uint32_t w4[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o8[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+        uint32_t h2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(uint16_t(hlf ? (w4[e] >> 16) : (w4[e] & 0xFFFFu))));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+        o8[2 * e + hlf] = pack_bf16(f.x * sc, f.y * sc);
+      }
+    }
+    out[2 * i] = make_uint4(o8[0], o8[1], o8[2], o8[3]);
+    out[2 * i + 1] = make_uint4(o8[4], o8[5], o8[6], o8[7]);
+  }
+}
+
 // 2^x on the FMA pipe, as the softmax uses it, over an array (self test).
 __global__ void debug_exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
   const long long stride = 2LL * gridDim.x * blockDim.x;
@@ -983,6 +1009,20 @@ hs_status hs_debug_wait_timeout(void* ws, size_t ws_bytes, uint64_t timeout_ns, 
   if (timeout_ns == 0 || timeout_ns > 2000000000ull) return HS_ERR_INVALID_ARG;
   WaitCtl wc{reinterpret_cast<ErrWord*>(ws), timeout_ns};
   debug_wait_kernel<<<1, 32, 0, S(stream)>>>(wc);
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_kv_dequantize(const void* codes, const float* scale, int64_t rows, int32_t head_dim, void* out,
+                           hs_stream_t stream) {
+  if (rows < 0 || head_dim <= 0 || head_dim % 16) return HS_ERR_INVALID_ARG;
+  if (rows == 0) return HS_OK;
+  if (!codes || !scale || !out || !aligned16(codes) || !aligned16(out) || (reinterpret_cast<uintptr_t>(scale) & 3))
+    return HS_ERR_INVALID_ARG;
+  const int cpr = head_dim / 16;
+  const long long n = rows * cpr;
+  const int grid = int(std::min<long long>(8LL * num_sms(), (n + 255) / 256));
+  kv_dequant_kernel<<<grid, 256, 0, S(stream)>>>(reinterpret_cast<const uint4*>(codes), scale,
+                                                 reinterpret_cast<uint4*>(out), rows, cpr);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 

@@ -264,6 +264,26 @@ HS_API hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* 
                                       void* ws, size_t ws_bytes, hs_stream_t stream);
 
 /*
+ * hs_kv_dequantize -- expand an FP8-e4m3 KV cache to bf16 for the prefill
+ * calls of a block (the HySparse2 key-data table on airebao.com sizes an FP8
+ * KV cache; the block's full layer and its sparse layers all read that one
+ * cache, KV Reuse).
+ *   out[r][i] = bf16_rn(scale[r] * e4m3(codes[r][i])),  r < rows, i < head_dim
+ * with one fp32 scale per (token, KV head) row (rows = T_kv * H_kv; the
+ * product is formed in fp32). Prefill attention is bound by the tensor cores,
+ * so one pass over the cache (1 + 2 bytes per element) per block, shared by
+ * the full layer and every sparse layer, stands in for expanding the codes
+ * inside each attention kernel; decode reads the codes directly
+ * (hs_sparse_attn_decode with HS_KV_FP8_E4M3).
+ * In: codes [rows, head_dim] uint8, scale [rows] fp32. Out: out [rows, head_dim]
+ * bf16 (device, caller-owned, must not overlap the inputs). head_dim a
+ * multiple of 16; pointers 16-byte aligned (scale 4-byte). rows = 0 is a
+ * no-op; negative sizes, null or misaligned pointers are HS_ERR_INVALID_ARG.
+ */
+HS_API hs_status hs_kv_dequantize(const void* codes, const float* scale, int64_t rows, int32_t head_dim,
+                                  void* out, hs_stream_t stream);
+
+/*
  * hs_full_attn_select_noalloc -- hs_full_attn_select for callers that cannot
  * allocate device memory. The pages have no counterpart to this entry point.
  *

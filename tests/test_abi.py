@@ -94,6 +94,12 @@ def test_host_validation_errors(lib):
     assert fused(128, 16, 24) == L.HS_ERR_INVALID_ARG
     assert lib.hs_debug_wait_timeout(None, 0, 1000, None) == L.HS_ERR_WORKSPACE
     assert lib.hs_debug_wait_timeout(16, 1 << 20, 0, None) == L.HS_ERR_INVALID_ARG
+    # FP8 expansion: empty is a no-op; bad sizes / pointers are rejected before launch
+    assert lib.hs_kv_dequantize(None, None, 0, 128, None, None) == L.HS_OK
+    assert lib.hs_kv_dequantize(16, 16, 4, 120, 16, None) == L.HS_ERR_INVALID_ARG  # head_dim % 16
+    assert lib.hs_kv_dequantize(None, 16, 4, 128, 16, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_kv_dequantize(16, 18, 4, 128, 16, None) == L.HS_ERR_INVALID_ARG  # misaligned scale
+    assert lib.hs_kv_dequantize(16, 16, -1, 128, 16, None) == L.HS_ERR_INVALID_ARG
     # unknown selection flags are rejected
     bad = L.HsSel(16, 16, 8, 32, 2)
     assert _call_full(lib, vl, bad) == L.HS_ERR_INVALID_ARG

@@ -73,6 +73,27 @@ def test_topk_exact_ties_bit_exact(name):
         assert row[k - 1] == row[k], "no tie straddles the k-th place"
 
 
+def test_kv_dequantize_bit_exact():
+    """hs_kv_dequantize: bf16_rn(fp32(scale) * fp32(e4m3(code))) for every row,
+    bit for bit against the same arithmetic by torch on the host (every code
+    value appears, including subnormals and +-448)."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    import workloads as W
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4)
+    x = torch.randn((3001, 2, 128), generator=g, device="cuda") * 3.0
+    codes, scale = W.quantize_e4m3_per_token(x)
+    codes = codes.clone()
+    codes[0, 0] = torch.arange(128, dtype=torch.uint8, device="cuda")          # codes 0..127
+    codes[0, 1] = torch.arange(128, 256, dtype=torch.uint8, device="cuda")     # codes 128..255
+    codes[0, 1, 127] = 0x7E  # keep NaN codes (0x7F, 0xFF) out of the comparison
+    codes[0, 0, 127] = 0x7E
+    out = hs.kv_dequantize(codes, scale)
+    torch.cuda.synchronize()
+    ref = (codes.cpu().view(torch.float8_e4m3fn).float() * scale.cpu().unsqueeze(-1)).to(torch.bfloat16)
+    assert torch.equal(out.cpu().view(torch.int16), ref.view(torch.int16))
+
+
 def _exp2_poly(x: np.ndarray) -> np.ndarray:
     import hybrid_sparse_attention_tma_b200._lib as L
     lib = L.load()
