@@ -339,7 +339,8 @@ size_t full_decode_ws_bytes(const hs_varlen* vl, const Shape& sh) { return full_
 
 // Sparse decode on the tensor cores (decode_tc.cuh, namespace sdec): each
 // (sequence, KV head) unit's slot space (window w + k selected tokens) is cut
-// into 128-slot tiles and those into `nsplit` ranges, one work item each.
+// into 128-slot tiles and those into `nsplit` <= 8 ranges, one work item each;
+// with more than one range, a unit's items are one thread-block cluster.
 struct SparseDecodePlan {
   int unit_tiles, nsplit, tiles_per_split, n_items;
 };
@@ -347,25 +348,18 @@ struct SparseDecodePlan {
 SparseDecodePlan sparse_decode_plan(const Shape& sh, const hs_sel* sel, int split_k) {
   SparseDecodePlan pl;
   const int U = sh.batch * sh.Hkv;
+  // ranges of equal slot counts (not whole tiles): the ranges of a unit finish together
   pl.unit_tiles = std::max(1, (sel->topk + sel->window + 127) / 128);
   int want = split_k > 0 ? split_k : std::max(1, num_sms() / std::max(1, U));
-  want = std::min(want, pl.unit_tiles);
+  want = std::min({want, pl.unit_tiles, dtc::sdec::kMaxSplit});
   pl.tiles_per_split = (pl.unit_tiles + want - 1) / want;
-  pl.nsplit = (pl.unit_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;  // no empty range
+  pl.nsplit = (pl.unit_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
   pl.n_items = U * pl.nsplit;
   return pl;
 }
 
-// Workspace: header | per-unit item counters | partial (m, l) [items][64] |
-// partial O [items][64][128] fp32 (used when a unit has more than one range).
-// Sized for the automatic split or any split_k up to the unit's tile count
-// (the largest split is one tile per item).
-size_t sparse_decode_ws_bytes(const Shape& sh, const hs_sel* sel) {
-  const size_t U = size_t(sh.batch) * sh.Hkv;
-  const size_t items = U * size_t(std::max(1, (sel->topk + sel->window + 127) / 128));
-  return align_up(kHeaderBytes + U * sizeof(int), 256) + align_up(items * 64 * 2 * sizeof(float), 256) +
-         align_up(items * 64 * 128 * sizeof(float), 256);
-}
+// Workspace: the header only (the ranges of a unit merge in shared memory).
+size_t sparse_decode_ws_bytes(const Shape&, const hs_sel*) { return kHeaderBytes; }
 
 // Token-level scores: items are (tile, KV head, 512-key range) up to the
 // tile's last query position.
@@ -825,15 +819,12 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   if (U > dtc::sdec::kMaxUnits) return HS_ERR_UNSUPPORTED;
   const SparseDecodePlan pl = sparse_decode_plan(sh, sel, split_k);
   cudaStream_t s = S(stream);
-  char* w = reinterpret_cast<char*>(ws);
-  const size_t off_ml = align_up(kHeaderBytes + size_t(U) * sizeof(int), 256);
-  const size_t off_o = off_ml + align_up(size_t(pl.n_items) * 64 * 2 * sizeof(float), 256);
   dtc::sdec::Params p{};
   p.idx = idx;
   p.cnt = sel->topk > 0 ? cnt : nullptr;
   p.cu_kv = vl->cu_kv;
-  p.k8 = reinterpret_cast<const uint8_t*>(k);
-  p.v8 = reinterpret_cast<const uint8_t*>(v);
+  p.k = reinterpret_cast<const uint8_t*>(k);
+  p.v = reinterpret_cast<const uint8_t*>(v);
   p.k_scale = k_scale;
   p.v_scale = v_scale;
   p.topk = sel->topk;
@@ -848,30 +839,41 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   p.unit_tiles = pl.unit_tiles;
   p.n_items = pl.n_items;
   p.scale_log2 = sh.scale * 1.4426950408889634f;
-  p.done = reinterpret_cast<int*>(w + kHeaderBytes);
-  p.part_ml = reinterpret_cast<float*>(w + off_ml);
-  p.part_o = reinterpret_cast<float*>(w + off_o);
   p.o = reinterpret_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.wc = wait_ctl(ws);
-  if (cudaMemsetAsync(p.done, 0, size_t(U) * sizeof(int), s) != cudaSuccess) return HS_ERR_CUDA;
-  Maps m;
-  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 1)) return HS_ERR_CUDA;
-  m.k = m.v = m.q;
-  if (!fp8 && (!make_map_rows(&m.k, k, sh.d, sh.Tkv * sh.Hkv) || !make_map_rows(&m.v, v, sh.d, sh.Tkv * sh.Hkv)))
-    return HS_ERR_CUDA;
-  const int grid = std::min(num_sms(), pl.n_items);
-  constexpr int smem = dtc::sdec::smem_bytes();
-  if (fp8) {
-    static PerDeviceOnce once;
-    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<true>, smem) != cudaSuccess) return HS_ERR_CUDA;
-    dtc::sdec::sparse_decode_tc_kernel<true><<<grid, dtc::sdec::threads<true>(), smem, s>>>(m.q, m.k, m.v, p);
-  } else {
-    static PerDeviceOnce once;
-    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<false>, smem) != cudaSuccess) return HS_ERR_CUDA;
-    dtc::sdec::sparse_decode_tc_kernel<false><<<grid, dtc::sdec::threads<false>(), smem, s>>>(m.q, m.k, m.v, p);
+  CUtensorMap map_q;
+  if (!make_map_3d(&map_q, q, sh.d, sh.Hq, sh.Tq, sh.G, 1)) return HS_ERR_CUDA;
+  // one range per unit: a persistent grid over the units; several: one CTA
+  // per range, a unit's ranges in one cluster
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(pl.nsplit > 1 ? pl.n_items : std::min(num_sms(), pl.n_items));
+  cfg.blockDim = dim3(dtc::sdec::kThreads);
+  cfg.stream = s;
+  if (pl.nsplit > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = unsigned(pl.nsplit);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
   }
-  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+  cudaError_t e;
+  if (fp8) {
+    cfg.dynamicSmemBytes = dtc::sdec::smem_bytes<true>();
+    static PerDeviceOnce once;
+    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<true>, int(cfg.dynamicSmemBytes)) != cudaSuccess)
+      return HS_ERR_CUDA;
+    e = cudaLaunchKernelEx(&cfg, dtc::sdec::sparse_decode_tc_kernel<true>, map_q, p);
+  } else {
+    cfg.dynamicSmemBytes = dtc::sdec::smem_bytes<false>();
+    static PerDeviceOnce once;
+    if (set_smem_once(once, dtc::sdec::sparse_decode_tc_kernel<false>, int(cfg.dynamicSmemBytes)) != cudaSuccess)
+      return HS_ERR_CUDA;
+    e = cudaLaunchKernelEx(&cfg, dtc::sdec::sparse_decode_tc_kernel<false>, map_q, p);
+  }
+  return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
 hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const void* k_swa, const void* v_swa,

@@ -724,68 +724,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 // other half, so O rows of copy c sum over that copy's keys only. At the end
 // of an item copy 1 hands its (m, l, O) to copy 0 through shared memory (the
 // Q buffer, free once the item's last QK is done).
-// The producer loads an item's sequence bounds once and the candidate
-// indices of eight tiles per round trip (FP8: then their scales), so the
-// slot lists cost about two memory latencies per eight tiles.
-// bf16 KV: the producer gathers the selected rows with tile::gather4 (each
-// lane four rows). FP8 KV: the producer only lists the rows; two converter
-// warps load the e4m3 codes and expand them into fp16 tiles (every e4m3 value
-// is an fp16 value), Q is converted to fp16 in shared memory, and the MMAs
-// run with fp16 operands. The K scale multiplies the logits, the V scale the
-// probabilities before PV.
+// The producer warp lists each tile's rows: it loads an item's sequence
+// bounds, selection count and first candidate indices in one round trip, and
+// the indices of several tiles per round trip after that (FP8: then their
+// scales). Two loader warps copy the listed rows with 16-byte cp.async, every
+// thread keeping several tiles' copies in flight: the rows are scattered
+// 256-byte (bf16) or 128-byte (FP8) pieces, and the number of bytes in flight
+// per SM is what bounds their rate. bf16 KV lands in the ring tile in the
+// 128-byte swizzle the MMA reads. FP8 KV lands in a staging tile; the thread
+// that copied a piece expands it to fp16 into the ring tile (every e4m3 value
+// is an fp16 value), Q is converted to fp16 in shared memory, and the MMAs run
+// with fp16 operands. The K scale multiplies the logits, the V scale the
+// probabilities before PV. The issuer thread loads Q (TMA) when the previous
+// item has released the buffer, so the slot lists and copies of the next item
+// run ahead across item boundaries.
 namespace sdec {
 
-constexpr int kStages = 5;      // 32 KB K or V tiles, in the order K0 V0 K1 V1 ...
-constexpr int kMeta = 4;        // per-tile slot metadata ring
 template <bool FP8>
-constexpr int batch_tiles() { return FP8 ? 4 : 8; }  // tiles whose slot lists are fetched per round trip
-constexpr int kMaxUnits = 4096;
+constexpr int stages() { return FP8 ? 4 : 5; }  // 32 KB K or V ring tiles, in the order K0 V0 K1 V1 ...
+constexpr int kMaxStages = 5;
+template <bool FP8>
+constexpr int lag() { return FP8 ? 2 : 3; }     // copy groups a loader thread keeps in flight behind the newest
+constexpr int kRaw = 3;                          // FP8 staging tiles (e4m3, 128 rows x 128 bytes) = lag + 1
+constexpr int kRawBytes = 128 * 128;
+constexpr int kMeta = 6;                         // per-tile slot metadata ring
+constexpr int kBatch = 8;                        // tiles whose candidate indices are fetched per round trip
+constexpr int kMaxUnits = 1 << 20;
+constexpr int kMaxSplit = 8;                     // a unit's ranges are one thread-block cluster (portable size)
+constexpr int kLoadWarps = 4;
+constexpr int kLoadThreads = 32 * kLoadWarps;
+// warps 0-3 softmax, 4 slot lists, 5 MMA issuer, 6-9 loaders
+constexpr int kThreads = 192 + kLoadThreads;
+static_assert(lag<true>() + 1 == kRaw, "FP8 staging ring = copy groups in flight");
 
 struct Meta {
   int row[128];       // packed row (token * Hkv + g) to load for each slot
   uint32_t valid[4];  // bit (4l + e) of word e: slot 4l + e holds a visible key
-  float ks[128], vs[128];
+  float ks[128], vs[128];  // FP8: the rows' scales, copied by the loaders with the tile's K
 };
 
+template <bool FP8>
 struct Layout {
-  static constexpr int kOffQ = 0;                             // 32 KB (Q, then copy 1's O at item end)
-  static constexpr int kOffKV = kTileBytes;                   // 5 x 32 KB
-  static constexpr int kOffMeta = kOffKV + kStages * kTileBytes;
+  static constexpr int kOffQ = 0;                                      // 32 KB (Q, then copy 1's O at item end)
+  static constexpr int kOffKV = kTileBytes;                            // ring of 32 KB tiles
+  static constexpr int kOffRaw = kOffKV + stages<FP8>() * kTileBytes;  // FP8 staging
+  static constexpr int kOffMeta = kOffRaw + (FP8 ? kRaw * kRawBytes : 0);
   static constexpr int kOffCtl = kOffMeta + kMeta * int(sizeof(Meta));
+  // at the end of a range (cluster launch): the range's (m, l) and unnormalised O, in the ring
+  static constexpr int kOffPartO = kOffKV;                 // [64 heads][32 float4], float4 j of head h at j ^ (h & 7)
+  static constexpr int kOffPartML = kOffKV + 64 * 128 * 4;  // [64] float2 (m, l), log2 units
 };
 
 struct Ctl {
   uint64_t q_full, q_ready, q_empty;
-  uint64_t kv_full[kStages], kv_empty[kStages];
-  uint64_t meta_full[kMeta], meta_empty[kMeta];
+  uint64_t kv_full[kMaxStages], kv_empty[kMaxStages];
+  uint64_t meta_full[kMeta], meta_empty[kMeta], sc_full[kMeta];
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t o_full, o_free, cbar, teardown;
   uint32_t tmem_base;
   int abort;
-  int last_flag;
   float cm[64], cl[64];  // copy 1's (m, l) at item end
 };
 
-constexpr int smem_bytes() { return Layout::kOffCtl + int(sizeof(Ctl)) + 1024; }
-static_assert(smem_bytes() <= 232448, "smem over 227 KB");
-
 template <bool FP8>
-constexpr int threads() { return FP8 ? 256 : 192; }  // + converter warps 6-7 for FP8
+constexpr int smem_bytes() { return Layout<FP8>::kOffCtl + int(sizeof(Ctl)) + 1024; }
+static_assert(smem_bytes<false>() <= 232448 && smem_bytes<true>() <= 232448, "smem over 227 KB");
+static_assert(Layout<true>::kOffPartML + 64 * 8 <= Layout<true>::kOffRaw, "partials fit in the ring");
 
 struct Params {
   const int* idx;     // [units, topk] (tile = sequence for decode)
   const int* cnt;     // [units]
   const int* cu_kv;   // device prefix sums
-  const uint8_t* k8;  // FP8 codes [T_kv, Hkv, 128]
-  const uint8_t* v8;
+  const uint8_t* k;   // cache rows [T_kv * Hkv]: 128 bf16 (256 bytes) or 128 e4m3 codes
+  const uint8_t* v;
   const float* k_scale;  // [T_kv, Hkv]
   const float* v_scale;
   int topk, w, G, Hq, Hkv, Tq;
   int n_units, nsplit, tiles_per_split, unit_tiles, n_items;
   float scale_log2;
-  float* part_o;   // [items][64][128] unnormalised O (nsplit > 1)
-  float* part_ml;  // [items][64][2] (m, l), log2 units
-  int* done;       // [units], zero on entry
   __nv_bfloat16* o;
   float* lse;
   WaitCtl wc;
@@ -802,32 +818,47 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Launch: nsplit == 1 -> grid min(SMs, items), each CTA loops over items;
+// nsplit > 1 -> one CTA per item, clusters of nsplit CTAs (a unit's ranges),
+// merged through distributed shared memory at the end.
 template <bool FP8>
-__global__ void __launch_bounds__(threads<FP8>(), 1)
-    sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kr,
-                            const __grid_constant__ CUtensorMap map_vr, const Params p) {
-  using L = Layout;
+__global__ void __launch_bounds__(kThreads, 1)
+    sparse_decode_tc_kernel(const __grid_constant__ CUtensorMap map_q, const Params p) {
+  using L = Layout<FP8>;
+  constexpr int kSt = stages<FP8>();
+  constexpr int kLag = lag<FP8>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl& c = *reinterpret_cast<Ctl*>(smem + L::kOffCtl);
   Meta* meta = reinterpret_cast<Meta*>(smem + L::kOffMeta);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kNT = threads<FP8>();
 
-  for (int i = threadIdx.x; i < kTileBytes / 16; i += kNT)
+  // the first item's sequence bounds, count and first candidate indices head
+  // for L2 while the CTA sets up (kBatch tiles = 32 lanes x 128 bytes)
+  if (warp == 4 && int(blockIdx.x) < p.n_items) {
+    const int u = blockIdx.x / p.nsplit;
+    const int j0 = (blockIdx.x % p.nsplit) * p.tiles_per_split * 128 - p.w + lane * 32;
+    if (lane == 0) {
+      prefetch_l2(p.cu_kv + u / p.Hkv);
+      if (p.cnt) prefetch_l2(p.cnt + u);
+    }
+    if (p.cnt && j0 + 31 >= 0 && j0 < p.topk) prefetch_l2(p.idx + size_t(u) * p.topk + max(j0, 0));
+  }
+  for (int i = threadIdx.x; i < kTileBytes / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem + L::kOffQ)[i] = make_uint4(0u, 0u, 0u, 0u);  // Q rows of absent heads
   fence_proxy_async_smem();
   if (threadIdx.x == 0) {
     mbar_init(&c.q_full, 1);
-    mbar_init(&c.q_ready, 2);  // FP8: the converter warps turned Q into fp16
-    mbar_init(&c.q_empty, 4);  // the softmax warps are done with the buffer (Q, then the copy merge)
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&c.kv_full[s], FP8 ? 2 : 1);
+    mbar_init(&c.q_ready, kLoadWarps);  // FP8: the loader warps turned Q into fp16
+    mbar_init(&c.q_empty, 4);           // the softmax warps are done with the buffer (Q, then the copy merge)
+    for (int s = 0; s < kSt; ++s) {
+      mbar_init(&c.kv_full[s], kLoadWarps);
       mbar_init(&c.kv_empty[s], 1);
     }
     for (int m = 0; m < kMeta; ++m) {
       mbar_init(&c.meta_full[m], 1);
-      mbar_init(&c.meta_empty[m], FP8 ? 6 : 4);  // softmax warps (+ converter warps)
+      mbar_init(&c.meta_empty[m], 4 + kLoadWarps);  // softmax warps and loader warps
+      mbar_init(&c.sc_full[m], kLoadWarps);         // FP8: the tile's scales have landed
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.s_full[i], 1);
@@ -845,13 +876,7 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
     tmem_alloc(&c.tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
-    prefetch_tensormap(&map_q);
-    if (!FP8) {
-      prefetch_tensormap(&map_kr);
-      prefetch_tensormap(&map_vr);
-    }
-  }
+  if (warp == 5 && lane == 0) prefetch_tensormap(&map_q);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -866,35 +891,19 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
   };
 
   if (warp == 4) {
-    // ============================ producer ============================
-    int ctr = 0, q_uses = 0, mctr = 0;
-    int last_use[kStages] = {-1, -1, -1, -1, -1};
+    // ============================ producer: slot lists ============================
+    int mctr = 0;
     bool ok = true;
-    auto wait0 = [&](uint64_t* bar, uint32_t parity, int site, int ctx) -> bool {
-      int r = 1;
-      if (lane == 0) r = mbar_wait(bar, parity, abort_flag, p.wc, site, ctx) ? 1 : 0;
-      return __shfl_sync(0xffffffffu, r, 0) != 0;
-    };
     for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
       int u, t0, t1;
       item_tiles(it, u, t0, t1);
       const int n = t1 - t0;
       const int b = u / p.Hkv, g = u % p.Hkv;
-      if (q_uses > 0 && !wait0(&c.q_empty, (q_uses - 1) & 1, 301, it << 8)) { ok = false; break; }
-      if (lane == 0) {
-        mbar_expect_tx(&c.q_full, 4 * 128 * p.G);
-        for (int cp = 0; cp < 2; ++cp)
-          for (int sl = 0; sl < 2; ++sl)
-            tma_load_3d(smem + L::kOffQ + sl * kSlab + cp * 64 * 128, &map_q, &c.q_full, sl * 64, g * p.G, b);
-      }
-      ++q_uses;
-      // the item's sequence bounds and selection count (one round trip)
+      // the sequence bounds, the selection count and the first batch of
+      // candidate indices do not depend on one another: one round trip
       const int kv0 = __ldg(p.cu_kv + b);
-      const int pos = __ldg(p.cu_kv + b + 1) - kv0 - 1;
+      const int kv1 = __ldg(p.cu_kv + b + 1);
       const int cnt = p.cnt ? __ldg(p.cnt + u) : 0;
-      const int win_lo = max(0, pos - p.w + 1);
-      const int n_win = p.w > 0 ? pos - win_lo + 1 : 0;
-      constexpr int kBatch = batch_tiles<FP8>();
       for (int tb = 0; tb < n && ok; tb += kBatch) {
         // slot keys of tiles tb .. tb + kBatch - 1 (lane: slots 4 lane .. 4 lane + 3 of each)
         int key[kBatch][4];
@@ -902,86 +911,57 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
         for (int bi = 0; bi < kBatch; ++bi)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int slot = (t0 + tb + bi) * 128 + lane * 4 + e;
-            const int jsel = slot - p.w;
-            key[bi][e] = (tb + bi < n && jsel >= 0 && jsel < cnt) ? __ldg(p.idx + size_t(u) * p.topk + jsel) : -1;
+            const int jsel = (t0 + tb + bi) * 128 + lane * 4 + e - p.w;
+            key[bi][e] = (p.cnt && tb + bi < n && jsel >= 0 && jsel < p.topk)
+                             ? __ldg(p.idx + size_t(u) * p.topk + jsel) : -1;
           }
+        const int pos = kv1 - kv0 - 1;
+        const int win_lo = max(0, pos - p.w + 1);
+        const int n_win = p.w > 0 ? pos - win_lo + 1 : 0;
 #pragma unroll
         for (int bi = 0; bi < kBatch; ++bi)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int slot = (t0 + tb + bi) * 128 + lane * 4 + e;
+            const int jsel = slot - p.w;
             if (slot < n_win) key[bi][e] = win_lo + slot;
-            else if (key[bi][e] > pos - p.w) key[bi][e] = -1;
+            else if (jsel < 0 || jsel >= cnt || key[bi][e] > pos - p.w) key[bi][e] = -1;
           }
-        float ksr[FP8 ? kBatch : 1][4], vsr[FP8 ? kBatch : 1][4];
-        if constexpr (FP8) {
-#pragma unroll
-          for (int bi = 0; bi < kBatch; ++bi)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k2 = key[bi][e];
-              const size_t row = (size_t(kv0) + (k2 >= 0 ? k2 : 0)) * p.Hkv + g;
-              ksr[bi][e] = k2 >= 0 ? __ldg(p.k_scale + row) : 0.f;
-              vsr[bi][e] = k2 >= 0 ? __ldg(p.v_scale + row) : 0.f;
-            }
-        }
 #pragma unroll
         for (int bi = 0; bi < kBatch; ++bi) {
           const int i = tb + bi;
           if (i < n && ok) {
-          // metadata of tile i
-          const int m = mctr % kMeta;
-          if (mctr >= kMeta && !wait0(&c.meta_empty[m], ((mctr / kMeta) - 1) & 1, 302, (it << 8) | i)) {
-            ok = false;
-            continue;
-          }
-          Meta& mt = meta[m];
-          int rows4[4];
-          uint32_t vbits = 0;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k2 = key[bi][e];
-            rows4[e] = (kv0 + (k2 >= 0 ? k2 : 0)) * p.Hkv + g;
-            mt.row[lane * 4 + e] = rows4[e];
-            if constexpr (FP8) {
-              mt.ks[lane * 4 + e] = ksr[bi][e];
-              mt.vs[lane * 4 + e] = vsr[bi][e];
+            const int m = mctr % kMeta;
+            bool got = true;
+            if (mctr >= kMeta) {
+              int r = 1;
+              if (lane == 0)
+                r = mbar_wait(&c.meta_empty[m], ((mctr / kMeta) - 1) & 1, abort_flag, p.wc, 302, (it << 8) | i) ? 1 : 0;
+              got = __shfl_sync(0xffffffffu, r, 0) != 0;
             }
-            vbits |= uint32_t(k2 >= 0) << e;
-          }
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t bl = __ballot_sync(0xffffffffu, (vbits >> e) & 1u);
-            if (lane == 0) mt.valid[e] = bl;
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c.meta_full[m]);
-          ++mctr;
-          if constexpr (!FP8) {
-            // K(i), then V(i): 32 KB each, gathered by all lanes
-            for (int kv = 0; kv < 2 && ok; ++kv) {
-              const int s = ctr % kStages;
-              if (!wait0(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, 303, (it << 8) | i)) { ok = false; break; }
-              if (lane == 0) mbar_expect_tx(&c.kv_full[s], kTileBytes);
-              __syncwarp();
-              uint8_t* dst = smem + L::kOffKV + s * kTileBytes;
-              for (int sl = 0; sl < 2; ++sl)
-                tma_load_2d_gather4(dst + sl * kSlab + lane * 4 * 128, kv ? &map_vr : &map_kr, &c.kv_full[s],
-                                    sl * 64, rows4[0], rows4[1], rows4[2], rows4[3]);
-              last_use[s] = ctr;
-              ++ctr;
+            if (!got) {
+              ok = false;
+              continue;
             }
+            Meta& mt = meta[m];
+            uint32_t vbits = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k2 = key[bi][e];
+              mt.row[lane * 4 + e] = (kv0 + (k2 >= 0 ? k2 : 0)) * p.Hkv + g;
+              vbits |= uint32_t(k2 >= 0) << e;
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t bl = __ballot_sync(0xffffffffu, (vbits >> e) & 1u);
+              if (lane == 0) mt.valid[e] = bl;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c.meta_full[m]);
+            ++mctr;
           }
-          }  // i < n && ok
         }
       }
-    }
-    if (lane == 0 && *abort_flag) {
-      if (!FP8)
-        for (int s = 0; s < kStages; ++s)
-          if (last_use[s] >= 0) mbar_wait_drain(&c.kv_full[s], (last_use[s] / kStages) & 1, p.wc, 390);
-      if (q_uses > 0) mbar_wait_drain(&c.q_full, (q_uses - 1) & 1, p.wc, 391);
     }
   } else if (warp == 5) {
     // ============================ UMMA issuer ============================
@@ -995,8 +975,8 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
       const uint64_t v_desc0 = sdesc_sw128(smem_u32(smem + L::kOffKV), kSlab, 1024);
       auto kstep = [](int kk) { return uint64_t(((kk >> 2) * kSlab + (kk & 3) * 32) >> 4); };
       auto wait_kv = [&](int site, int ctx) -> int {
-        const int s = ctr % kStages;
-        if (!mbar_wait(&c.kv_full[s], (ctr / kStages) & 1, abort_flag, p.wc, site, ctx)) return -1;
+        const int s = ctr % kSt;
+        if (!mbar_wait(&c.kv_full[s], (ctr / kSt) & 1, abort_flag, p.wc, site, ctx)) return -1;
         ++ctr;
         return s;
       };
@@ -1016,7 +996,18 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
         int u, t0, t1;
         item_tiles(it, u, t0, t1);
         const int n = t1 - t0;
-        if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 310, it << 8)) { ok = false; break; }
+        const int b = u / p.Hkv, g = u % p.Hkv;
+        // Q of the item (two copies of its G heads) once the buffer is free
+        if (q_uses > 0 && !mbar_wait(&c.q_empty, (q_uses - 1) & 1, abort_flag, p.wc, 301, it << 8)) { ok = false; break; }
+        mbar_expect_tx(&c.q_full, 4 * 128 * p.G);
+        for (int cp = 0; cp < 2; ++cp)
+          for (int sl = 0; sl < 2; ++sl)
+            tma_load_3d(smem + L::kOffQ + sl * kSlab + cp * 64 * 128, &map_q, &c.q_full, sl * 64, g * p.G, b);
+        if (!mbar_wait(&c.q_full, q_uses & 1, abort_flag, p.wc, 310, it << 8)) {
+          mbar_wait_drain(&c.q_full, q_uses & 1, p.wc, 391);  // no copy outlives the kernel
+          ok = false;
+          break;
+        }
         if (FP8 && !mbar_wait(&c.q_ready, q_uses & 1, abort_flag, p.wc, 316, it << 8)) { ok = false; break; }
         ++q_uses;
         tc_fence_after();
@@ -1076,6 +1067,7 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
         const int buf = (tiles + i) & 1;
         const int mm = mctr % kMeta;
         if (!mbar_wait_warp(&c.meta_full[mm], (mctr / kMeta) & 1, abort_flag, p.wc, 320, (it << 8) | i) ||
+            (FP8 && !mbar_wait_warp(&c.sc_full[mm], (mctr / kMeta) & 1, abort_flag, p.wc, 324, (it << 8) | i)) ||
             !mbar_wait_warp(&c.s_full[buf], ((tiles + i) >> 1) & 1, abort_flag, p.wc, 321, (it << 8) | i)) {
           ok = false;
           break;
@@ -1189,7 +1181,8 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
         const bool direct = p.nsplit == 1;  // the item is the whole unit: write O and lse
         const float inv = direct ? (Lm > 0.f ? 1.f / Lm : 0.f) : 1.f;
         const float* src = scratch + h * kD;
-        float* po = p.part_o + (size_t(it) * 64 + h) * kD;
+        // a range's partial stays in this CTA's ring for the cluster merge
+        float4* po = reinterpret_cast<float4*>(smem + L::kOffPartO) + h * 32;
         uint2* dst = reinterpret_cast<uint2*>(p.o + (size_t(b) * p.Hq + g * p.G + min(h, p.G - 1)) * kD);
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -1205,7 +1198,7 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
                                          (__uint_as_float(ov[4 * q4 + 3]) * w0 + o1.w * w1) * inv);
             if (has_head) {
               if (direct) dst[ch * 8 + q4] = make_uint2(pack_bf16(v.x, v.y), pack_bf16(v.z, v.w));
-              else reinterpret_cast<float4*>(po + ch * 32)[q4] = v;
+              else po[(ch * 8 + q4) ^ (h & 7)] = v;
             }
           }
         }
@@ -1213,7 +1206,7 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
           if (direct) {
             if (p.lse) p.lse[size_t(g * p.G + h) * p.Tq + b] = (Lm > 0.f ? M + __log2f(Lm) : -INFINITY) * 0.69314718055994531f;
           } else {
-            reinterpret_cast<float2*>(p.part_ml)[size_t(it) * 64 + h] = make_float2(M, Lm);
+            reinterpret_cast<float2*>(smem + L::kOffPartML)[h] = make_float2(M, Lm);
           }
         }
       }
@@ -1224,113 +1217,135 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
         mbar_arrive(&c.q_empty);
       }
       ++items;
-      if (p.nsplit == 1) continue;
-      __threadfence();
-      if (!cbar(it)) { ok = false; break; }
-      if (r == 0) c.last_flag = (atomicAdd(p.done + u, 1) == p.nsplit - 1);
-      if (!cbar(it)) { ok = false; break; }
-      if (c.last_flag) {
-        // merge the unit's nsplit partials: thread = (head, half of d); the
-        // (m, l) of every range first, then two ranges' O at a time in flight
-        __threadfence();
-        const int hh = r >> 1, half = r & 1;
-        if (hh < p.G) {
-          const int pbase = u * p.nsplit;
-          float M = -INFINITY;
-          for (int q = 0; q < p.nsplit; ++q) M = fmaxf(M, __ldcg(p.part_ml + (size_t(pbase + q) * 64 + hh) * 2));
-          float Lsum = 0.f;
-          float4 acc[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (int q = 0; q < p.nsplit; q += 2) {
-            float wq[2] = {0.f, 0.f};
-            float4 v[2][16];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int qq = q + e;
-              if (qq < p.nsplit) {
-                const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml) + size_t(pbase + qq) * 64 + hh);
-                wq[e] = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
-                Lsum += wq[e] * ml.y;
-                const float4* src = reinterpret_cast<const float4*>(p.part_o + (size_t(pbase + qq) * 64 + hh) * kD + half * 64);
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[e][j] = __ldcg(src + j);
-              } else {
-#pragma unroll
-                for (int j = 0; j < 16; ++j) v[e][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                acc[j].x = fmaf(wq[e], v[e][j].x, acc[j].x);
-                acc[j].y = fmaf(wq[e], v[e][j].y, acc[j].y);
-                acc[j].z = fmaf(wq[e], v[e][j].z, acc[j].z);
-                acc[j].w = fmaf(wq[e], v[e][j].w, acc[j].w);
-              }
-          }
-          const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-          uint2* dst = reinterpret_cast<uint2*>(p.o + (size_t(b) * p.Hq + g * p.G + hh) * kD + half * 64);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            dst[j] = make_uint2(pack_bf16(acc[j].x * inv, acc[j].y * inv), pack_bf16(acc[j].z * inv, acc[j].w * inv));
-          if (p.lse && half == 0)
-            p.lse[size_t(g * p.G + hh) * p.Tq + b] = (Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY) * 0.69314718055994531f;
-        }
-      }
     }
-  } else if (FP8) {
-    // ============================ converter warps (FP8) ============================
-    // Q: bf16 -> fp16 in place once per item; K / V: e4m3 rows of the tile
-    // (8 threads per 128-byte row, 16 rows per thread) -> fp16 tiles in the
-    // 128-byte swizzle, in the ring order K0 V0 K1 V1 ...
-    const int t = threadIdx.x - 192;  // 0..63
-    int ctr = 0, q_uses = 0, mctr = 0;
+  } else {
+    // ============================ loader warps ============================
+    // Steps K0 V0 K1 V1 ... of the CTA's items, each 128 listed rows. Issue:
+    // 16-byte cp.async of every row piece (bf16: into ring tile `step % kSt`
+    // in the 128-byte swizzle; FP8: into staging tile `step % kRaw`, and with
+    // a K step the rows' K and V scales into the tile's metadata), one commit
+    // group per step. Completion, kLag steps later: wait for the thread's
+    // group (FP8: signal the scales, then expand the thread's own pieces to
+    // fp16 into the ring tile), fence for the tensor core, arrive on the
+    // tile's barrier. The ring tile is claimed at issue (bf16) or at
+    // completion (FP8); either way the issuer can always release enough
+    // tiles for the loaders to move on (it holds at most V(i) and K(i + 1)
+    // while waiting). Each warp issues its own copies: the number of warps
+    // issuing scattered copies is what sets the rate.
+    const int t = threadIdx.x - 192;  // 0 .. kLoadThreads - 1
+    int issued = 0, completed = 0, mi = 0, cmi = 0, q_uses = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < p.n_items && ok; it += gridDim.x) {
+    // cursors over (item, step within the item)
+    int iss_it = blockIdx.x, iss_n = 0, iss_i2 = 0, cmp_it = blockIdx.x, cmp_n = 0, cmp_i2 = 0;
+    auto item_len = [&](int it) {
       int u, t0, t1;
       item_tiles(it, u, t0, t1);
-      const int n = t1 - t0;
-      if (!mbar_wait_warp(&c.q_full, q_uses & 1, abort_flag, p.wc, 330, it << 8)) { ok = false; break; }
-      for (int qc = 0; qc < 32; ++qc) {  // rows t and t + 64 of the Q tile: 16 chunks of 8 values each
-        const int qr = t + 64 * (qc >> 4), chn = qc & 15;
-        uint8_t* ptr = smem + L::kOffQ + (chn >> 3) * kSlab + qr * 128 + (((chn & 7) ^ (qr & 7)) << 4);
-        uint4 v = *reinterpret_cast<uint4*>(ptr);
-        uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
-          w4[e] = pack_f16(f.x, f.y);
-        }
-        *reinterpret_cast<uint4*>(ptr) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&c.q_ready);
-      ++q_uses;
-      for (int step = 0; step < 2 * n && ok; ++step) {
-        const int tile = step >> 1;
-        const bool is_v = step & 1;
-        const int mi = mctr + tile;  // meta entry of that tile
+      return t1 - t0;
+    };
+    if (iss_it < p.n_items) iss_n = cmp_n = item_len(iss_it);
+    while (ok) {
+      if (iss_it < p.n_items) {
+        const bool is_v = iss_i2 & 1;
         const int mm = mi % kMeta;
-        if (!mbar_wait_warp(&c.meta_full[mm], (mi / kMeta) & 1, abort_flag, p.wc, 331, (it << 8) | tile)) { ok = false; break; }
-        const int s = ctr % kStages;
-        if (!mbar_wait_warp(&c.kv_empty[s], ((ctr / kStages) & 1) ^ 1, abort_flag, p.wc, 332, (it << 8) | tile)) { ok = false; break; }
-        const Meta& mt = meta[mm];
-        const uint8_t* src = is_v ? p.v8 : p.k8;
-        uint8_t* dst = smem + L::kOffKV + s * kTileBytes;
-        const int sub = t & 7;  // 16-code chunk of the row
-        uint4 raw[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int row = (t >> 3) + 8 * j;
-          raw[j] = __ldg(reinterpret_cast<const uint4*>(src + size_t(mt.row[row]) * kD) + sub);
+        const int ctx = (iss_it << 8) | (iss_i2 >> 1);
+        if (!is_v && !mbar_wait_warp(&c.meta_full[mm], (mi / kMeta) & 1, abort_flag, p.wc, 331, ctx)) {
+          ok = false;
+          break;
         }
+        const int* rows = meta[mm].row;
+        const uint8_t* src = is_v ? p.v : p.k;
+        if constexpr (!FP8) {
+          const int s = issued % kSt;
+          if (!mbar_wait_warp(&c.kv_empty[s], ((issued / kSt) & 1) ^ 1, abort_flag, p.wc, 332, ctx)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = smem + L::kOffKV + s * kTileBytes;
+          const int ch = t & 15;  // 16-byte piece of the 256-byte row
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int row = (t >> 3) + 8 * j;
-          const uint32_t w4[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+          for (int j = 0; j < 2048 / kLoadThreads; ++j) {
+            const int row = (t >> 4) + (kLoadThreads / 16) * j;
+            cp_async16(dst + (ch >> 3) * kSlab + row * 128 + (((ch & 7) ^ (row & 7)) << 4),
+                       src + size_t(rows[row]) * 256 + ch * 16);
+          }
+        } else {
+          uint8_t* dst = smem + L::kOffRaw + (issued % kRaw) * kRawBytes;
+          const int sub = t & 7;  // 16-code piece of the 128-byte row
+#pragma unroll
+          for (int j = 0; j < 1024 / kLoadThreads; ++j) {
+            const int row = (t >> 3) + (kLoadThreads / 8) * j;
+            cp_async16(dst + row * 128 + sub * 16, src + size_t(rows[row]) * 128 + sub * 16);
+          }
+          if (!is_v) {
+            static_assert(kLoadThreads == 128, "one scale pair per loader thread");
+            cp_async4(&meta[mm].ks[t], p.k_scale + rows[t]);
+            cp_async4(&meta[mm].vs[t], p.v_scale + rows[t]);
+          }
+        }
+        cp_async_commit();
+        if (is_v) {  // the loaders are done with the tile's row list
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.meta_empty[mm]);
+          ++mi;
+        }
+        ++issued;
+        if (++iss_i2 == 2 * iss_n) {
+          iss_i2 = 0;
+          iss_it += gridDim.x;
+          if (iss_it < p.n_items) iss_n = item_len(iss_it);
+        }
+      }
+      if (completed == issued) break;
+      const bool tail = iss_it >= p.n_items;
+      if (!tail && issued - completed <= kLag) continue;
+      if (tail) cp_async_wait<0>();
+      else cp_async_wait<kLag>();
+      // ---- completion of step `completed` ----
+      const int s = completed % kSt;
+      const int ctx = (cmp_it << 8) | (cmp_i2 >> 1);
+      if constexpr (FP8) {
+        if (!(cmp_i2 & 1)) {  // a K step: the tile's scales are in place
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.sc_full[cmi % kMeta]);
+        } else {
+          ++cmi;
+        }
+        if (cmp_i2 == 0) {
+          // the item's first step: its Q (row t) to fp16 for the issuer
+          if (!mbar_wait_warp(&c.q_full, q_uses & 1, abort_flag, p.wc, 330, ctx)) {
+            ok = false;
+            break;
+          }
+          static_assert(kLoadThreads == 128, "one Q row per loader thread");
+#pragma unroll 4
+          for (int chn = 0; chn < 16; ++chn) {
+            uint8_t* ptr = smem + L::kOffQ + (chn >> 3) * kSlab + t * 128 + (((chn & 7) ^ (t & 7)) << 4);
+            uint4 v = *reinterpret_cast<uint4*>(ptr);
+            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+              w4[e] = pack_f16(f.x, f.y);
+            }
+            *reinterpret_cast<uint4*>(ptr) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&c.q_ready);
+          ++q_uses;
+        }
+        if (!mbar_wait_warp(&c.kv_empty[s], ((completed / kSt) & 1) ^ 1, abort_flag, p.wc, 332, ctx)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = smem + L::kOffRaw + (completed % kRaw) * kRawBytes;
+        uint8_t* dst = smem + L::kOffKV + s * kTileBytes;
+        const int sub = t & 7;
+#pragma unroll 4
+        for (int j = 0; j < 1024 / kLoadThreads; ++j) {
+          const int row = (t >> 3) + (kLoadThreads / 8) * j;
+          const uint4 r4 = *reinterpret_cast<const uint4*>(raw + row * 128 + sub * 16);  // this thread's copy
+          const uint32_t w4[4] = {r4.x, r4.y, r4.z, r4.w};
           uint32_t hv[8];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -1345,17 +1360,18 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
                 make_uint4(hv[4 * hc], hv[4 * hc + 1], hv[4 * hc + 2], hv[4 * hc + 3]);
           }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&c.kv_full[s]);
-        ++ctr;
-        if (is_v) {  // the converters are done with the tile's metadata
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&c.meta_empty[mm]);
-        }
       }
-      mctr += n;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.kv_full[s]);
+      ++completed;
+      if (++cmp_i2 == 2 * cmp_n) {
+        cmp_i2 = 0;
+        cmp_it += gridDim.x;
+        if (cmp_it < p.n_items) cmp_n = item_len(cmp_it);
+      }
     }
+    cp_async_wait<0>();  // no copy outlives the loaders (abort paths included)
   }
 
   tc_fence_before();
@@ -1363,6 +1379,52 @@ __global__ void __launch_bounds__(threads<FP8>(), 1)
   if (warp == 5) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (p.nsplit > 1) {
+    // ---- the unit's ranges are the CTAs of this cluster: merge their partials ----
+    // CTA rank r writes heads r, r + nsplit, ...; thread = (head, quarter of d).
+    // Every thread of every CTA passes both cluster barriers (abort paths too):
+    // the second keeps each CTA's shared memory alive while its peers read it.
+    cluster_sync_all();
+    const int rank = int(cluster_ctarank());
+    const int t = threadIdx.x;
+    const int hh = rank + p.nsplit * (t >> 2), part = t & 3;
+    if (t < 128 && hh < p.G) {
+      const int u = blockIdx.x / p.nsplit, b = u / p.Hkv, g = u % p.Hkv;
+      const float2* ml_local = reinterpret_cast<const float2*>(smem + L::kOffPartML) + hh;
+      const float4* o_local = reinterpret_cast<const float4*>(smem + L::kOffPartO) + hh * 32;
+      float M = -INFINITY;
+      for (int q = 0; q < p.nsplit; ++q) M = fmaxf(M, ld_dsmem_f2(dsmem_addr(ml_local, q)).x);
+      float Lsum = 0.f;
+      float4 acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int q = 0; q < p.nsplit; ++q) {
+        const float2 ml = ld_dsmem_f2(dsmem_addr(ml_local, q));
+        const float wq = ml.x == -INFINITY ? 0.f : ex2(ml.x - M);
+        Lsum += wq * ml.y;
+        float4 v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = ld_dsmem_f4(dsmem_addr(o_local + ((part * 8 + e) ^ (hh & 7)), q));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          acc[e].x = fmaf(wq, v[e].x, acc[e].x);
+          acc[e].y = fmaf(wq, v[e].y, acc[e].y);
+          acc[e].z = fmaf(wq, v[e].z, acc[e].z);
+          acc[e].w = fmaf(wq, v[e].w, acc[e].w);
+        }
+      }
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (size_t(b) * p.Hq + g * p.G + hh) * kD + part * 32);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2)
+        dst[e >> 1] = make_uint4(pack_bf16(acc[e].x * inv, acc[e].y * inv), pack_bf16(acc[e].z * inv, acc[e].w * inv),
+                                 pack_bf16(acc[e + 1].x * inv, acc[e + 1].y * inv),
+                                 pack_bf16(acc[e + 1].z * inv, acc[e + 1].w * inv));
+      if (p.lse && part == 0)
+        p.lse[size_t(g * p.G + hh) * p.Tq + b] = (Lsum > 0.f ? M + __log2f(Lsum) : -INFINITY) * 0.69314718055994531f;
+    }
+    cluster_sync_all();
   }
 }
 

@@ -208,9 +208,12 @@ HS_API hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel,
  * The slots of each (sequence, KV head) -- the window, then the selected
  * tokens -- form ceil((k + w) / 128) tiles of 128 keys, cut into split_k
  * contiguous ranges of whole tiles, one tensor-core work item each; the
- * ranges' partial results are merged by log-sum-exp inside the same launch.
+ * ranges of a unit run as one thread-block cluster and their partial results
+ * are merged by log-sum-exp through the cluster's shared memory, inside the
+ * same launch (the workspace holds only the error header).
  * split_k: 0 = automatic (about one range per SM over all units); a value
- * above the tile count is clamped to it; negative values are rejected.
+ * above the tile count or above 8 (the portable cluster size) is clamped;
+ * negative values are rejected.
  * An empty batch (T_q = 0) returns HS_OK without touching any pointer.
  * Requires n_b = 1 for every sequence and sel->q_tile = 1.
  */
