@@ -299,6 +299,23 @@ def visible_counts(w, idx, cnt):
     return float(total)
 
 
+def distinct_selected_rows(w, idx, cnt):
+    """Distinct (token, KV head) rows among all tiles' selected tokens: what a
+    gather of the selected rows has to read at least once (neighbouring tiles
+    share most of their selections)."""
+    dev = idx.device
+    tile_seq = []
+    for b, (a, e) in enumerate(zip(w.cu_q()[:-1], w.cu_q()[1:])):
+        tile_seq += [b] * ((e - a + w.q_tile - 1) // w.q_tile)
+    kv0 = torch.tensor(w.cu_kv()[:-1], device=dev)[torch.tensor(tile_seq, device=dev)]
+    total = 0
+    for g in range(w.n_kv_heads):
+        valid = torch.arange(w.topk, device=dev)[None, :] < cnt[:, g, None]
+        rows = (kv0[:, None] + idx[:, g, :w.topk].long())[valid]
+        total += int(torch.unique(rows).numel())
+    return total
+
+
 def needle_recall(w, inp, idx, cnt):
     """Share of planted keys that the sparse layers see from the query they
     were aimed at: the key lies in that query's forced window, or its block is
@@ -343,8 +360,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     import torch.distributed as dist
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
-                                                  sparse_attn_decode, sparse_swa_gated_prefill, HS_KV_BF16,
-                                                  HS_KV_FP8_E4M3)
+                                                  sparse_attn_decode, sparse_swa_gated_prefill,
+                                                  gather_selected_kv, HS_KV_BF16, HS_KV_FP8_E4M3)
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
     w = workload(args) if w is None else w
@@ -375,7 +392,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     hs.check_error(blk.ws)
     recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"]) if world == 1 else None
 
-    kinds = ["full", "topk", "sparse"]
+    kinds = ["full", "topk", "sparse"] + (["gather"] if blk.gathered else [])
     L0 = layers[0]
 
     def call(kind, st):
@@ -386,6 +403,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                              ws=blk.ws, stream=st)
         elif kind == "topk":
             topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws, stream=st)
+        elif kind == "gather":
+            gather_selected_kv(vl, sel, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["kg"], bufs["vg"], stream=st)
         elif blk.decode:
             if fp8_kv is not None:
                 sparse_attn_decode(vl, sel, L0.q, inp.k_fp8, inp.v_fp8, bufs["idx"], bufs["cnt"], inp.k_scale,
@@ -400,7 +419,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                                      L0.v_swa, L0.gamma, o=bufs["o_l0"], ws=blk.ws, stream=st)
         else:
             sparse_attn_prefill(vl, sel, L0.q, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["o_sp0"],
-                                bufs["lse_sp0"], ws=blk.ws, stream=st)
+                                bufs["lse_sp0"], ws=blk.ws, stream=st, kg=bufs.get("kg"), vg=bufs.get("vg"))
 
     # Launch-bound steps (decode: dozens of microsecond kernels) would time the
     # host's enqueue rate rather than the GPU, so the step and every kernel
@@ -513,7 +532,12 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
         swa_flop = 4.0 * d * hq * swa_pairs(w) if w.swa_window > 0 else 0.0
         entry("sparse", kms["sparse"], 4.0 * d * G * vis + swa_flop, "tensor")
     entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
-    per_step = {"full": 1, "topk": 1, "sparse": len(layers)}
+    if blk.gathered:
+        # K and V: every (tile, KV head) plane of topk rows written once, the
+        # distinct selected rows read once (the rest of the reads hit L2)
+        uniq = distinct_selected_rows(w, blk._bufs["idx"], blk._bufs["cnt"])
+        entry("gather", kms["gather"], (n_tiles * hkv * w.topk + uniq) * d * 2 * 2, "hbm")
+    per_step = {"full": 1, "topk": 1, "sparse": len(layers), "gather": 1}
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])

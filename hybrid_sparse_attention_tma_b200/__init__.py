@@ -17,8 +17,8 @@ from . import _lib as L
 from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
 
 __all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
-           "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "kv_dequantize", "workspace_size",
-           "check_error", "HsError"]
+           "gather_selected_kv", "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "kv_dequantize",
+           "workspace_size", "check_error", "HsError"]
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -144,8 +144,10 @@ def topk_select(vl: Varlen, sel: L.HsSel, scores, idx=None, cnt=None, ws: Option
 
 
 def sparse_attn_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, o=None, lse=None,
-                        ws: Optional[Workspace] = None, stream=None, want_lse: bool = True):
-    """Sparse layer over the reused KV cache and indices. Returns (o, lse)."""
+                        ws: Optional[Workspace] = None, stream=None, want_lse: bool = True, kg=None, vg=None):
+    """Sparse layer over the reused KV cache and indices. Returns (o, lse).
+    With kg / vg from gather_selected_kv (token-level selection) the selected
+    rows are read from those buffers (same result)."""
     lib = L.load()
     dev = q.device
     Tq, Hq, d = q.shape
@@ -154,10 +156,29 @@ def sparse_attn_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, o=None, lse
         lse = torch.empty((Hq, Tq), dtype=torch.float32, device=dev)
     w = _ws(ws, dev)
     buf = w.get(workspace_size(L.HS_OP_SPARSE_ATTN_PREFILL, vl, sel), stream)
+    if kg is not None:
+        L.check("hs_sparse_attn_prefill_gathered", lib.hs_sparse_attn_prefill_gathered(
+            ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(kg), _ptr(vg), _ptr(idx),
+            _ptr(cnt), _ptr(o), _ptr(lse), _ptr(buf), buf.numel(), _stream(stream)))
+        return o, lse
     L.check("hs_sparse_attn_prefill", lib.hs_sparse_attn_prefill(
         ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), _ptr(o),
         _ptr(lse), _ptr(buf), buf.numel(), _stream(stream)))
     return o, lse
+
+
+def gather_selected_kv(vl: Varlen, sel: L.HsSel, k, v, idx, cnt, kg=None, vg=None, stream=None):
+    """Token-level selection: the selected tokens' K / V rows of every
+    (selection tile, KV head), [n_tiles, H_kv, topk, d], zero past cnt; once
+    per block, read by every sparse prefill layer. Returns (kg, vg)."""
+    lib = L.load()
+    shape = (vl.n_tiles(sel.q_tile), vl.n_kv_heads, max(sel.topk, 1), k.shape[-1])
+    kg = torch.empty(shape, dtype=k.dtype, device=k.device) if kg is None else kg
+    vg = torch.empty(shape, dtype=v.dtype, device=v.device) if vg is None else vg
+    L.check("hs_gather_selected_kv", lib.hs_gather_selected_kv(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(k), _ptr(v), _ptr(idx), _ptr(cnt), _ptr(kg), _ptr(vg),
+        _stream(stream)))
+    return kg, vg
 
 
 def sparse_swa_gated_prefill(vl: Varlen, sel: L.HsSel, q, k, v, idx, cnt, swa_window: int, k_swa, v_swa, gamma,

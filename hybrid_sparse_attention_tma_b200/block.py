@@ -13,7 +13,7 @@ from typing import List, Optional
 import torch
 
 from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
-               swa_gated, sparse_swa_gated_prefill, kv_dequantize, HS_KV_BF16, HS_KV_FP8_E4M3)
+               swa_gated, sparse_swa_gated_prefill, kv_dequantize, gather_selected_kv, HS_KV_BF16, HS_KV_FP8_E4M3)
 
 
 @dataclass
@@ -40,6 +40,9 @@ class HybridBlock:
         # the split-K decode path
         self.decode = q_tile == 1 and block == 1 and all(
             b - a == 1 for a, b in zip(vl.cu_q_list, vl.cu_q_list[1:]))
+        # token-level prefill: the selected rows are gathered once per block
+        # (hs_gather_selected_kv) and every plain sparse layer reads them
+        self.gathered = (not self.decode and block == 1 and topk > 0 and not (swa_window > 0 and fused))
 
     def _buf(self, name, shape, dtype):
         t = self._bufs.get(name)
@@ -76,6 +79,11 @@ class HybridBlock:
             v = kv_dequantize(vq, vs, self._buf("v_deq", tuple(vq.shape), torch.bfloat16), stream=stream)
         full_attn_select(vl, sel, q, k, v, o, lse, scores, ws=self.ws, stream=stream)
         topk_select(vl, sel, scores, idx, cnt, ws=self.ws, stream=stream)
+        kg = vg = None
+        if self.gathered and layers:
+            gshape = (nt, vl.n_kv_heads, sel.topk, d)
+            kg, vg = gather_selected_kv(vl, sel, k, v, idx, cnt, self._buf("kg", gshape, torch.bfloat16),
+                                        self._buf("vg", gshape, torch.bfloat16), stream=stream)
         outs = []
         for i, L in enumerate(layers):
             tag = str(i) if keep_all else str(i % 2)
@@ -98,7 +106,8 @@ class HybridBlock:
                 outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
                 continue
             else:
-                sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream)
+                sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream,
+                                    kg=kg, vg=vg)
             if self.swa_window > 0:
                 o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
                 swa_gated(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, ws=self.ws,
@@ -114,11 +123,13 @@ class HybridBlock:
         score pass) / 1 (decode: both passes in one launch); top-k 1; each
         sparse layer 1 (prefill, with its window branch and gate when fused;
         decode, with its key ranges merged in the same launch), plus 1 for an
-        unfused gated SWA branch; an FP8 prefill adds the two expansions."""
+        unfused gated SWA branch; an FP8 prefill adds the two expansions, a
+        token-level prefill the gather of the selected rows."""
         if self.decode:
             full = 1
         else:
             full = 1 if self.sel.block > 1 else 3
         sparse = 1
         swa = 1 if (self.swa_window > 0 and not (self.fused and not self.decode)) else 0
-        return full + 1 + n_layers * (sparse + swa) + (2 if fp8_prefill else 0)
+        gather = 1 if (self.gathered and n_layers > 0) else 0
+        return full + 1 + n_layers * (sparse + swa) + (2 if fp8_prefill else 0) + gather

@@ -149,6 +149,13 @@ bool fill_seqtable(const hs_varlen* vl, int T, SeqTable* st) {
   return true;
 }
 
+// Selection tiles of a batch: sum over sequences of ceil(n_b / T).
+long long n_sel_tiles(const hs_varlen* vl, int T) {
+  long long n = 0;
+  for (int b = 0; b < vl->batch; ++b) n += (vl->cu_q_host[b + 1] - vl->cu_q_host[b] + T - 1) / T;
+  return n;
+}
+
 // Schedule of the tcgen05 attention kernel (see attn::Sched).
 bool fill_sched(const hs_varlen* vl, const Shape& sh, int mode, int T, int chunks_per_tile, attn::Sched* sc) {
   if (vl->batch > attn::kMaxSched) return false;
@@ -697,9 +704,15 @@ struct SwaArgs {
   void* o_sparse;  // optional
 };
 
+// Selected rows gathered once per block (token level): kg / vg [n_tiles][Hkv][topk][d].
+struct GatheredKV {
+  const void* kg;
+  const void* vg;
+};
+
 static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k, const void* v,
                               const int32_t* idx, const int32_t* cnt, void* o, float* lse, const SwaArgs* swa,
-                              void* ws, size_t ws_bytes, hs_stream_t stream) {
+                              void* ws, size_t ws_bytes, hs_stream_t stream, const GatheredKV* gkv = nullptr) {
   Shape sh;
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
@@ -716,11 +729,20 @@ static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void
   if (!is_pow2(sh.G) || sh.G > 128) return HS_ERR_UNSUPPORTED;
   if (vl->batch > attn::kMaxSched) return HS_ERR_UNSUPPORTED;
   const int T = sel->q_tile, B = sel->block;
+  if (gkv && (B != 1 || swa || !gkv->kg || !gkv->vg || !aligned16(gkv->kg) || !aligned16(gkv->vg)))
+    return HS_ERR_INVALID_ARG;
   Maps m;
   if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, 128 / sh.G) ||
       !make_map_3d(&m.k, k, sh.d, sh.Hkv, sh.Tkv, 1, 128) || !make_map_3d(&m.v, v, sh.d, sh.Hkv, sh.Tkv, 1, 128))
     return HS_ERR_CUDA;
-  if (B == 1) {
+  if (gkv) {
+    // planes of topk slots, one per (selection tile, KV head); 128-slot boxes
+    const long long planes = (long long)n_sel_tiles(vl, T) * sh.Hkv;
+    if (sel->topk > 0 && (!make_map_3d(&m.kb, gkv->kg, sh.d, sel->topk, planes, 128, 1) ||
+                          !make_map_3d(&m.vb, gkv->vg, sh.d, sel->topk, planes, 128, 1)))
+      return HS_ERR_CUDA;
+    if (sel->topk == 0) m.kb = m.vb = m.k;
+  } else if (B == 1) {
     if (!make_map_rows(&m.kb, k, sh.d, sh.Tkv * sh.Hkv) || !make_map_rows(&m.vb, v, sh.d, sh.Tkv * sh.Hkv))
       return HS_ERR_CUDA;
   } else if (!make_map_3d(&m.kb, k, sh.d, sh.Hkv, sh.Tkv, 1, B) || !make_map_3d(&m.vb, v, sh.d, sh.Hkv, sh.Tkv, 1, B)) {
@@ -750,6 +772,7 @@ static hs_status sparse_layer(const hs_varlen* vl, const hs_sel* sel, const void
   p.cnt = cnt;
   p.topk = sel->topk;
   p.w = sel->window;
+  p.gathered = gkv ? 1 : 0;
   p.wc = wait_ctl(ws);
   if (swa) {
     p.ws = swa->window;
@@ -785,6 +808,66 @@ hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel, const v
                                  const void* v, const int32_t* idx, const int32_t* cnt, void* o, float* lse,
                                  void* ws, size_t ws_bytes, hs_stream_t stream) {
   return sparse_layer(vl, sel, q, k, v, idx, cnt, o, lse, nullptr, ws, ws_bytes, stream);
+}
+
+hs_status hs_sparse_attn_prefill_gathered(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                          const void* v, const void* kg, const void* vg, const int32_t* idx,
+                                          const int32_t* cnt, void* o, float* lse, void* ws, size_t ws_bytes,
+                                          hs_stream_t stream) {
+  const GatheredKV gkv{kg, vg};
+  return sparse_layer(vl, sel, q, k, v, idx, cnt, o, lse, nullptr, ws, ws_bytes, stream, &gkv);
+}
+
+// One CTA per (selection tile, KV head) plane; thread = 16-byte piece of a
+// slot row (16 consecutive threads read one 256-byte row and write it out
+// contiguously). Slots past cnt are zero. HBM-bound: 2 x (topk rows read +
+// topk rows written) per plane.
+__global__ void __launch_bounds__(256) gather_selected_kernel(const __grid_constant__ SeqTable st, int Hkv, int topk,
+                                                              int pieces, const uint4* __restrict__ k,
+                                                              const uint4* __restrict__ v, const int* __restrict__ idx,
+                                                              const int* __restrict__ cnt, uint4* __restrict__ kg,
+                                                              uint4* __restrict__ vg) {
+  const int plane = blockIdx.x;  // tile * Hkv + g
+  const int tile = plane / Hkv, g = plane % Hkv;
+  const TileInfo ti = tile_info(st, tile);
+  const int c = __ldg(cnt + plane);
+  const int* ip = idx + size_t(plane) * topk;
+  const size_t base = size_t(plane) * topk * pieces;
+  const int n = topk * pieces;
+#pragma unroll 4
+  for (int e = threadIdx.x; e < n; e += blockDim.x) {
+    const int s = e / pieces, pc = e - s * pieces;
+    uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+    if (s < c) {
+      const size_t row = (size_t(ti.kv0) + __ldg(ip + s)) * Hkv + g;
+      kv = __ldg(k + row * pieces + pc);
+      vv = __ldg(v + row * pieces + pc);
+    }
+    kg[base + e] = kv;
+    vg[base + e] = vv;
+  }
+}
+
+hs_status hs_gather_selected_kv(const hs_varlen* vl, const hs_sel* sel, const void* k, const void* v,
+                                const int32_t* idx, const int32_t* cnt, void* kg, void* vg, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sel->block != 1) return HS_ERR_INVALID_ARG;
+  if (sh.Tq == 0 || sel->topk == 0) return HS_OK;
+  if (!k || !v || !idx || !cnt || !kg || !vg || !aligned16(k) || !aligned16(v) || !aligned16(kg) || !aligned16(vg))
+    return HS_ERR_INVALID_ARG;
+  if (sh.d % 8) return HS_ERR_UNSUPPORTED;
+  SeqTable table;
+  if (!fill_seqtable(vl, sel->q_tile, &table)) return HS_ERR_UNSUPPORTED;
+  const long long planes = (long long)table.n_tiles * sh.Hkv;
+  if (planes == 0) return HS_OK;
+  if (planes > INT32_MAX) return HS_ERR_UNSUPPORTED;
+  gather_selected_kernel<<<unsigned(planes), 256, 0, S(stream)>>>(
+      table, sh.Hkv, sel->topk, sh.d / 8, reinterpret_cast<const uint4*>(k), reinterpret_cast<const uint4*>(v), idx,
+      cnt, reinterpret_cast<uint4*>(kg), reinterpret_cast<uint4*>(vg));
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
 }
 
 hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,

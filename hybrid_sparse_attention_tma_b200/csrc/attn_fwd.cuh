@@ -115,6 +115,7 @@ struct Params {
   const int* cnt;  // [n_tiles, Hkv]
   int topk;
   int w;
+  int gathered;    // token level: map_kb / map_vb view buffers of the selected rows, [n_tiles * Hkv][topk][D]
   // gate epilogue (sliding-window branch): o = sig(gamma) * o_other + (1 - sig(gamma)) * o_this
   const float* gamma;                // [Tq, Hq] or null
   const __nv_bfloat16* o_other;      // [Tq, Hq, D] sparse-branch output
@@ -374,7 +375,13 @@ __global__ void __launch_bounds__(threads_for<MODE, SB>(), 1)
                 tma_load_3d(dst + sl * kSlabBytes, mc, &c.kv_full[s], sl * 64, it.g, it.kv0 + key0);
           } else {
             const CUtensorMap* mb = kind == 0 ? &map_kb : &map_vb;
-            if constexpr (SB == 1) {
+            if (SB == 1 && p.gathered) {
+              // token level, rows gathered once per block: slots i*128 .. i*128+127
+              // of the (tile, kv head) plane are one tile load
+              if (lane == 0)
+                for (int sl = 0; sl < L::kSlabs; ++sl)
+                  tma_load_3d(dst + sl * kSlabBytes, mb, &c.kv_full[s], sl * 64, i * 128, it.tile0 * p.Hkv + it.g);
+            } else if constexpr (SB == 1) {
               // token level: lane l gathers selected rows 4l..4l+3 of the tile
               // from the 2-D row view (row = token * H_kv + kv head); padded
               // slots re-read the first selected row and are masked

@@ -209,27 +209,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       ++items;
+      // the chunk's lse values (rows lane + 32 k, row = query * G + head-in-group)
+      // are loaded one chunk ahead, so their latency overlaps the ring wait
+      const int qpc = 128 / p.G;
+      const float inv_c = 1.f / p.scale_log2;
+      auto load_lse = [&](int qc, float (&x)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = lane + 32 * k;
+          const int ql = qc * qpc + rr / p.G;
+          const int h = it.g * p.G + rr % p.G;
+          x[k] = ql < it.ti.n ? __ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) : 0.f;
+        }
+      };
+      float lse_nx[4];
+      load_lse(0, lse_nx);
       for (int qc = 0; qc < it.nchunks && ok; ++qc) {
         const int s = qctr % kQStages;
+        float lse_cur[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) lse_cur[k] = lse_nx[k];
+        if (qc + 1 < it.nchunks) load_lse(qc + 1, lse_nx);
         int okw = 1;
         if (lane == 0) okw = mbar_wait(&c.q_empty[s], ((qctr / kQStages) & 1) ^ 1, abort_flag, p.wc, 102, (wi << 12) | qc);
         okw = __shfl_sync(0xffffffffu, okw, 0);
         if (!okw) { ok = false; break; }
-        // augmentation of the chunk's 128 rows (row = query * G + head-in-group):
-        // [hi, lo] = -lse2 / c as a bf16 pair; rows past the tile get a huge
-        // negative hi so they never win a maximum
-        const int qpc = 128 / p.G;
-        const float inv_c = 1.f / p.scale_log2;
-        for (int rr = lane; rr < 128; rr += 32) {
+        // augmentation of the chunk's 128 rows: [hi, lo] = -lse2 / c as a bf16
+        // pair; rows past the tile get a huge negative hi so they never win a maximum
+        uint8_t* qa = smem + L::kOffQa + s * L::kAug;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int rr = lane + 32 * k;
           const int ql = qc * qpc + rr / p.G;
-          const int h = it.g * p.G + rr % p.G;
           uint32_t hl = pack_bf16(-3.0e38f, 0.f);
           if (ql < it.ti.n) {
-            const float x = -(__ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) * 1.4426950408889634f) * inv_c;
+            const float x = -(lse_cur[k] * 1.4426950408889634f) * inv_c;
             const float hi = __bfloat162float(__float2bfloat16_rn(x));
             hl = pack_bf16(hi, x - hi);
           }
-          uint8_t* qa = smem + L::kOffQa + s * L::kAug;
           *reinterpret_cast<uint4*>(qa + aug_off(rr, 0)) = make_uint4(hl, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(qa + aug_off(rr, 1)) = make_uint4(0u, 0u, 0u, 0u);
         }

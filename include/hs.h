@@ -198,6 +198,44 @@ HS_API hs_status hs_sparse_attn_prefill(const hs_varlen* vl, const hs_sel* sel,
                                  void* ws, size_t ws_bytes, hs_stream_t stream);
 
 /*
+ * hs_gather_selected_kv -- token-level selection (sel->block = 1): copy the
+ * selected tokens' K and V rows of every (selection tile, KV head) into
+ * contiguous buffers, once per hybrid block. All sparse layers of a block
+ * reuse the full layer's cache and its selected tokens (KV Reuse: QbitAI
+ * repost; HySparse2 release note), so the gather is paid once and every
+ * sparse prefill layer then reads whole 128-slot tiles
+ * (hs_sparse_attn_prefill_gathered).
+ *   kg[tile][g][s] = k[cu_kv[b(tile)] + idx[tile][g][s]][g]   for s < cnt[tile][g]
+ *   kg[tile][g][s] = 0                                          for cnt <= s < topk
+ * and the same for vg from v (b(tile): the tile's sequence).
+ * In: k/v [T_kv, H_kv, d] bf16; idx/cnt from hs_topk_select for the same
+ * (vl, sel). Out: kg/vg [n_tiles, H_kv, topk, d] bf16, n_tiles = sum over
+ * sequences of ceil(n_b / q_tile) (device, caller-owned, 16-byte aligned, not
+ * overlapping the inputs). topk = 0 or T_q = 0 is a no-op; block != 1, null or
+ * misaligned pointers are HS_ERR_INVALID_ARG.
+ */
+HS_API hs_status hs_gather_selected_kv(const hs_varlen* vl, const hs_sel* sel,
+                                const void* k, const void* v,
+                                const int32_t* idx, const int32_t* cnt,
+                                void* kg, void* vg, hs_stream_t stream);
+
+/*
+ * hs_sparse_attn_prefill_gathered -- hs_sparse_attn_prefill for token-level
+ * selection (sel->block = 1) reading the selected tokens from kg/vg, filled
+ * by hs_gather_selected_kv for the same (vl, sel, idx, cnt); k and v are still
+ * read for the forced window and idx for the visibility mask. Same V_q, same
+ * arithmetic in the same order as hs_sparse_attn_prefill, so o and lse are
+ * identical. Argument rules as hs_sparse_attn_prefill, plus kg/vg non-null
+ * and 16-byte aligned.
+ */
+HS_API hs_status hs_sparse_attn_prefill_gathered(const hs_varlen* vl, const hs_sel* sel,
+                                 const void* q, const void* k, const void* v,
+                                 const void* kg, const void* vg,
+                                 const int32_t* idx, const int32_t* cnt,
+                                 void* o, float* lse,
+                                 void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
  * hs_sparse_attn_decode -- sparse layer for one new token per sequence.
  *
  * Same set V_q as the prefill call with T = 1, computed split-K over the

@@ -100,6 +100,20 @@ def test_host_validation_errors(lib):
     assert lib.hs_kv_dequantize(None, 16, 4, 128, 16, None) == L.HS_ERR_INVALID_ARG
     assert lib.hs_kv_dequantize(16, 18, 4, 128, 16, None) == L.HS_ERR_INVALID_ARG  # misaligned scale
     assert lib.hs_kv_dequantize(16, 16, -1, 128, 16, None) == L.HS_ERR_INVALID_ARG
+    # rows gathered once per block: token level only; topk = 0 is a no-op; null
+    # or misaligned buffers are rejected before launch, also by the layer reading them
+    tok = L.HsSel(16, 1, 8, 32)
+    gath = lambda s_, kg, vg: lib.hs_gather_selected_kv(ctypes.byref(vl), ctypes.byref(s_), 16, 16, 16, 16, kg, vg,
+                                                        None)
+    assert gath(sel, 16, 16) == L.HS_ERR_INVALID_ARG       # block 16
+    assert gath(tok, None, 16) == L.HS_ERR_INVALID_ARG
+    assert gath(tok, 16, 24) == L.HS_ERR_INVALID_ARG       # misaligned
+    assert gath(L.HsSel(16, 1, 0, 32), None, None) == L.HS_OK
+    layer = lambda s_, kg: lib.hs_sparse_attn_prefill_gathered(ctypes.byref(vl), ctypes.byref(s_), 16, 16, 16, kg,
+                                                               16, 16, 16, 16, 16, 16, 1 << 20, None)
+    assert layer(sel, 16) == L.HS_ERR_INVALID_ARG          # block 16
+    assert layer(tok, None) == L.HS_ERR_INVALID_ARG
+    assert layer(tok, 40) == L.HS_ERR_INVALID_ARG          # misaligned
     # unknown selection flags are rejected
     bad = L.HsSel(16, 16, 8, 32, 2)
     assert _call_full(lib, vl, bad) == L.HS_ERR_INVALID_ARG

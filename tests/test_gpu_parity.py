@@ -223,6 +223,46 @@ def test_fp8_kv_prefill_full_size_sampled_tiles():
     run_and_check(w, tile_ids=[0, n_t // 2, n_t - 1], fp8=True)
 
 
+@pytest.mark.parametrize("name", ["tok_mqa32", "tok_gqa4_d64", "tok_exclusive"])
+def test_gathered_rows_and_layer_match_the_per_tile_gather(name):
+    """Token level: hs_gather_selected_kv copies exactly the selected rows of
+    every (tile, KV head), zero past cnt (against a host gather), and the
+    sparse layer reading them equals the layer that gathers each tile with
+    tile::gather4, bit for bit (o and lse). The block runner uses the gathered
+    layer, so the oracle checks of the token-level variants cover it."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    w = VARIANTS[name]
+    inp = W.make_block_inputs(w, device="cuda", seed=13)
+    blk = GpuBlock(w, inp)
+    res = blk.run()
+    idx, cnt = res["idx"], res["cnt"]
+    kg, vg = hs.gather_selected_kv(blk.vl, blk.sel, inp.k, inp.v, idx, cnt)
+    L0 = inp.layers[0]
+    o_a, lse_a = hs.sparse_attn_prefill(blk.vl, blk.sel, L0.q, inp.k, inp.v, idx, cnt)
+    o_b, lse_b = hs.sparse_attn_prefill(blk.vl, blk.sel, L0.q, inp.k, inp.v, idx, cnt, kg=kg, vg=vg)
+    torch.cuda.synchronize()
+    assert torch.equal(o_a.view(torch.int16), o_b.view(torch.int16))
+    assert torch.equal(lse_a.view(torch.int32), lse_b.view(torch.int32))
+    # host gather of the selected rows
+    cu_q, cu_kv, T = w.cu_q(), w.cu_kv(), w.q_tile
+    k_h, v_h, idx_h, cnt_h = inp.k.cpu(), inp.v.cpu(), idx.cpu(), cnt.cpu()
+    kg_ref = torch.zeros(tuple(kg.shape), dtype=torch.bfloat16)
+    vg_ref = torch.zeros(tuple(vg.shape), dtype=torch.bfloat16)
+    tile = 0
+    for b in range(len(cu_q) - 1):
+        n_b = cu_q[b + 1] - cu_q[b]
+        for _ in range((n_b + T - 1) // T):
+            for g in range(w.n_kv_heads):
+                c = int(cnt_h[tile, g])
+                rows = cu_kv[b] + idx_h[tile, g, :c].long()
+                kg_ref[tile, g, :c] = k_h[rows, g]
+                vg_ref[tile, g, :c] = v_h[rows, g]
+            tile += 1
+    assert tile == kg.shape[0]
+    assert torch.equal(kg.cpu().view(torch.int16), kg_ref.view(torch.int16))
+    assert torch.equal(vg.cpu().view(torch.int16), vg_ref.view(torch.int16))
+
+
 def test_swa_gate_two_call_path():
     """The unfused layer (hs_sparse_attn_prefill then hs_swa_gated) against the oracle."""
     run_and_check(VARIANTS["swa_gate"], seed=7, fused=False)
