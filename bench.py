@@ -264,7 +264,10 @@ def make_runner(w_r, inp, device):
     vl = hs.Varlen(w_r.cu_q(), w_r.cu_kv(), w_r.n_q_heads, w_r.n_kv_heads, w_r.head_dim, device=device)
     blk = HybridBlock(vl, w_r.q_tile, w_r.block, w_r.topk, w_r.window, w_r.swa_window, device=device,
                       exclusive=w_r.exclusive)
-    layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
+    if blk.decode and w_r.swa_window > 0:  # decode reads each layer's own window cache as a ring
+        layers = [SparseLayerIn(L.q, *blk.swa_rings(L.k_swa, L.v_swa), L.gamma) for L in inp.layers]
+    else:
+        layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
     return vl, blk, layers
 
 
@@ -361,7 +364,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     import hybrid_sparse_attention_tma_b200 as hs
     from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
                                                   sparse_attn_decode, sparse_swa_gated_prefill,
-                                                  gather_selected_kv, HS_KV_BF16, HS_KV_FP8_E4M3)
+                                                  gather_selected_kv, swa_gated_decode, HS_KV_BF16,
+                                                  HS_KV_FP8_E4M3)
     device = f"cuda:{local}"
     torch.cuda.set_device(local)
     w = workload(args) if w is None else w
@@ -392,7 +396,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     hs.check_error(blk.ws)
     recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"]) if world == 1 else None
 
-    kinds = ["full", "topk", "sparse"] + (["gather"] if blk.gathered else [])
+    swa_dec = blk.decode and blk.swa_window > 0
+    kinds = ["full", "topk", "sparse"] + (["gather"] if blk.gathered else []) + (["swa"] if swa_dec else [])
     L0 = layers[0]
 
     def call(kind, st):
@@ -403,6 +408,9 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
                              ws=blk.ws, stream=st)
         elif kind == "topk":
             topk_select(vl, sel, bufs["scores"], bufs["idx"], bufs["cnt"], ws=blk.ws, stream=st)
+        elif kind == "swa":
+            swa_gated_decode(vl, blk.swa_window, L0.q, L0.k_swa, L0.v_swa, L0.gamma, bufs["o_sp0"], bufs["o_l0"],
+                             stream=st)
         elif kind == "gather":
             gather_selected_kv(vl, sel, inp.k, inp.v, bufs["idx"], bufs["cnt"], bufs["kg"], bufs["vg"], stream=st)
         elif blk.decode:
@@ -537,7 +545,11 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
         # distinct selected rows read once (the rest of the reads hit L2)
         uniq = distinct_selected_rows(w, blk._bufs["idx"], blk._bufs["cnt"])
         entry("gather", kms["gather"], (n_tiles * hkv * w.topk + uniq) * d * 2 * 2, "hbm")
-    per_step = {"full": 1, "topk": 1, "sparse": len(layers), "gather": 1}
+    if swa_dec:
+        # the window rows of K and V read from the rings, q, o_sparse and o
+        win = sum(min(w.swa_window, kb - ka) for ka, kb in zip(w.cu_kv()[:-1], w.cu_kv()[1:]))
+        entry("swa", kms["swa"], win * hkv * d * 2 * 2 + 3 * q_bytes, "hbm")
+    per_step = {"full": 1, "topk": 1, "sparse": len(layers), "gather": 1, "swa": len(layers)}
     for kd, e in kernels.items():
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])
@@ -578,7 +590,8 @@ def shard_kind(w, world):
             "q_tiles": "selection tiles per rank + K/V all-gather"}[sh[0].kind]
 
 
-EXTRA = [("hys_block", False), ("hys2_prefill", False), ("decode", False), ("decode", True), ("tiny", False)]
+EXTRA = [("hys_block", False), ("hys2_prefill", False), ("decode", False), ("decode", True), ("decode_swa", False),
+         ("tiny", False)]
 
 
 def bench_extra(args, world, rank, local, headline):

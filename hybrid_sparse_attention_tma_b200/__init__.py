@@ -18,6 +18,7 @@ from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
 
 __all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
            "gather_selected_kv", "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "kv_dequantize",
+           "swa_ring_write", "swa_gated_decode",
            "workspace_size", "check_error", "HsError"]
 
 
@@ -223,6 +224,26 @@ def kv_dequantize(codes, scale, out=None, stream=None):
     out = torch.empty((T, H, d), dtype=torch.bfloat16, device=codes.device) if out is None else out
     L.check("hs_kv_dequantize", lib.hs_kv_dequantize(_ptr(codes), _ptr(scale), T * H, d, _ptr(out), _stream(stream)))
     return out
+
+
+def swa_ring_write(vl: Varlen, k_new, v_new, k_ring, v_ring, stream=None):
+    """Store the new tokens' rows [T_q, H_kv, d] of a layer's own SWA cache in
+    its rings [batch, R, H_kv, d] (position p at slot p mod R)."""
+    lib = L.load()
+    L.check("hs_swa_ring_write", lib.hs_swa_ring_write(
+        ctypes.byref(vl.c), k_ring.shape[1], _ptr(k_new), _ptr(v_new), _ptr(k_ring), _ptr(v_ring), _stream(stream)))
+    return k_ring, v_ring
+
+
+def swa_gated_decode(vl: Varlen, window: int, q, k_ring, v_ring, gamma, o_sparse, o=None, stream=None):
+    """Decode: the own-cache sliding-window branch over the rings and the
+    sigmoid gate with the sparse branch. Returns o."""
+    lib = L.load()
+    o = torch.empty_like(q) if o is None else o
+    L.check("hs_swa_gated_decode", lib.hs_swa_gated_decode(
+        ctypes.byref(vl.c), window, k_ring.shape[1], _ptr(q), _ptr(k_ring), _ptr(v_ring), _ptr(gamma),
+        _ptr(o_sparse), _ptr(o), _stream(stream)))
+    return o
 
 
 def swa_gated(vl: Varlen, window: int, q, k_swa, v_swa, gamma, o_sparse, o=None,

@@ -18,7 +18,7 @@ EXPORTS = [
     "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
     "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
     "hs_full_attn_select_noalloc", "hs_sparse_swa_gated_prefill", "hs_debug_exp2_poly", "hs_kv_dequantize",
-    "hs_gather_selected_kv", "hs_sparse_attn_prefill_gathered",
+    "hs_gather_selected_kv", "hs_sparse_attn_prefill_gathered", "hs_swa_ring_write", "hs_swa_gated_decode",
 ]
 
 
@@ -75,6 +75,10 @@ def load():
     lib.hs_sparse_attn_prefill.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hs_gather_selected_kv.restype = i32
     lib.hs_gather_selected_kv.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, vp]
+    lib.hs_swa_ring_write.restype = i32
+    lib.hs_swa_ring_write.argtypes = [VL, i32, vp, vp, vp, vp, vp]
+    lib.hs_swa_gated_decode.restype = i32
+    lib.hs_swa_gated_decode.argtypes = [VL, i32, i32, vp, vp, vp, vp, vp, vp, vp]
     lib.hs_sparse_attn_prefill_gathered.restype = i32
     lib.hs_sparse_attn_prefill_gathered.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hs_sparse_attn_decode.restype = i32

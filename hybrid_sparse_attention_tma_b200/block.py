@@ -13,13 +13,15 @@ from typing import List, Optional
 import torch
 
 from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
-               swa_gated, sparse_swa_gated_prefill, kv_dequantize, gather_selected_kv, HS_KV_BF16, HS_KV_FP8_E4M3)
+               swa_gated, sparse_swa_gated_prefill, kv_dequantize, gather_selected_kv, swa_gated_decode,
+               swa_ring_write, HS_KV_BF16, HS_KV_FP8_E4M3)
 
 
 @dataclass
 class SparseLayerIn:
     q: torch.Tensor                       # [T_q, H_q, d] bf16, this layer's queries
-    k_swa: Optional[torch.Tensor] = None  # [T_kv, H_kv, d] bf16, own SWA cache (HySparse)
+    k_swa: Optional[torch.Tensor] = None  # own SWA cache (HySparse): prefill [T_kv, H_kv, d] bf16;
+    #   decode: the ring [batch, R, H_kv, d] (hs_swa_ring_write), R >= the window
     v_swa: Optional[torch.Tensor] = None
     gamma: Optional[torch.Tensor] = None  # [T_q, H_q] fp32 gate logits
 
@@ -36,13 +38,26 @@ class HybridBlock:
         self.ws = Workspace(device)
         self.device = device
         self._bufs = {}
-        # one query per sequence with single-token tiles: the sparse layers use
-        # the split-K decode path
-        self.decode = q_tile == 1 and block == 1 and all(
-            b - a == 1 for a, b in zip(vl.cu_q_list, vl.cu_q_list[1:]))
+        # one query per sequence with single-query tiles: the sparse layers use
+        # the decode path (token- or block-level selection; a window branch
+        # reads the layer's own cache as a ring)
+        self.decode = q_tile == 1 and all(b - a == 1 for a, b in zip(vl.cu_q_list, vl.cu_q_list[1:]))
         # token-level prefill: the selected rows are gathered once per block
         # (hs_gather_selected_kv) and every plain sparse layer reads them
         self.gathered = (not self.decode and block == 1 and topk > 0 and not (swa_window > 0 and fused))
+
+    def swa_rings(self, k_swa, v_swa, stream=None):
+        """Decode: a layer's own window cache [T_kv, H_kv, d] (all positions, in
+        cu_kv order) as the rings [batch, swa_window, H_kv, d] the decode path
+        reads (hs_swa_ring_write with every cached token new: the last
+        swa_window positions of each sequence land at slot p mod swa_window)."""
+        vl = self.vl
+        every = Varlen(vl.cu_kv_list, vl.cu_kv_list, vl.n_q_heads, vl.n_kv_heads, vl.head_dim, device=self.device)
+        shape = (vl.batch, self.swa_window, vl.n_kv_heads, vl.head_dim)
+        kr = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
+        vr = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
+        swa_ring_write(every, k_swa, v_swa, kr, vr, stream=stream)
+        return kr, vr
 
     def _buf(self, name, shape, dtype):
         t = self._bufs.get(name)
@@ -108,7 +123,10 @@ class HybridBlock:
             else:
                 sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream,
                                     kg=kg, vg=vg)
-            if self.swa_window > 0:
+            if self.swa_window > 0 and self.decode:
+                o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
+                swa_gated_decode(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, stream=stream)
+            elif self.swa_window > 0:
                 o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
                 swa_gated(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, ws=self.ws,
                           stream=stream)

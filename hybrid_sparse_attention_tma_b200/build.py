@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhs.so")
 SOURCES = ["api.cu"]
 HEADERS = ["hs_common.cuh", "attn_fwd.cuh", "topk.cuh", "seqtable.cuh", "token_scores.cuh",
-           "decode_tc.cuh"]
+           "decode_tc.cuh", "swa_decode.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [

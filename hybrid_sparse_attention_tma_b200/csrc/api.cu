@@ -14,6 +14,7 @@
 #include "hs_common.cuh"
 #include "seqtable.cuh"
 #include "decode_tc.cuh"
+#include "swa_decode.cuh"
 #include "token_scores.cuh"
 #include "topk.cuh"
 
@@ -291,6 +292,15 @@ bool is_decode(const hs_varlen* vl, const hs_sel* sel) {
   return true;
 }
 
+// One query per sequence and single-query tiles, any selection block (the
+// sparse decode; the token-level full-layer decode kernel needs block 1).
+bool is_decode_batch(const hs_varlen* vl, const hs_sel* sel) {
+  if (sel->q_tile != 1) return false;
+  for (int b = 0; b < vl->batch; ++b)
+    if (vl->cu_q_host[b + 1] - vl->cu_q_host[b] != 1) return false;
+  return true;
+}
+
 // Full-layer decode on the tensor cores (decode_tc.cuh): keys per work item.
 // Pass 2 re-reads a unit's K about D = (one unit's chunks + two grids of
 // items) pass-1 items after pass 1 read it. Each item costs a few
@@ -356,7 +366,7 @@ SparseDecodePlan sparse_decode_plan(const Shape& sh, const hs_sel* sel, int spli
   SparseDecodePlan pl;
   const int U = sh.batch * sh.Hkv;
   // ranges of equal slot counts (not whole tiles): the ranges of a unit finish together
-  pl.unit_tiles = std::max(1, (sel->topk + sel->window + 127) / 128);
+  pl.unit_tiles = std::max(1, (sel->topk * sel->block + sel->window + 127) / 128);
   int want = split_k > 0 ? split_k : std::max(1, num_sms() / std::max(1, U));
   want = std::min({want, pl.unit_tiles, dtc::sdec::kMaxSplit});
   pl.tiles_per_split = (pl.unit_tiles + want - 1) / want;
@@ -480,6 +490,23 @@ hs_status noalloc_scratch(void** out) {
 }  // namespace
 
 // ============================================================================
+template <int D>
+hs_status launch_swa_gated_decode(const hs_varlen* vl, const Shape& sh, int window, int ring_len,
+                                         const void* q, const void* k_ring, const void* v_ring, const float* gamma,
+                                         const void* o_sparse, void* o, cudaStream_t s) {
+  const int smem = 4 * swad::smem_words<D>(sh.G, window);
+  static PerDeviceOnce once;
+  if (set_smem_once(once, swad::swa_gated_decode_kernel<D>, 4 * swad::smem_words<D>(swad::kMaxG, swad::kMaxWindow)) !=
+      cudaSuccess)
+    return HS_ERR_CUDA;
+  swad::swa_gated_decode_kernel<D><<<vl->batch * sh.Hkv, swad::kThreads, smem, s>>>(
+      vl->cu_q, vl->cu_kv, sh.Hq, sh.Hkv, sh.G, window, ring_len, sh.scale * 1.4426950408889634f,
+      reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(k_ring),
+      reinterpret_cast<const __nv_bfloat16*>(v_ring), gamma, reinterpret_cast<const __nv_bfloat16*>(o_sparse),
+      reinterpret_cast<__nv_bfloat16*>(o));
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
 extern "C" {
 
 const char* hs_status_string(hs_status s) {
@@ -888,7 +915,7 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   if (st != HS_OK) return st;
   if ((st = check_sel(sel)) != HS_OK) return st;
   if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
-  if (!is_decode(vl, sel)) return HS_ERR_INVALID_ARG;  // one query per sequence, q_tile = block = 1
+  if (!is_decode_batch(vl, sel)) return HS_ERR_INVALID_ARG;  // one query per sequence, q_tile = 1
   if (sh.d != 128 || sh.G > 64) return HS_ERR_UNSUPPORTED;
   if (kv_dtype != HS_KV_BF16 && kv_dtype != HS_KV_FP8_E4M3) return HS_ERR_INVALID_ARG;
   const bool fp8 = kv_dtype == HS_KV_FP8_E4M3;
@@ -912,6 +939,7 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
   p.v_scale = v_scale;
   p.topk = sel->topk;
   p.w = sel->window;
+  p.log2_block = __builtin_ctz(unsigned(sel->block));  // a power of two (check_sel)
   p.G = sh.G;
   p.Hq = sh.Hq;
   p.Hkv = sh.Hkv;
@@ -957,6 +985,45 @@ hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel, const vo
     e = cudaLaunchKernelEx(&cfg, dtc::sdec::sparse_decode_tc_kernel<false>, map_q, p);
   }
   return e == cudaSuccess && cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_swa_ring_write(const hs_varlen* vl, int32_t ring_len, const void* k_new, const void* v_new,
+                            void* k_ring, void* v_ring, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if (ring_len < 1) return HS_ERR_INVALID_ARG;
+  if (sh.Tq == 0) return HS_OK;
+  if (!k_new || !v_new || !k_ring || !v_ring || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_ring) ||
+      !aligned16(v_ring))
+    return HS_ERR_INVALID_ARG;
+  const int row_pieces = sh.Hkv * sh.d / 8;
+  const long long n = sh.Tq * row_pieces;
+  const int grid = int(std::min<long long>(8LL * num_sms(), (n + 255) / 256));
+  swad::ring_write_kernel<<<grid, 256, 0, S(stream)>>>(
+      vl->cu_q, vl->cu_kv, vl->batch, sh.Tq, row_pieces, ring_len, reinterpret_cast<const uint4*>(k_new),
+      reinterpret_cast<const uint4*>(v_new), reinterpret_cast<uint4*>(k_ring), reinterpret_cast<uint4*>(v_ring));
+  return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+hs_status hs_swa_gated_decode(const hs_varlen* vl, int32_t window, int32_t ring_len, const void* q,
+                              const void* k_ring, const void* v_ring, const float* gamma, const void* o_sparse,
+                              void* o, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if (window < 1 || ring_len < window) return HS_ERR_INVALID_ARG;
+  if (sh.Tq == 0) return HS_OK;
+  for (int b = 0; b < vl->batch; ++b)  // one new token per sequence, which sees itself
+    if (vl->cu_q_host[b + 1] - vl->cu_q_host[b] != 1 || vl->cu_kv_host[b + 1] - vl->cu_kv_host[b] < 1)
+      return HS_ERR_INVALID_ARG;
+  if (window > swad::kMaxWindow || sh.G > swad::kMaxG) return HS_ERR_UNSUPPORTED;
+  if (!q || !k_ring || !v_ring || !gamma || !o_sparse || !o || !aligned16(k_ring) || !aligned16(v_ring) ||
+      (reinterpret_cast<uintptr_t>(gamma) & 3) || (reinterpret_cast<uintptr_t>(q) & 3) ||
+      (reinterpret_cast<uintptr_t>(o) & 3) || (reinterpret_cast<uintptr_t>(o_sparse) & 3))
+    return HS_ERR_INVALID_ARG;
+  if (sh.d == 64) return launch_swa_gated_decode<64>(vl, sh, window, ring_len, q, k_ring, v_ring, gamma, o_sparse, o, S(stream));
+  return launch_swa_gated_decode<128>(vl, sh, window, ring_len, q, k_ring, v_ring, gamma, o_sparse, o, S(stream));
 }
 
 hs_status hs_swa_gated(const hs_varlen* vl, int32_t window, const void* q, const void* k_swa, const void* v_swa,

@@ -800,6 +800,7 @@ struct Params {
   const float* k_scale;  // [T_kv, Hkv]
   const float* v_scale;
   int topk, w, G, Hq, Hkv, Tq;
+  int log2_block;  // selected blocks of 2^log2_block keys (0: token level)
   int n_units, nsplit, tiles_per_split, unit_tiles, n_items;
   float scale_log2;
   __nv_bfloat16* o;
@@ -837,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // for L2 while the CTA sets up (kBatch tiles = 32 lanes x 128 bytes)
   if (warp == 4 && int(blockIdx.x) < p.n_items) {
     const int u = blockIdx.x / p.nsplit;
-    const int j0 = (blockIdx.x % p.nsplit) * p.tiles_per_split * 128 - p.w + lane * 32;
+    const int j0 = ((blockIdx.x % p.nsplit) * p.tiles_per_split * 128 - p.w + lane * 32) >> p.log2_block;
     if (lane == 0) {
       prefetch_l2(p.cu_kv + u / p.Hkv);
       if (p.cnt) prefetch_l2(p.cnt + u);
@@ -911,9 +912,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int bi = 0; bi < kBatch; ++bi)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
+            // selected part: slot w + j holds key idx[j >> log2 B] * B + (j mod B)
             const int jsel = (t0 + tb + bi) * 128 + lane * 4 + e - p.w;
-            key[bi][e] = (p.cnt && tb + bi < n && jsel >= 0 && jsel < p.topk)
-                             ? __ldg(p.idx + size_t(u) * p.topk + jsel) : -1;
+            const int jb = jsel >> p.log2_block;
+            key[bi][e] = (p.cnt && tb + bi < n && jsel >= 0 && jb < p.topk)
+                             ? (__ldg(p.idx + size_t(u) * p.topk + jb) << p.log2_block) +
+                                   (jsel & ((1 << p.log2_block) - 1))
+                             : -1;
           }
         const int pos = kv1 - kv0 - 1;
         const int win_lo = max(0, pos - p.w + 1);
@@ -925,7 +930,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int slot = (t0 + tb + bi) * 128 + lane * 4 + e;
             const int jsel = slot - p.w;
             if (slot < n_win) key[bi][e] = win_lo + slot;
-            else if (jsel < 0 || jsel >= cnt || key[bi][e] > pos - p.w) key[bi][e] = -1;
+            else if (jsel < 0 || (jsel >> p.log2_block) >= cnt || key[bi][e] > pos - p.w) key[bi][e] = -1;
           }
 #pragma unroll
         for (int bi = 0; bi < kBatch; ++bi) {

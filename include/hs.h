@@ -243,8 +243,10 @@ HS_API hs_status hs_sparse_attn_prefill_gathered(const hs_varlen* vl, const hs_s
  * FP8 e4m3 (the HySparse2 key-data table sizes an FP8 KV cache); FP8 values
  * decode as x = scale[token, kv_head] * e4m3(code), with separate fp32 scale
  * arrays for K and V ([T_kv, H_kv]; NULL for bf16).
- * The slots of each (sequence, KV head) -- the window, then the selected
- * tokens -- form ceil((k + w) / 128) tiles of 128 keys, cut into split_k
+ * The slots of each (sequence, KV head) -- the window, then the tokens of
+ * the selected blocks (block B = sel->block: token-level selection with B = 1;
+ * HySparse's 64-token blocks with B = 64) -- form ceil((k B + w) / 128) tiles
+ * of 128 keys, cut into split_k
  * contiguous ranges of whole tiles, one tensor-core work item each; the
  * ranges of a unit run as one thread-block cluster and their partial results
  * are merged by log-sum-exp through the cluster's shared memory, inside the
@@ -253,7 +255,7 @@ HS_API hs_status hs_sparse_attn_prefill_gathered(const hs_varlen* vl, const hs_s
  * above the tile count or above 8 (the portable cluster size) is clamped;
  * negative values are rejected.
  * An empty batch (T_q = 0) returns HS_OK without touching any pointer.
- * Requires n_b = 1 for every sequence and sel->q_tile = 1.
+ * Requires n_b = 1 for every sequence and sel->q_tile = 1 (any block).
  */
 HS_API hs_status hs_sparse_attn_decode(const hs_varlen* vl, const hs_sel* sel,
                                 const void* q, hs_kv_dtype kv_dtype,
@@ -321,6 +323,41 @@ HS_API hs_status hs_sparse_swa_gated_prefill(const hs_varlen* vl, const hs_sel* 
  * multiple of 16; pointers 16-byte aligned (scale 4-byte). rows = 0 is a
  * no-op; negative sizes, null or misaligned pointers are HS_ERR_INVALID_ARG.
  */
+/*
+ * hs_swa_ring_write -- keep a layer's own sliding-window K/V cache as a ring
+ * buffer (the SWA branch of HySparse reads only the last `window` positions
+ * of its own small cache: QbitAI repost, two-branch paragraph; techwalker.com
+ * explainer, the window branch must not share the full layer's KV).
+ *   k_ring[b][p mod R][g] = k_new[row of the new token of sequence b at position p][g]
+ * for the new tokens of each sequence (positions kv_b - n_b .. kv_b - 1) that
+ * are among its last R positions; the same for v. R = ring_len >= the window.
+ * In: k_new / v_new [T_q, H_kv, d] bf16 (rows in cu_q order). Out (device,
+ * caller-owned, updated in place): k_ring / v_ring [batch, R, H_kv, d] bf16.
+ * Pointers 16-byte aligned. T_q = 0 is a no-op; ring_len < 1, null or
+ * misaligned pointers are HS_ERR_INVALID_ARG.
+ */
+HS_API hs_status hs_swa_ring_write(const hs_varlen* vl, int32_t ring_len,
+                                   const void* k_new, const void* v_new,
+                                   void* k_ring, void* v_ring, hs_stream_t stream);
+
+/*
+ * hs_swa_gated_decode -- the HySparse sliding-window branch and its gate for
+ * one new token per sequence, over the layer's own K/V in a ring (written by
+ * hs_swa_ring_write, the new token's row included):
+ *   o_swa[b, h] = sum_{p = max(0, pos - window + 1)}^{pos} softmax_p(s) v_ring[b][p mod R][g(h)]
+ *   o[b, h]     = sig(gamma[b, h]) o_sparse[b, h] + (1 - sig(gamma[b, h])) o_swa[b, h]
+ * with pos = kv_b - 1 and the same scale as the other calls (the gate as in
+ * hs_swa_gated). In: q [batch, H_q, d] bf16, gamma [batch, H_q] fp32,
+ * o_sparse [batch, H_q, d] bf16 (the sparse decode layer's output). Out: o
+ * [batch, H_q, d] bf16. Requires one new token per sequence (kv_b >= 1),
+ * 1 <= window <= ring_len; window <= 128 and G <= 64 (else
+ * HS_ERR_UNSUPPORTED). Null or misaligned pointers are HS_ERR_INVALID_ARG.
+ */
+HS_API hs_status hs_swa_gated_decode(const hs_varlen* vl, int32_t window, int32_t ring_len,
+                                     const void* q, const void* k_ring, const void* v_ring,
+                                     const float* gamma, const void* o_sparse, void* o,
+                                     hs_stream_t stream);
+
 HS_API hs_status hs_kv_dequantize(const void* codes, const float* scale, int64_t rows, int32_t head_dim,
                                   void* out, hs_stream_t stream);
 

@@ -104,7 +104,11 @@ class GpuBlock:
         self.sel = hs.Sel(w.q_tile, w.block, w.topk, w.window, w.exclusive)
         self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device,
                                  fused=fused, exclusive=w.exclusive)
-        self.layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
+        if self.block.decode and w.swa_window > 0:
+            # decode reads each layer's own window cache as a ring of swa_window slots
+            self.layers = [SparseLayerIn(L.q, *self.block.swa_rings(L.k_swa, L.v_swa), L.gamma) for L in inp.layers]
+        else:
+            self.layers = [SparseLayerIn(L.q, L.k_swa, L.v_swa, L.gamma) for L in inp.layers]
 
     def run(self, stream=None, fp8=False, intermediates=True):
         fp8_kv = None

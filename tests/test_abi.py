@@ -114,6 +114,19 @@ def test_host_validation_errors(lib):
     assert layer(sel, 16) == L.HS_ERR_INVALID_ARG          # block 16
     assert layer(tok, None) == L.HS_ERR_INVALID_ARG
     assert layer(tok, 40) == L.HS_ERR_INVALID_ARG          # misaligned
+    # SWA ring: ring length >= 1, pointers 16-byte aligned; the decode branch needs
+    # one new token per sequence and 1 <= window <= ring length (window <= 128)
+    assert lib.hs_swa_ring_write(ctypes.byref(vl), 0, 16, 16, 16, 16, None) == L.HS_ERR_INVALID_ARG
+    assert lib.hs_swa_ring_write(ctypes.byref(vl), 8, 16, 24, 16, 16, None) == L.HS_ERR_INVALID_ARG
+    dec = _varlen([0, 1, 2], [0, 300, 600])
+    swad = lambda vl_, win, ring, gam: lib.hs_swa_gated_decode(ctypes.byref(vl_), win, ring, 16, 16, 16, gam, 16,
+                                                                16, None)
+    assert swad(vl, 128, 128, 16) == L.HS_ERR_INVALID_ARG       # 512 new tokens in one sequence
+    assert swad(dec, 0, 128, 16) == L.HS_ERR_INVALID_ARG
+    assert swad(dec, 128, 64, 16) == L.HS_ERR_INVALID_ARG       # ring shorter than the window
+    assert swad(dec, 256, 256, 16) == L.HS_ERR_UNSUPPORTED
+    assert swad(dec, 128, 128, None) == L.HS_ERR_INVALID_ARG
+    assert swad(dec, 128, 128, 18) == L.HS_ERR_INVALID_ARG      # misaligned gate
     # unknown selection flags are rejected
     bad = L.HsSel(16, 16, 8, 32, 2)
     assert _call_full(lib, vl, bad) == L.HS_ERR_INVALID_ARG

@@ -348,6 +348,14 @@ DECODE = {
     # k = 0: the sparse layer sees only the forced window (one context shorter than the window)
     "dec_window_only": W.Workload("d3", ctx=(200, 45), new=(1, 1), n_q_heads=64, n_kv_heads=1, head_dim=128,
                                   q_tile=1, block=1, topk=0, window=48, n_sparse=1),
+    # HySparse layer shape at decode time: 64-token blocks, top-4, no forced window,
+    # own sliding-window branch over a 128-slot ring + sigmoid gate; ragged
+    # contexts (one shorter than the window, one a multiple of the block)
+    "dec_block_swa": W.Workload("d5", ctx=(300, 1000, 63, 2047), new=(1,) * 4, n_q_heads=16, n_kv_heads=4,
+                                head_dim=128, q_tile=1, block=64, topk=4, window=0, n_sparse=2, swa_window=128),
+    # block-level decode with a forced window (16-token blocks), GQA 4
+    "dec_block_window": W.Workload("d6", ctx=(500, 77), new=(1, 1), n_q_heads=8, n_kv_heads=2, head_dim=128,
+                                   q_tile=1, block=16, topk=6, window=24, n_sparse=1),
 }
 
 

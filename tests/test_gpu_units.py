@@ -73,6 +73,38 @@ def test_topk_exact_ties_bit_exact(name):
         assert row[k - 1] == row[k], "no tie straddles the k-th place"
 
 
+def test_swa_ring_write_keeps_the_last_positions():
+    """hs_swa_ring_write puts the row of position p at slot p mod R and, when a
+    call brings more than R new tokens of a sequence, only the last R land
+    (a prefill that builds the ring, then one decode token appended)."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    R, hkv, d = 8, 2, 128
+    cu_q, cu_kv = [0, 5, 25, 26], [0, 5, 25, 26]          # 5, 20 and 1 new tokens, no cache
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    k = torch.randn((26, hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    v = torch.randn((26, hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    kr = torch.zeros((3, R, hkv, d), dtype=torch.bfloat16, device="cuda")
+    vr = torch.zeros_like(kr)
+    vl = hs.Varlen(cu_q, cu_kv, 4, hkv, d)
+    hs.swa_ring_write(vl, k, v, kr, vr)
+    # one decode token per sequence at positions 5, 20, 1
+    kn = torch.randn((3, hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    vn = torch.randn((3, hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    hs.swa_ring_write(hs.Varlen([0, 1, 2, 3], [0, 6, 27, 29], 4, hkv, d), kn, vn, kr, vr)
+    torch.cuda.synchronize()
+    ref_k = torch.zeros_like(kr).cpu()
+    ref_v = torch.zeros_like(vr).cpu()
+    kh, vh, knh, vnh = k.cpu(), v.cpu(), kn.cpu(), vn.cpu()
+    for b, (a, e) in enumerate(zip(cu_q[:-1], cu_q[1:])):
+        for p in range(max(0, (e - a) - R), e - a):
+            ref_k[b, p % R], ref_v[b, p % R] = kh[a + p], vh[a + p]
+        p = e - a  # the decode token
+        ref_k[b, p % R], ref_v[b, p % R] = knh[b], vnh[b]
+    assert torch.equal(kr.cpu().view(torch.int16), ref_k.view(torch.int16))
+    assert torch.equal(vr.cpu().view(torch.int16), ref_v.view(torch.int16))
+
+
 def test_kv_dequantize_bit_exact():
     """hs_kv_dequantize: bf16_rn(fp32(scale) * fp32(e4m3(code))) for every row,
     bit for bit against the same arithmetic by torch on the host (every code

@@ -122,6 +122,11 @@ WORKLOADS = {
     "decode": Workload("decode", ctx=(131071,) * 64, new=(1,) * 64, n_q_heads=64, n_kv_heads=1,
                        head_dim=128, q_tile=1, block=1, topk=1024, window=128, n_sparse=11,
                        config_index=3),
+    # the HySparse layer shape (C2) at decode time: 64-token blocks, top-16, own
+    # 128-token window kept as a ring + sigmoid gate; 64 sequences x 32k cached tokens
+    "decode_swa": Workload("decode_swa", ctx=(32767,) * 64, new=(1,) * 64, n_q_heads=32, n_kv_heads=8,
+                           head_dim=128, q_tile=1, block=64, topk=16, window=0, n_sparse=3, swa_window=128,
+                           config_index=1),
     "agentic": Workload("agentic", ctx=(262144, 131072, 65536, 16384), new=(8192, 4096, 8192, 2048),
                         n_q_heads=64, n_kv_heads=1, head_dim=128, q_tile=64, block=1, topk=1024,
                         window=128, n_sparse=11, needle_rate=0.005, config_index=4),
