@@ -343,19 +343,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool full = (c_min == 0) && (c_max == 128);
           const uint32_t taddr = tmem + b * 128 + (uint32_t(warp * 32) << 16);
           float m = best[b];  // max over rows of s - lse2 / c
+          // the accumulator's 128 columns in four loads, one wait
+          uint32_t v[4][32];
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) tmem_ld32(taddr + ch * 32, v[ch]);
+          tmem_ld_wait();
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
-            uint32_t v[32];
-            tmem_ld32(taddr + ch * 32, v);
-            tmem_ld_wait();
             if (full) {
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) m = max3f(m, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+              for (int e = 0; e < 32; e += 2) m = max3f(m, __uint_as_float(v[ch][e]), __uint_as_float(v[ch][e + 1]));
             } else {
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
                 const int col = ch * 32 + e;
-                if (col >= c_min && col < c_max) m = fmaxf(m, __uint_as_float(v[e]));
+                if (col >= c_min && col < c_max) m = fmaxf(m, __uint_as_float(v[ch][e]));
               }
             }
           }
