@@ -611,39 +611,23 @@ def bench_extra(args, world, rank, local, headline):
 
 
 def bench_e2e(args, w, inp, vl, blk, layers, device, block_tokens, fp8_kv=None):
-    """Same metric through HybridBlock.forward with the step's inputs copied
-    from pinned host memory each step and the last layer's output read back."""
+    """Same metric through the block runner's public call with the step's
+    inputs in pinned host memory (HybridBlock.forward_from_host: Q, K, V
+    copied first, each sparse layer's inputs streamed in on a copy stream
+    while the earlier layers compute) and the last layer's output read back."""
     from hybrid_sparse_attention_tma_b200.block import SparseLayerIn
-    host = {"q": inp.q.cpu().pin_memory(), "k": inp.k.cpu().pin_memory(), "v": inp.v.cpu().pin_memory()}
-    hl = []
-    for L in inp.layers:
-        d = {"q": L.q.cpu().pin_memory()}
-        if L.k_swa is not None:
-            d.update(k_swa=L.k_swa.cpu().pin_memory(), v_swa=L.v_swa.cpu().pin_memory(),
-                     gamma=L.gamma.cpu().pin_memory())
-        hl.append(d)
-    dev_q, dev_k, dev_v = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
-    dev_layers = [SparseLayerIn(torch.empty_like(L.q),
-                                torch.empty_like(L.k_swa) if L.k_swa is not None else None,
-                                torch.empty_like(L.v_swa) if L.v_swa is not None else None,
-                                torch.empty_like(L.gamma) if L.gamma is not None else None) for L in inp.layers]
+    pin = (lambda t: None if t is None else t.cpu().pin_memory())
+    host_q, host_k, host_v = pin(inp.q), pin(inp.k), pin(inp.v)
+    hl = [SparseLayerIn(pin(L.q), pin(L.k_swa), pin(L.v_swa), pin(L.gamma)) for L in layers]
     out_host = torch.empty(inp.q.shape, dtype=torch.bfloat16).pin_memory()
     stream = torch.cuda.current_stream()
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    h2d += sum(t.numel() * t.element_size() for d in hl for t in d.values())
+    nbytes = (lambda t: 0 if t is None else t.numel() * t.element_size())
+    h2d = nbytes(host_q) + nbytes(host_k) + nbytes(host_v)
+    h2d += sum(nbytes(getattr(L, f)) for L in hl for f in ("q", "k_swa", "v_swa", "gamma"))
     d2h = out_host.numel() * out_host.element_size()
 
     def step():
-        dev_q.copy_(host["q"], non_blocking=True)
-        dev_k.copy_(host["k"], non_blocking=True)
-        dev_v.copy_(host["v"], non_blocking=True)
-        for dl, d in zip(dev_layers, hl):
-            dl.q.copy_(d["q"], non_blocking=True)
-            if dl.k_swa is not None:
-                dl.k_swa.copy_(d["k_swa"], non_blocking=True)
-                dl.v_swa.copy_(d["v_swa"], non_blocking=True)
-                dl.gamma.copy_(d["gamma"], non_blocking=True)
-        res = blk.forward(dev_q, dev_k, dev_v, dev_layers, stream=stream, fp8_kv=fp8_kv, intermediates=False)
+        res = blk.forward_from_host(host_q, host_k, host_v, hl, stream=stream, fp8_kv=fp8_kv, intermediates=False)
         out_host.copy_(res["layers"][-1]["o"], non_blocking=True)
 
     for _ in range(3):

@@ -67,7 +67,7 @@ class HybridBlock:
         return t
 
     def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False, fp8_kv=None,
-                intermediates: bool = True):
+                intermediates: bool = True, layer_hook=None):
         """Returns dict(o_full, lse_full, scores, idx, cnt, layers=[{o_sparse, lse_sparse, o}]).
 
         With keep_all=False, output buffers are reused across calls (no
@@ -78,7 +78,9 @@ class HybridBlock:
         (hs_kv_dequantize) and the full and sparse layers use the expansion
         (k and v may then be None). With
         intermediates=False a fused layer does not write o_sparse / lse_sparse
-        (they are returned as None)."""
+        (they are returned as None). layer_hook (see forward_from_host) supplies
+        each layer's inputs just before its launches and is told when they are
+        enqueued."""
         vl, sel = self.vl, self.sel
         Tq, Hq, d = q.shape
         nblk = (vl.max_kv + sel.block - 1) // sel.block
@@ -101,6 +103,8 @@ class HybridBlock:
                                         self._buf("vg", gshape, torch.bfloat16), stream=stream)
         outs = []
         for i, L in enumerate(layers):
+            if layer_hook is not None:
+                L = layer_hook.before(i)  # this layer's inputs, once they are on the device
             tag = str(i) if keep_all else str(i % 2)
             o_sp = self._buf("o_sp" + tag, (Tq, Hq, d), torch.bfloat16)
             lse_sp = self._buf("lse_sp" + tag, (Hq, Tq), torch.float32)
@@ -112,18 +116,16 @@ class HybridBlock:
                 else:
                     sparse_attn_decode(vl, sel, L.q, k, v, idx, cnt, kv_dtype=HS_KV_BF16, o=o_sp, lse=lse_sp,
                                        ws=self.ws, stream=stream)
-            elif self.swa_window > 0 and self.fused:
+            elif not (self.swa_window > 0 and self.fused):
+                sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream,
+                                    kg=kg, vg=vg)
+            if self.swa_window > 0 and self.fused and not self.decode:
                 o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
                 if not intermediates:
                     o_sp = lse_sp = None
                 sparse_swa_gated_prefill(vl, sel, L.q, k, v, idx, cnt, self.swa_window, L.k_swa, L.v_swa, L.gamma,
                                          o=o_l, o_sparse=o_sp, lse_sparse=lse_sp, ws=self.ws, stream=stream)
-                outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
-                continue
-            else:
-                sparse_attn_prefill(vl, sel, L.q, k, v, idx, cnt, o_sp, lse_sp, ws=self.ws, stream=stream,
-                                    kg=kg, vg=vg)
-            if self.swa_window > 0 and self.decode:
+            elif self.swa_window > 0 and self.decode:
                 o_l = self._buf("o_l" + tag, (Tq, Hq, d), torch.bfloat16)
                 swa_gated_decode(vl, self.swa_window, L.q, L.k_swa, L.v_swa, L.gamma, o_sp, o_l, stream=stream)
             elif self.swa_window > 0:
@@ -133,7 +135,66 @@ class HybridBlock:
             else:
                 o_l = o_sp
             outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
+            if layer_hook is not None:
+                layer_hook.after(i)  # every launch that reads this layer's inputs is enqueued
         return {"o_full": o, "lse_full": lse, "scores": scores, "idx": idx, "cnt": cnt, "layers": outs}
+
+    def forward_from_host(self, q_h, k_h, v_h, layers_h: List[SparseLayerIn], stream=None, fp8_kv=None,
+                          intermediates: bool = True, slots: Optional[int] = None):
+        """forward() with its inputs in pinned host memory. Q, K and V are copied
+        first; every sparse layer's inputs then stream in on a second stream
+        while the full layer and the layers before it compute. `slots` device
+        copies of a layer's inputs are used in turn (default: one per layer, so
+        every copy overlaps the full layer; fewer bound the device memory, a slot
+        being refilled once the layer that last used it has run). The outputs
+        are device tensors as in forward()."""
+        cs = torch.cuda.current_stream(self.device) if stream is None else stream
+        if getattr(self, "_copy_stream", None) is None:
+            self._copy_stream = torch.cuda.Stream(self.device)
+        cp = self._copy_stream
+        dev = lambda name, t: None if t is None else self._buf(name, tuple(t.shape), t.dtype)
+        q, k, v = dev("h_q", q_h), dev("h_k", k_h), dev("h_v", v_h)
+        n_slots = len(layers_h) if slots is None else max(1, min(slots, len(layers_h)))
+        slot = [SparseLayerIn(*(dev(f"h_s{j}_{f}", getattr(layers_h[0], f)) for f in ("q", "k_swa", "v_swa",
+                                                                                      "gamma")))
+                for j in range(n_slots)]
+        ready = [torch.cuda.Event() for _ in layers_h]
+        done = [torch.cuda.Event() for _ in layers_h]
+
+        def load(i):  # layer i's inputs into slot i % n_slots, on the copy stream
+            dst, src = slot[i % n_slots], layers_h[i]
+            with torch.cuda.stream(cp):
+                for f in ("q", "k_swa", "v_swa", "gamma"):
+                    if getattr(src, f) is not None:
+                        getattr(dst, f).copy_(getattr(src, f), non_blocking=True)
+                ready[i].record(cp)
+
+        cp.wait_stream(cs)  # the previous call is done with these buffers
+        with torch.cuda.stream(cp):
+            for d_, h_ in ((q, q_h), (k, k_h), (v, v_h)):
+                if h_ is not None:
+                    d_.copy_(h_, non_blocking=True)
+            qkv = torch.cuda.Event()
+            qkv.record(cp)
+        for i in range(n_slots):
+            load(i)
+        cs.wait_event(qkv)
+
+        class Hook:
+            def before(_, i):
+                cs.wait_event(ready[i])
+                return slot[i % n_slots]
+
+            def after(_, i):
+                done[i].record(cs)
+                if i + n_slots < len(layers_h):
+                    cp.wait_event(done[i])  # the slot is free once layer i has run
+                    load(i + n_slots)
+
+        res = self.forward(q, k, v, [None] * len(layers_h), stream=cs, fp8_kv=fp8_kv, intermediates=intermediates,
+                           layer_hook=Hook())
+        cs.wait_stream(cp)
+        return res
 
     def launches_per_forward(self, n_layers: int, fp8_prefill: bool = False) -> int:
         """Kernels of this library launched by one forward (memsets excluded):

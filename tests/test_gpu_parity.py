@@ -263,6 +263,29 @@ def test_gathered_rows_and_layer_match_the_per_tile_gather(name):
     assert torch.equal(vg.cpu().view(torch.int16), vg_ref.view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["tok_mqa32", "swa_gate", "dec_block_swa"])
+def test_forward_from_host_equals_forward(name):
+    """HybridBlock.forward_from_host (inputs in pinned host memory, each layer's
+    inputs streamed in under the earlier layers' compute) writes exactly what
+    forward() writes on device inputs, with a slot per layer and with two slots
+    (three sparse layers, so a slot is refilled)."""
+    from hybrid_sparse_attention_tma_b200.block import SparseLayerIn
+    w = (VARIANTS.get(name) or DECODE[name]).with_(n_sparse=3)
+    inp = W.make_block_inputs(w, device="cuda", seed=21)
+    blk = GpuBlock(w, inp)
+    a = blk.run()
+    ref = {"o_full": a["o_full"].clone(), "idx": a["idx"].clone(),
+           "o": [L["o"].clone() for L in a["layers"]]}
+    pin = (lambda t: None if t is None else t.cpu().pin_memory())
+    hl = [SparseLayerIn(pin(L.q), pin(L.k_swa), pin(L.v_swa), pin(L.gamma)) for L in blk.layers]
+    for slots in (None, 2):  # a slot per layer; two slots, refilled
+        b = blk.block.forward_from_host(pin(inp.q), pin(inp.k), pin(inp.v), hl, slots=slots)
+        torch.cuda.synchronize()
+        assert torch.equal(ref["o_full"], b["o_full"]) and torch.equal(ref["idx"], b["idx"])
+        assert torch.equal(ref["o"][-1], b["layers"][-1]["o"])
+        assert torch.equal(ref["o"][-2], b["layers"][-2]["o"])
+
+
 def test_swa_gate_two_call_path():
     """The unfused layer (hs_sparse_attn_prefill then hs_swa_gated) against the oracle."""
     run_and_check(VARIANTS["swa_gate"], seed=7, fused=False)
