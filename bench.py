@@ -6,8 +6,9 @@ chunked prefill -- 4 sequences with cached contexts {262144, 131072, 65536,
 16384} and new chunks {8192, 4096, 8192, 2048} queries, 64 query heads / 1 KV
 head, d = 128, token-level top-1024 + forced recent 128, tile 64, 1 full layer
 feeding 11 sparse layers; seeded synthetic bf16 N(0,1) inputs with 0.5 %
-planted keys. A "step" is one pass of the whole block: hs_full_attn_select
-(forward + token-score pass) -> hs_topk_select -> 11 x hs_sparse_attn_prefill.
+planted keys. A "step" is one pass of the whole block: hs_full_attn_select_topk
+(forward + token-score pass with the top-k inside it) -> hs_gather_selected_kv
+-> 11 x hs_sparse_attn_prefill.
 The per-step working set (~5 GB) is larger than the 126 MB L2. On one GPU the
 same line also carries a shorter measurement of every other configuration
 ("workloads"): the block-level HySparse prefill (with its own-cache window
@@ -362,7 +363,8 @@ def swa_pairs(w):
 def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=None, workload_name=None):
     import torch.distributed as dist
     import hybrid_sparse_attention_tma_b200 as hs
-    from hybrid_sparse_attention_tma_b200 import (full_attn_select, topk_select, sparse_attn_prefill,
+    from hybrid_sparse_attention_tma_b200 import (full_attn_select, full_attn_select_topk, topk_select,
+                                                  sparse_attn_prefill,
                                                   sparse_attn_decode, sparse_swa_gated_prefill,
                                                   gather_selected_kv, swa_gated_decode, HS_KV_BF16,
                                                   HS_KV_FP8_E4M3)
@@ -397,13 +399,18 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"]) if world == 1 else None
 
     swa_dec = blk.decode and blk.swa_window > 0
-    kinds = ["full", "topk", "sparse"] + (["gather"] if blk.gathered else []) + (["swa"] if swa_dec else [])
+    # token-level prefill takes the top-k inside the score pass: no top-k launch
+    kinds = (["full"] + ([] if blk.fuse_topk else ["topk"]) + ["sparse"] + (["gather"] if blk.gathered else [])
+             + (["swa"] if swa_dec else []))
     L0 = layers[0]
 
     def call(kind, st):
         """One library call of `kind` on stream `st` (the first sparse layer's inputs)."""
         sel, bufs = blk.sel, blk._bufs
-        if kind == "full":
+        if kind == "full" and blk.fuse_topk:
+            full_attn_select_topk(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"], bufs["scores"],
+                                  bufs["idx"], bufs["cnt"], ws=blk.ws, stream=st)
+        elif kind == "full":
             full_attn_select(vl, sel, inp.q, inp.k, inp.v, bufs["o_full"], bufs["lse_full"], bufs["scores"],
                              ws=blk.ws, stream=st)
         elif kind == "topk":
@@ -539,7 +546,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
         # visible (query, key) pair of the window)
         swa_flop = 4.0 * d * hq * swa_pairs(w) if w.swa_window > 0 else 0.0
         entry("sparse", kms["sparse"], 4.0 * d * G * vis + swa_flop, "tensor")
-    entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
+    if "topk" in kms:
+        entry("topk", kms["topk"], n_tiles * hkv * (nblk * 4 + w.topk * 4), "hbm")
     if blk.gathered:
         # K and V: every (tile, KV head) plane of topk rows written once, the
         # distinct selected rows read once (the rest of the reads hit L2)
@@ -554,7 +562,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])
     dom["kernel"] = ("full_decode_tc_kernel (both exact passes, one persistent launch)" if blk.decode
-                     else "attn_fwd_kernel<d, full, B> (+ token-score pass when B = 1)")
+                     else "attn_fwd_kernel<d, full, B> (+ token-score pass with the top-k fused when B = 1)")
     dom["traffic"] = traffic_for("attn_fwd_full", workload_name)
     dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
 

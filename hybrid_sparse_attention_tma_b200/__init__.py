@@ -16,7 +16,7 @@ import torch
 from . import _lib as L
 from ._lib import HsError, HS_KV_BF16, HS_KV_FP8_E4M3  # noqa: F401
 
-__all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "topk_select", "sparse_attn_prefill",
+__all__ = ["Varlen", "Sel", "Workspace", "full_attn_select", "full_attn_select_topk", "topk_select", "sparse_attn_prefill",
            "gather_selected_kv", "sparse_attn_decode", "swa_gated", "sparse_swa_gated_prefill", "kv_dequantize",
            "swa_ring_write", "swa_gated_decode",
            "workspace_size", "check_error", "HsError"]
@@ -126,6 +126,31 @@ def full_attn_select(vl: Varlen, sel: L.HsSel, q, k, v, o=None, lse=None, scores
         ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(scores),
         _ptr(buf), buf.numel(), _stream(stream)))
     return o, lse, scores
+
+
+def full_attn_select_topk(vl: Varlen, sel: L.HsSel, q, k, v, o=None, lse=None, scores=None, idx=None, cnt=None,
+                          ws: Optional[Workspace] = None, stream=None):
+    """Full layer and top-k in one call: (o, lse, idx, cnt) equal to those of
+    full_attn_select followed by topk_select. Token-level prefill takes the
+    top-k inside the score pass (`scores` is then scratch with undefined
+    content); other shapes run the two calls. Returns (o, lse, idx, cnt)."""
+    lib = L.load()
+    dev = q.device
+    Tq, Hq, d = q.shape
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty((Hq, Tq), dtype=torch.float32, device=dev) if lse is None else lse
+    nblk = (vl.max_kv + sel.block - 1) // sel.block
+    nt = vl.n_tiles(sel.q_tile)
+    if scores is None:
+        scores = torch.empty((nt, vl.n_kv_heads, nblk), dtype=torch.float32, device=dev)
+    idx = torch.empty((nt, vl.n_kv_heads, max(sel.topk, 1)), dtype=torch.int32, device=dev) if idx is None else idx
+    cnt = torch.empty((nt, vl.n_kv_heads), dtype=torch.int32, device=dev) if cnt is None else cnt
+    w = _ws(ws, dev)
+    buf = w.get(workspace_size(L.HS_OP_FULL_ATTN_SELECT, vl, sel), stream)
+    L.check("hs_full_attn_select_topk", lib.hs_full_attn_select_topk(
+        ctypes.byref(vl.c), ctypes.byref(sel), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(scores),
+        _ptr(idx), _ptr(cnt), _ptr(buf), buf.numel(), _stream(stream)))
+    return o, lse, idx, cnt
 
 
 def topk_select(vl: Varlen, sel: L.HsSel, scores, idx=None, cnt=None, ws: Optional[Workspace] = None,

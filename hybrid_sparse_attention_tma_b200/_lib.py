@@ -15,7 +15,7 @@ HS_KV_BF16, HS_KV_FP8_E4M3 = 0, 1
 # Every function the header declares; the CPU test checks the library exports them all.
 EXPORTS = [
     "hs_workspace_size", "hs_workspace_init", "hs_check_error", "hs_status_string",
-    "hs_full_attn_select", "hs_topk_select", "hs_sparse_attn_prefill",
+    "hs_full_attn_select", "hs_full_attn_select_topk", "hs_topk_select", "hs_sparse_attn_prefill",
     "hs_sparse_attn_decode", "hs_swa_gated", "hs_debug_wait_timeout", "hs_last_error_detail",
     "hs_full_attn_select_noalloc", "hs_sparse_swa_gated_prefill", "hs_debug_exp2_poly", "hs_kv_dequantize",
     "hs_gather_selected_kv", "hs_sparse_attn_prefill_gathered", "hs_swa_ring_write", "hs_swa_gated_decode",
@@ -69,6 +69,8 @@ def load():
     lib.hs_status_string.argtypes = [i32]
     lib.hs_full_attn_select.restype = i32
     lib.hs_full_attn_select.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hs_full_attn_select_topk.restype = i32
+    lib.hs_full_attn_select_topk.argtypes = [VL, SEL, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hs_topk_select.restype = i32
     lib.hs_topk_select.argtypes = [VL, SEL, vp, vp, vp, vp, sz, vp]
     lib.hs_sparse_attn_prefill.restype = i32

@@ -12,7 +12,8 @@ from typing import List, Optional
 
 import torch
 
-from . import (Varlen, Sel, Workspace, full_attn_select, topk_select, sparse_attn_prefill, sparse_attn_decode,
+from . import (Varlen, Sel, Workspace, full_attn_select, full_attn_select_topk, topk_select, sparse_attn_prefill,
+               sparse_attn_decode,
                swa_gated, sparse_swa_gated_prefill, kv_dequantize, gather_selected_kv, swa_gated_decode,
                swa_ring_write, HS_KV_BF16, HS_KV_FP8_E4M3)
 
@@ -28,7 +29,7 @@ class SparseLayerIn:
 
 class HybridBlock:
     def __init__(self, vl: Varlen, q_tile: int, block: int, topk: int, window: int, swa_window: int = 0,
-                 device="cuda", fused: bool = True, exclusive: bool = False):
+                 device="cuda", fused: bool = True, exclusive: bool = False, fuse_topk: bool = True):
         self.vl = vl
         self.sel = Sel(q_tile, block, topk, window, exclusive)
         self.swa_window = swa_window
@@ -45,6 +46,10 @@ class HybridBlock:
         # token-level prefill: the selected rows are gathered once per block
         # (hs_gather_selected_kv) and every plain sparse layer reads them
         self.gathered = (not self.decode and block == 1 and topk > 0 and not (swa_window > 0 and fused))
+        # token-level prefill: the top-k is taken inside the score pass
+        # (hs_full_attn_select_topk; the scores then stay scratch) unless
+        # fuse_topk=False (full layer, then hs_topk_select on the stored scores)
+        self.fuse_topk = fuse_topk and block == 1 and not self.decode
 
     def swa_rings(self, k_swa, v_swa, stream=None):
         """Decode: a layer's own window cache [T_kv, H_kv, d] (all positions, in
@@ -69,6 +74,7 @@ class HybridBlock:
     def forward(self, q, k, v, layers: List[SparseLayerIn], stream=None, keep_all: bool = False, fp8_kv=None,
                 intermediates: bool = True, layer_hook=None):
         """Returns dict(o_full, lse_full, scores, idx, cnt, layers=[{o_sparse, lse_sparse, o}]).
+        scores is None when the top-k ran inside the score pass (fuse_topk).
 
         With keep_all=False, output buffers are reused across calls (no
         allocation in steady state) and only the last layer's tensors are
@@ -94,8 +100,11 @@ class HybridBlock:
             kq, vq, ks, vs = fp8_kv
             k = kv_dequantize(kq, ks, self._buf("k_deq", tuple(kq.shape), torch.bfloat16), stream=stream)
             v = kv_dequantize(vq, vs, self._buf("v_deq", tuple(vq.shape), torch.bfloat16), stream=stream)
-        full_attn_select(vl, sel, q, k, v, o, lse, scores, ws=self.ws, stream=stream)
-        topk_select(vl, sel, scores, idx, cnt, ws=self.ws, stream=stream)
+        if self.fuse_topk:
+            full_attn_select_topk(vl, sel, q, k, v, o, lse, scores, idx, cnt, ws=self.ws, stream=stream)
+        else:
+            full_attn_select(vl, sel, q, k, v, o, lse, scores, ws=self.ws, stream=stream)
+            topk_select(vl, sel, scores, idx, cnt, ws=self.ws, stream=stream)
         kg = vg = None
         if self.gathered and layers:
             gshape = (nt, vl.n_kv_heads, sel.topk, d)
@@ -137,7 +146,8 @@ class HybridBlock:
             outs.append({"o_sparse": o_sp, "lse_sparse": lse_sp, "o": o_l})
             if layer_hook is not None:
                 layer_hook.after(i)  # every launch that reads this layer's inputs is enqueued
-        return {"o_full": o, "lse_full": lse, "scores": scores, "idx": idx, "cnt": cnt, "layers": outs}
+        return {"o_full": o, "lse_full": lse, "scores": None if self.fuse_topk else scores, "idx": idx, "cnt": cnt,
+                "layers": outs}
 
     def forward_from_host(self, q_h, k_h, v_h, layers_h: List[SparseLayerIn], stream=None, fp8_kv=None,
                           intermediates: bool = True, slots: Optional[int] = None):
@@ -199,7 +209,8 @@ class HybridBlock:
     def launches_per_forward(self, n_layers: int, fp8_prefill: bool = False) -> int:
         """Kernels of this library launched by one forward (memsets excluded):
         full layer 1 (block scores) / 3 (token scores: forward, item prefix,
-        score pass) / 1 (decode: both passes in one launch); top-k 1; each
+        score pass) / 1 (decode: both passes in one launch); top-k 1 (none
+        when it runs inside the score pass); each
         sparse layer 1 (prefill, with its window branch and gate when fused;
         decode, with its key ranges merged in the same launch), plus 1 for an
         unfused gated SWA branch; an FP8 prefill adds the two expansions, a
@@ -211,4 +222,5 @@ class HybridBlock:
         sparse = 1
         swa = 1 if (self.swa_window > 0 and not (self.fused and not self.decode)) else 0
         gather = 1 if (self.gathered and n_layers > 0) else 0
-        return full + 1 + n_layers * (sparse + swa) + (2 if fp8_prefill else 0) + gather
+        topk = 0 if self.fuse_topk else 1
+        return full + topk + n_layers * (sparse + swa) + (2 if fp8_prefill else 0) + gather

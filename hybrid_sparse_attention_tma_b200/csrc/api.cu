@@ -273,13 +273,23 @@ size_t spill_floats_per_cta(int max_kv, int B) {
   return 2 * size_t((max_kv + 127) / 128) * size_t(128 / B) * attn::kMaxItemRows;
 }
 
+// Workspace of the token-level score pass after the header: the item prefix
+// (n_tiles + 1 ints), then for the fused top-k the item order (n_tiles ints),
+// the per-plane arrival counters, the queue of completed planes (one int per
+// plane each) and the queue's two counters.
+size_t token_prefix_bytes(int n_tiles) { return align_up(sizeof(int) * (size_t(n_tiles) + 1), 256); }
+size_t token_arrive_bytes(int n_tiles, int Hkv) {
+  return align_up(sizeof(int) * (size_t(n_tiles) + 2 * size_t(n_tiles) * Hkv + 2), 256);
+}
+
 size_t full_ws_bytes(const hs_varlen* vl, const Shape& sh, const hs_sel* sel) {
   if (is_decode(vl, sel) && sh.d == 128 && sh.G <= 64) return full_decode_ws_bytes(vl, sh);
   size_t b = kHeaderBytes;
   if (sel->block > 1) {
     b += size_t(num_sms()) * spill_floats_per_cta(sh.max_kv, sel->block) * sizeof(float);
   } else {
-    b += align_up(sizeof(int) * (size_t(n_tiles_of(vl, sel->q_tile)) + 1), 256);  // token-score item prefix
+    const int nt = n_tiles_of(vl, sel->q_tile);
+    b += token_prefix_bytes(nt) + token_arrive_bytes(nt, sh.Hkv);  // token-score items, fused top-k counters
   }
   return align_up(b, 256);
 }
@@ -445,15 +455,72 @@ __global__ void debug_exp2_poly_kernel(const float* __restrict__ x, float* __res
   }
 }
 
-template <int D>
+template <int D, bool SELECT>
 hs_status launch_token_scores(const Maps& m, const tscore::Params& p, const SeqTable& st, const int* prefix,
                               int grid, cudaStream_t s) {
-  auto kern = tscore::token_scores_kernel<D>;
-  constexpr int smem = tscore::smem_bytes<D>() > 116 * 1024 ? tscore::smem_bytes<D>() : 116 * 1024;
+  auto kern = tscore::token_scores_kernel<D, SELECT>;
+  constexpr int smem =
+      tscore::smem_bytes<D, SELECT>() > 116 * 1024 ? tscore::smem_bytes<D, SELECT>() : 116 * 1024;
   static PerDeviceOnce once;
   if (set_smem_once(once, kern, smem) != cudaSuccess) return HS_ERR_CUDA;
-  kern<<<grid, tscore::kThreads, smem, s>>>(m.q, m.k, p, st, prefix);
+  kern<<<grid, tscore::threads<SELECT>(), smem, s>>>(m.q, m.k, p, st, prefix);
   return cudaGetLastError() == cudaSuccess ? HS_OK : HS_ERR_CUDA;
+}
+
+// Top-k taken inside the score pass (token level).
+struct FusedTopk {
+  const hs_sel* sel;
+  int32_t* idx;
+  int32_t* cnt;
+};
+
+// The token-level score pass: a second QK pass reduces max(s - lse) per key
+// (see token_scores.cuh); with `top`, each plane's top-k is selected in the
+// same kernel and the scores are left as scratch.
+hs_status token_pass(const hs_varlen* vl, const Shape& sh, int T, const Maps& m, const float* lse, float* scores,
+                     int nblk, float scale_log2, void* ws, cudaStream_t s, const FusedTopk* top) {
+  SeqTable table;
+  if (!fill_seqtable(vl, T, &table)) return HS_ERR_UNSUPPORTED;
+  const long long items = token_score_items(vl, T, sh.Hkv);
+  if (items > (1LL << 30)) return HS_ERR_UNSUPPORTED;
+  char* w = reinterpret_cast<char*>(ws) + kHeaderBytes;
+  int* prefix = reinterpret_cast<int*>(w);
+  int* order = top ? reinterpret_cast<int*>(w + token_prefix_bytes(table.n_tiles)) : nullptr;
+  const size_t n_planes = size_t(table.n_tiles) * sh.Hkv;
+  int* arrive = top ? order + table.n_tiles : nullptr;
+  int* queue = top ? arrive + n_planes : nullptr;
+  int* qctr = top ? queue + n_planes : nullptr;
+  tscore::item_prefix_kernel<<<1, 1024, 0, s>>>(table, sh.Hkv, prefix, order, arrive, queue, qctr);
+  if (cudaGetLastError() != cudaSuccess) return HS_ERR_CUDA;
+  tscore::Params tp{};
+  tp.lse = lse;
+  tp.scores = scores;
+  tp.G = sh.G;
+  tp.Hq = sh.Hq;
+  tp.Hkv = sh.Hkv;
+  tp.Tq = int(sh.Tq);
+  tp.nblk = nblk;
+  tp.scale_log2 = scale_log2;
+  tp.n_items = int(items);
+  tp.wc = wait_ctl(ws);
+  if (top) {
+    tp.arrive = arrive;
+    tp.queue = queue;
+    tp.qctr = qctr;
+    tp.idx = top->idx;
+    tp.cnt = top->cnt;
+    tp.k = top->sel->topk;
+    tp.w = top->sel->window;
+    tp.exclusive = (top->sel->flags & HS_SEL_WINDOW_EXCLUSIVE) ? 1 : 0;
+    tp.discard = 1;
+    tp.order = order;
+  }
+  const int tgrid = int(std::min<long long>(num_sms(), std::max<long long>(1, items)));
+  if (top)
+    return sh.d == 64 ? launch_token_scores<64, true>(m, tp, table, prefix, tgrid, s)
+                      : launch_token_scores<128, true>(m, tp, table, prefix, tgrid, s);
+  return sh.d == 64 ? launch_token_scores<64, false>(m, tp, table, prefix, tgrid, s)
+                    : launch_token_scores<128, false>(m, tp, table, prefix, tgrid, s);
 }
 
 }  // namespace
@@ -561,9 +628,11 @@ hs_status hs_check_error(void* ws, hs_stream_t stream) {
   return HS_OK;
 }
 
-hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
-                              const void* v, void* o, float* lse, float* scores, void* ws, size_t ws_bytes,
-                              hs_stream_t stream) {
+// The full layer; with `top` (token-level prefill only) the top-k is taken
+// inside the score pass and `scores` is scratch.
+static hs_status full_attn_select_impl(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                       const void* v, void* o, float* lse, float* scores, void* ws,
+                                       size_t ws_bytes, hs_stream_t stream, const FusedTopk* top) {
   Shape sh;
   hs_status st = check_varlen(vl, &sh);
   if (st != HS_OK) return st;
@@ -578,9 +647,11 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   const int n_tiles = n_tiles_of(vl, T);
   const int nblk = (sh.max_kv + B - 1) / B;
   cudaStream_t s = S(stream);
-  if (cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
+  // the fused top-k reads only keys the score pass wrote: no zero fill
+  if (!top && cudaMemsetAsync(scores, 0, size_t(n_tiles) * sh.Hkv * nblk * sizeof(float), s) != cudaSuccess)
     return HS_ERR_CUDA;
   if (is_decode(vl, sel) && sh.d == 128 && sh.G <= 64) {
+    if (top) return HS_ERR_UNSUPPORTED;
     // one query per sequence: both exact passes in one persistent tcgen05 kernel
     const int U = sh.batch * sh.Hkv;
     if (U > dtc::kMaxUnits) return HS_ERR_UNSUPPORTED;
@@ -665,29 +736,36 @@ hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void
   const int grid = std::min(num_sms(), std::max(1, sc.n_items));
   hs_status rc = dispatch_full(sh.d, B, m, p, sc, grid, s);
   if (rc != HS_OK || B > 1) return rc;
-  // token level: a second QK pass reduces max(s - lse) per key (see token_scores.cuh)
+  // token level: the second QK pass (see token_scores.cuh), with the top-k fused when asked
   if (!lse) return HS_ERR_INVALID_ARG;
-  SeqTable table;
-  if (!fill_seqtable(vl, T, &table)) return HS_ERR_UNSUPPORTED;
-  const long long items = token_score_items(vl, T, sh.Hkv);
-  if (items > (1LL << 30)) return HS_ERR_UNSUPPORTED;
-  int* prefix = reinterpret_cast<int*>(reinterpret_cast<char*>(ws) + kHeaderBytes);
-  tscore::item_prefix_kernel<<<1, 1024, 0, s>>>(table, sh.Hkv, prefix);
-  if (cudaGetLastError() != cudaSuccess) return HS_ERR_CUDA;
-  tscore::Params tp{};
-  tp.lse = lse;
-  tp.scores = scores;
-  tp.G = sh.G;
-  tp.Hq = sh.Hq;
-  tp.Hkv = sh.Hkv;
-  tp.Tq = int(sh.Tq);
-  tp.nblk = nblk;
-  tp.scale_log2 = p.scale_log2;
-  tp.n_items = int(items);
-  tp.wc = p.wc;
-  const int tgrid = int(std::min<long long>(num_sms(), std::max<long long>(1, items)));
-  return sh.d == 64 ? launch_token_scores<64>(m, tp, table, prefix, tgrid, s)
-                    : launch_token_scores<128>(m, tp, table, prefix, tgrid, s);
+  return token_pass(vl, sh, T, m, lse, scores, nblk, p.scale_log2, ws, s, top);
+}
+
+hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                              const void* v, void* o, float* lse, float* scores, void* ws, size_t ws_bytes,
+                              hs_stream_t stream) {
+  return full_attn_select_impl(vl, sel, q, k, v, o, lse, scores, ws, ws_bytes, stream, nullptr);
+}
+
+hs_status hs_full_attn_select_topk(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,
+                                   const void* v, void* o, float* lse, float* scores, int32_t* idx,
+                                   int32_t* cnt, void* ws, size_t ws_bytes, hs_stream_t stream) {
+  Shape sh;
+  hs_status st = check_varlen(vl, &sh);
+  if (st != HS_OK) return st;
+  if ((st = check_sel(sel)) != HS_OK) return st;
+  if (sh.Tq == 0) return HS_OK;  // nothing to read or write (pointers may be null)
+  if (!idx || !cnt) return HS_ERR_INVALID_ARG;
+  if (vl->batch > kMaxSeq) return HS_ERR_UNSUPPORTED;
+  const bool fused = sel->block == 1 && !(is_decode(vl, sel) && sh.d == 128 && sh.G <= 64);
+  if (fused) {
+    const FusedTopk top{sel, idx, cnt};
+    return full_attn_select_impl(vl, sel, q, k, v, o, lse, scores, ws, ws_bytes, stream, &top);
+  }
+  // block-level scores and the decode kernel: the two calls back to back
+  st = full_attn_select_impl(vl, sel, q, k, v, o, lse, scores, ws, ws_bytes, stream, nullptr);
+  if (st != HS_OK) return st;
+  return hs_topk_select(vl, sel, scores, idx, cnt, ws, ws_bytes, stream);
 }
 
 hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const float* scores, int32_t* idx, int32_t* cnt,

@@ -16,15 +16,33 @@
 // keys each) stay in shared memory while the tile's T*G query rows stream
 // through a 3-stage ring of 128-row chunks (with their lse). TMEM holds one
 // 128 x 128 fp32 accumulator per key block (4 x 128 columns).
+//
+// Fused top-k (SELECT): the top-k of a (tile, KV head) plane is taken inside
+// this kernel (HySparse2 release note: the selection is a free by-product of
+// the full layer). Items stay spread over all CTAs. The reducers of the item
+// that completes a plane (a per-plane arrival counter) append the plane to a
+// global queue of completed planes; two selector warps in every CTA take the
+// next queue slot whenever they are free, wait for it to be filled, and run
+// the row selection of topk.cuh on that plane's scores while they are still
+// in L2, then drop those L2 lines without write-back, so the scores neither
+// return from nor reach HBM. (Handing each plane to the CTA that completed it
+// instead piles the selections onto the slowest CTA: every CTA holds items of
+// every long plane, so the slowest one completes them all.) Tiles run longest
+// first across all sequences, so the planes completed last, whose selection
+// is not hidden behind other items, are the shortest.
 #pragma once
 
 #include "hs_common.cuh"
 #include "seqtable.cuh"
+#include "topk.cuh"
 
 namespace hs {
 namespace tscore {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;     // reducers (4 warps), producer, issuer
+constexpr int kSelThreads = 64;   // selector warps of the fused top-k (8 warps in all: no register cap below 255)
+template <bool SELECT>
+constexpr int threads() { return SELECT ? kThreads + kSelThreads : kThreads; }
 constexpr int kBlocks = 4;   // key blocks per item
 constexpr int kQStagesMax = 3;
 template <int D>
@@ -38,6 +56,15 @@ struct Params {
   float scale_log2;
   int n_items;
   WaitCtl wc;
+  // fused top-k only (the work areas are set up by item_prefix_kernel)
+  int* arrive;       // [n_tiles * Hkv] items finished per plane (zeroed)
+  int* queue;        // [n_tiles * Hkv] completed planes in completion order (-1 = slot not filled yet)
+  int* qctr;         // [0] slots handed out to selectors, [1] slots filled
+  int* idx;          // [n_tiles, Hkv, k]
+  int* cnt;          // [n_tiles, Hkv]
+  int k, w, exclusive;
+  int discard;       // 1: drop each selected plane's score lines from L2 (scores are scratch)
+  const int* order;  // [n_tiles] tile at each position of the item order (longest first), or null
 };
 
 // The row's lse enters the MMA as one extra K step of 16 columns: K rows get
@@ -56,6 +83,7 @@ struct Layout {
   static constexpr int kOffQa = kOffQ + kQStages * kTile;
   static constexpr int kOffKa = kOffQa + kQStages * kAug;
   static constexpr int kOffCtl = kOffKa + kAug;
+  static constexpr int kOffSel = kOffCtl + 512;  // selector scratch (fused top-k)
 };
 
 struct Ctl {
@@ -63,15 +91,18 @@ struct Ctl {
   uint64_t q_full[kQStagesMax], q_empty[kQStagesMax];
   uint64_t acc_full[kBlocks], acc_free[kBlocks];
   uint64_t teardown;
+  uint64_t sel_bar;
+  int sel_slot;  // queue slot taken by the selector group
   uint32_t tmem_base;
   int abort;
 };
+static_assert(sizeof(Ctl) <= 512, "control block over its slot");
 
-template <int D>
+template <int D, bool SELECT = false>
 constexpr int smem_bytes() {
-  return Layout<D>::kOffCtl + int(sizeof(Ctl)) + 1024;
+  return Layout<D>::kOffSel + (SELECT ? int(sizeof(topk::SelScratch<kSelThreads>)) : 0) + 1024;
 }
-static_assert(smem_bytes<128>() <= 232448 && smem_bytes<64>() <= 232448, "smem over 227 KB");
+static_assert(smem_bytes<128, true>() <= 232448 && smem_bytes<64, true>() <= 232448, "smem over 227 KB");
 
 // unswizzled K-major descriptor (layout type 0)
 __device__ __forceinline__ uint64_t sdesc_noswz(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -99,6 +130,47 @@ __device__ __forceinline__ int ranges_of(const TileInfo& ti) {
   return (ti.pos0 + ti.n - 1) / (kBlocks * 128) + 1;
 }
 
+// Last query position of tile i of sequence b (the tile's longest plane).
+__device__ __forceinline__ int tile_last(const SeqTable& st, int b, int i) {
+  const int n_b = st.cu_q[b + 1] - st.cu_q[b];
+  const int ctx = st.cu_kv[b + 1] - st.cu_kv[b] - n_b;
+  return ctx + min((i + 1) * st.T, n_b) - 1;
+}
+
+// Position of `tile` in the longest-first order: tiles by last position
+// descending, ties to the lower sequence. Inside one sequence the last
+// position rises with the tile index, so each sequence contributes the count
+// of its tiles that come first, found by binary search.
+__device__ int longest_first_rank(const SeqTable& st, int tile) {
+  int b = 0;
+  {
+    int lo = 0, hi = st.batch - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (st.tile_base[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+  }
+  const int i = tile - st.tile_base[b];
+  const int x = tile_last(st, b, i);
+  int rank = st.tile_base[b + 1] - st.tile_base[b] - 1 - i;  // own sequence: its later tiles
+  for (int c = 0; c < st.batch; ++c) {
+    if (c == b) continue;
+    const int nt = st.tile_base[c + 1] - st.tile_base[c];
+    // first tile of c that comes before `tile`: last > x (or >= x for c < b)
+    int lo = 0, hi = nt;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      const int y = tile_last(st, c, mid);
+      if (y > x || (c < b && y == x)) hi = mid; else lo = mid + 1;
+    }
+    rank += nt - lo;
+  }
+  return rank;
+}
+
+__device__ __forceinline__ int order_tile(const int* order, int v) { return order ? order[v] : v; }
+
 // items are laid out tile-major: item = tile_item_base(tile) + g * ranges + r.
 // The prefix of items per tile is computed on the fly by a binary search over
 // tiles using the closed form of ranges per tile inside one sequence.
@@ -109,8 +181,8 @@ __device__ __forceinline__ Item get_item(const SeqTable& st, const Params& p, co
     if (tile_items_prefix[mid] <= w) lo = mid; else hi = mid - 1;
   }
   Item it;
-  it.tile = lo;
-  it.ti = tile_info(st, lo);
+  it.tile = order_tile(p.order, lo);
+  it.ti = tile_info(st, it.tile);
   const int nr = ranges_of(it.ti);
   const int local = w - tile_items_prefix[lo];
   it.g = local / nr;
@@ -122,14 +194,27 @@ __device__ __forceinline__ Item get_item(const SeqTable& st, const Params& p, co
   return it;
 }
 
-// Prefix sums of items per tile (Hkv * 512-key ranges), one CTA of 1024 threads.
-__global__ void __launch_bounds__(1024) item_prefix_kernel(const __grid_constant__ SeqTable st, int Hkv, int* out) {
+// Prefix sums of items per tile in item order (Hkv * 512-key ranges), one CTA
+// of 1024 threads. With `order` (fused top-k) the item order is longest tile
+// first, written to order[], and the top-k's per-plane arrival counters, its
+// queue of completed planes and the queue's two counters are reset.
+__global__ void __launch_bounds__(1024) item_prefix_kernel(const __grid_constant__ SeqTable st, int Hkv, int* out,
+                                                           int* order, int* arrive, int* queue, int* qctr) {
   __shared__ int part[1024];
   const int n = st.n_tiles;
+  if (order) {
+    for (int t = threadIdx.x; t < n; t += 1024) order[longest_first_rank(st, t)] = t;
+    for (int i = threadIdx.x; i < n * Hkv; i += 1024) {
+      arrive[i] = 0;
+      queue[i] = -1;
+    }
+    if (threadIdx.x < 2) qctr[threadIdx.x] = 0;
+    __syncthreads();  // order[] complete before the prefix reads it
+  }
   const int per = (n + 1023) / 1024;
   const int t0 = threadIdx.x * per, t1 = min(n, t0 + per);
   int sum = 0;
-  for (int t = t0; t < t1; ++t) sum += Hkv * ranges_of(tile_info(st, t));
+  for (int t = t0; t < t1; ++t) sum += Hkv * ranges_of(tile_info(st, order_tile(order, t)));
   part[threadIdx.x] = sum;
   __syncthreads();
   for (int off = 1; off < 1024; off <<= 1) {  // inclusive scan (Hillis-Steele)
@@ -141,13 +226,49 @@ __global__ void __launch_bounds__(1024) item_prefix_kernel(const __grid_constant
   int acc = threadIdx.x > 0 ? part[threadIdx.x - 1] : 0;
   for (int t = t0; t < t1; ++t) {
     out[t] = acc;
-    acc += Hkv * ranges_of(tile_info(st, t));
+    acc += Hkv * ranges_of(tile_info(st, order_tile(order, t)));
   }
   if (threadIdx.x == 1023) out[n] = part[1023];
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+// Drop the L2 lines that lie wholly inside [base, base + bytes) without
+// writing them back (their content becomes undefined). Lines shared with
+// neighbouring data are left alone.
+__device__ __forceinline__ void discard_lines(const void* base, size_t bytes, int t, int nthreads) {
+  const uintptr_t b = reinterpret_cast<uintptr_t>(base);
+  const uintptr_t first = (b + 127) & ~uintptr_t(127), end = (b + bytes) & ~uintptr_t(127);
+  for (uintptr_t a = first + uintptr_t(t) * 128; a < end; a += uintptr_t(nthreads) * 128)
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(a) : "memory");
+}
+
+// A selector's wait for queue slot h to be filled may last as long as the
+// whole pass: it gives up only when no plane at all was completed (the filled
+// count stood still) for the time limit. Returns the plane, or -1.
+__device__ __noinline__ int wait_for_slot(const int* slot, const int* filled, volatile int* abort_flag,
+                                          const WaitCtl& wc, int site, int ctx) {
+  unsigned long long t0 = global_ns();
+  long long c0 = clock64();
+  int seen = -1;
+  while (true) {
+    const int v = *reinterpret_cast<const volatile int*>(slot);
+    if (v >= 0) return v;
+    if (*abort_flag) return -1;
+    const int now = *reinterpret_cast<const volatile int*>(filled);
+    if (now != seen) {
+      seen = now;
+      t0 = global_ns();
+      c0 = clock64();
+    } else if (wait_expired(t0, c0, wc.timeout_ns)) {
+      *abort_flag = 1;
+      record_failure(wc, site, ctx);
+      return -1;
+    }
+    __nanosleep(1024);
+  }
+}
+
+template <int D, bool SELECT>
+__global__ void __launch_bounds__(threads<SELECT>(), 1)
     token_scores_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                         const Params p, const __grid_constant__ SeqTable st, const int* __restrict__ tile_items_prefix) {
   using L = Layout<D>;
@@ -175,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&c.acc_free[b], 4);
     }
     mbar_init(&c.teardown, 1);
+    if constexpr (SELECT) mbar_init(&c.sel_bar, kSelThreads / 32);  // selector group barrier
     c.abort = 0;
     fence_mbar_init();
   }
@@ -314,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(&c.teardown);
       mbar_wait_drain(&c.teardown, 0, p.wc, 192);
     }
-  } else {
+  } else if (warp < 4) {
     // ===================== reducers: thread = key lane =====================
     const int kl = warp * 32 + lane;  // key within each 128-key block
     int acc_cnt[kBlocks] = {0, 0, 0, 0};
@@ -376,6 +498,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (b < nb && key < it.key0 + it.nkeys) out[key] = best[b] > -1.0e30f ? ex2(best[b] * cs) : 0.f;
         }
       }
+      if constexpr (SELECT) {
+        // Count the item on its plane once all four warps' scores are visible
+        // device-wide; the CTA that brings the count to the plane's item total
+        // appends the plane to the queue of completed planes. Every reducer
+        // thread takes this barrier once per item, whatever its `ok`.
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 0 && ok && !*abort_flag) {
+          const int plane = it.tile * p.Hkv + it.g;
+          if (atomicAdd(p.arrive + plane, 1) == ranges_of(it.ti) - 1) {
+            __threadfence();  // the other CTAs' scores of the plane are seen before the slot is
+            const int slot = atomicAdd(p.qctr + 1, 1);
+            atomicExch(p.queue + slot, plane);
+          }
+        }
+      }
+    }
+  } else if constexpr (SELECT) {
+    // ===================== selectors: top-k of each completed plane =====================
+    const int t = threadIdx.x - kThreads;
+    topk::SelScratch<kSelThreads>& ss = *reinterpret_cast<topk::SelScratch<kSelThreads>*>(smem + L::kOffSel);
+    bool ok = true;
+    uint32_t ph = 0;
+    // bounded group barrier of the selector warps (release / acquire at CTA scope)
+    auto gsync = [&]() {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.sel_bar);
+      if (ok && !mbar_wait_warp(&c.sel_bar, ph, abort_flag, p.wc, 140)) ok = false;
+      ph ^= 1;
+    };
+    const int n_planes = st.n_tiles * p.Hkv;
+    while (ok) {
+      // take the next queue slot (one thread), share it with the group
+      if (t == 0) c.sel_slot = atomicAdd(p.qctr, 1);
+      gsync();
+      const int h = *reinterpret_cast<volatile int*>(&c.sel_slot);
+      gsync();  // both warps have read it before it is overwritten
+      if (!ok || h >= n_planes) break;
+      int plane = -1;
+      if (lane == 0) plane = wait_for_slot(p.queue + h, p.qctr + 1, abort_flag, p.wc, 141, h);
+      plane = __shfl_sync(0xffffffffu, plane, 0);
+      if (plane < 0 || plane >= n_planes) break;
+      __threadfence();
+      const TileInfo ti = tile_info(st, plane / p.Hkv);
+      const int n = topk::n_candidates(ti, p.nblk, 1, p.w, p.exclusive);
+      const float* row = p.scores + size_t(plane) * p.nblk;
+      // written by other CTAs during this kernel: read at L2, the point of
+      // coherence (a line of this SM's L1 could hold an older copy of a
+      // neighbouring plane's edge); 32 loads in flight per lane
+      auto key_at = [&](int j) -> uint32_t { return __float_as_uint(__ldcg(row + j)); };
+      topk::select_row<kSelThreads, 32>(n, p.k, t, key_at, gsync, ss, p.idx + size_t(plane) * p.k,
+                                        p.cnt + plane);
+      gsync();  // every read of the plane is done before its lines are dropped
+      if (p.discard) discard_lines(row, size_t(ti.pos0 + ti.n) * sizeof(float), t, kSelThreads);
     }
   }
   tc_fence_before();

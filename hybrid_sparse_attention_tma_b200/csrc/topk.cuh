@@ -12,9 +12,14 @@
 // A 4-pass MSB-first radix select (8 bits per pass, per-warp histograms in
 // shared memory) finds the k-th largest bit pattern tau and how many of the
 // k slots go to entries equal to tau. A final compaction over the row in
-// index order (each thread a contiguous segment, one block scan) keeps every
-// entry > tau plus the first (k - #greater) entries == tau. Index order both
-// breaks ties toward the lower index and emits the result already sorted.
+// index order (each warp a contiguous range walked 32 keys at a time, one
+// scan over the warps, ballots inside a warp) keeps every entry > tau plus
+// the first (k - #greater) entries == tau. Index order both breaks ties
+// toward the lower index and emits the result already sorted.
+//
+// The row selection is a device function over any number of whole warps and
+// any barrier: the kernel below runs it per CTA, and the token-score pass
+// runs it on two of its warps for the fused top-k.
 //
 // Two shapes of the same kernel: rows of up to kStageMax candidates are
 // staged once in shared memory by a 256-thread CTA (block-level selection,
@@ -38,11 +43,21 @@ struct Params {
   int w, exclusive;  // forced window; 1 = candidates stop before the last query's window
 };
 
-// Block-wide exclusive scan of one int per thread; returns the total.
+// Shared scratch of one row selection (kWarps per-warp histograms).
 template <int THREADS>
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total) {
+struct SelScratch {
+  int hist[THREADS / 32][256];
+  int warp_sums[32];
+  uint32_t prefix;
+  int krem;
+};
+
+// Exclusive scan of one int per thread over THREADS threads (t = 0 ..
+// THREADS - 1, whole warps) with `sync()` as their barrier; returns the total.
+template <int THREADS, typename Sync>
+__device__ __forceinline__ int group_excl_scan(int v, int t, int* warp_sums, int& total, Sync sync) {
   constexpr int kWarps = THREADS / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lane = t & 31, warp = t >> 5;
   int x = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
@@ -50,7 +65,7 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
     if (lane >= off) x += y;
   }
   if (lane == 31) warp_sums[warp] = x;
-  __syncthreads();
+  sync();
   if (warp == 0) {
     int s = lane < kWarps ? warp_sums[lane] : 0;
 #pragma unroll
@@ -60,66 +75,51 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_sums, int& total
     }
     if (lane < kWarps) warp_sums[lane] = s;  // inclusive
   }
-  __syncthreads();
+  sync();
   total = warp_sums[kWarps - 1];
   const int base = warp > 0 ? warp_sums[warp - 1] : 0;
-  __syncthreads();
+  sync();
   return base + x - v;
 }
 
-template <int THREADS, bool STAGED>
-__global__ void __launch_bounds__(THREADS)
-    topk_kernel(const Params p, const __grid_constant__ SeqTable st) {
+// Top-k of one row of n candidates, run by THREADS threads (t = 0 .. THREADS
+// - 1, whole warps) with `sync()` as their barrier; key(j) is the fp32 bit
+// pattern of candidate j (scores are >= 0, so bit order is value order).
+// Writes out[0 .. k) (kept indices ascending, padded -1) and *cnt_out.
+template <int THREADS, int kU = 8, typename Key, typename Sync>
+__device__ void select_row(int n, int k, int t, Key key_at, Sync sync, SelScratch<THREADS>& sc, int* out,
+                           int* cnt_out) {
   constexpr int kWarps = THREADS / 32;
-  __shared__ int hist[kWarps][256];
-  __shared__ int warp_sums[32];
-  __shared__ uint32_t s_prefix;
-  __shared__ int s_krem;
-  __shared__ uint32_t staged[STAGED ? kStageMax : 1];
-
-  const int row = blockIdx.x;  // tile * Hkv + g
-  const int tile = row / p.Hkv;
-  const TileInfo ti = tile_info(st, tile);
-  const int last_pos = ti.pos0 + ti.n - 1;
-  const int lim = p.exclusive ? last_pos - p.w : last_pos;  // candidates: b * B <= lim
-  const int n = lim < 0 ? 0 : min(p.nblk, lim / p.B + 1);
-  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
-  int* out = p.idx + size_t(row) * p.k;
-  const int k = p.k;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-
+  const int lane = t & 31, warp = t >> 5;
   if (n <= k) {
     // every candidate is kept
-    for (int j = threadIdx.x; j < k; j += THREADS) out[j] = j < n ? j : -1;
-    if (threadIdx.x == 0) p.cnt[row] = n;
+    for (int j = t; j < k; j += THREADS) out[j] = j < n ? j : -1;
+    if (t == 0) *cnt_out = n;
     return;
   }
   if (k == 0) {
-    if (threadIdx.x == 0) p.cnt[row] = 0;
+    if (t == 0) *cnt_out = 0;
     return;
   }
-  if constexpr (STAGED) {
-    for (int j = threadIdx.x; j < n; j += THREADS) staged[j] = __ldg(gkeys + j);
-    __syncthreads();
-  }
-  auto key_at = [&](int j) -> uint32_t {
-    if constexpr (STAGED) return staged[j];
-    else return __ldg(gkeys + j);
-  };
-
   // ---- radix select of the k-th largest bit pattern ----
   uint32_t prefix = 0;  // fixed high bits of tau
   int krem = k;         // how many of the k still to place at/below the prefix
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
-    for (int b = lane; b < 256; b += 32) hist[warp][b] = 0;
+    for (int b = lane; b < 256; b += 32) sc.hist[warp][b] = 0;
     __syncwarp();
-    for (int j = threadIdx.x; j < n; j += THREADS) {
-      const uint32_t key = key_at(j);
-      if ((key & hi_mask) == prefix) atomicAdd(&hist[warp][(key >> shift) & 0xFF], 1);
+    // kU loads in flight per thread before their histogram updates (rows read
+    // from L2 are latency-bound); consecutive threads read consecutive keys
+    for (int j0 = t; j0 < n; j0 += kU * THREADS) {
+      uint32_t kk[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) kk[u] = j0 + u * THREADS < n ? key_at(j0 + u * THREADS) : 0u;
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (j0 + u * THREADS < n && (kk[u] & hi_mask) == prefix) atomicAdd(&sc.hist[warp][(kk[u] >> shift) & 0xFF], 1);
     }
-    __syncthreads();
+    sync();
     // bins reduced across warps; warp 0 finds the bucket holding the krem-th largest
     if (warp == 0) {
       int cnt8[8];
@@ -128,7 +128,7 @@ __global__ void __launch_bounds__(THREADS)
       for (int e = 0; e < 8; ++e) {  // lane handles bins 255 - (lane*8 + e), descending
         const int b = 255 - (lane * 8 + e);
         int s = 0;
-        for (int w = 0; w < kWarps; ++w) s += hist[w][b];
+        for (int w = 0; w < kWarps; ++w) s += sc.hist[w][b];
         cnt8[e] = s;
         tot += s;
       }
@@ -149,58 +149,107 @@ __global__ void __launch_bounds__(THREADS)
           acc += cnt8[e];
         }
         const int b = 255 - (lane * 8 + e);
-        s_prefix = prefix | (uint32_t(b) << shift);
-        s_krem = krem - acc;
+        sc.prefix = prefix | (uint32_t(b) << shift);
+        sc.krem = krem - acc;
       }
     }
-    __syncthreads();
-    prefix = s_prefix;
-    krem = s_krem;
+    sync();
+    prefix = sc.prefix;
+    krem = sc.krem;
+    sync();  // every thread has read them before the next pass overwrites
   }
   const uint32_t tau = prefix;
   const int take_eq = krem;  // entries equal to tau to keep (lowest indices)
 
   // ---- ordered compaction ----
-  // Thread t owns the contiguous segment [t*L, t*L + L) of the row: it counts
-  // its entries > tau and == tau, one pair of block scans gives every thread
-  // its output offset and the number of tau-entries before it, and a second
-  // walk writes the kept indices. Segments are in index order, so the output
-  // is ascending and ties go to the lowest indices.
-  const int L = (n + THREADS - 1) / THREADS;
-  const int j0 = min(n, threadIdx.x * L), j1 = min(n, j0 + L);
+  // Warp w owns the contiguous range [w*Lw, w*Lw + Lw) of the row (Lw a
+  // multiple of 32) and walks it 32 keys at a time, lane l reading key
+  // base + l (coalesced). A first walk counts the entries > tau and == tau
+  // of each warp; a scan over the warps gives each warp its output offset and
+  // the number of tau-entries before its range; the second walk writes the
+  // kept indices, each lane finding its place among the 32 by ballots. Ranges
+  // and lanes follow index order, so the output is ascending and ties go to
+  // the lowest indices.
+  const int Lw = ((n + kWarps - 1) / kWarps + 31) & ~31;
+  const int w0 = min(n, warp * Lw), w1 = min(n, w0 + Lw);
   int gt = 0, eq = 0;
-  {
-    // counting may go in any order: start each lane at a different offset so
-    // staged (shared-memory) segments whose length is a multiple of 32 do not
-    // put a warp's accesses in one bank
-    const int len = j1 - j0;
-    int off = len > 0 ? lane % len : 0;
-    for (int c = 0; c < len; ++c) {
-      const uint32_t key = key_at(j0 + off);
-      gt += key > tau ? 1 : 0;
-      eq += key == tau ? 1 : 0;
-      off = off + 1 == len ? 0 : off + 1;
-    }
+  for (int c0 = w0; c0 < w1; c0 += 32 * kU) {
+    uint32_t kk[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) kk[u] = c0 + u * 32 + lane < w1 ? key_at(c0 + u * 32 + lane) : 0u;
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (c0 + u * 32 + lane < w1) {
+        gt += kk[u] > tau ? 1 : 0;
+        eq += kk[u] == tau ? 1 : 0;
+      }
   }
+  gt = __reduce_add_sync(0xffffffffu, gt);
+  eq = __reduce_add_sync(0xffffffffu, eq);
   int gt_total, eq_total;
-  const int gt_before = block_excl_scan<THREADS>(gt, warp_sums, gt_total);
-  const int eq_before = block_excl_scan<THREADS>(eq, warp_sums, eq_total);
-  int pos = gt_before + min(eq_before, take_eq);
-  int eq_seen = eq_before;
+  const int gt_before = __shfl_sync(
+      0xffffffffu, group_excl_scan<THREADS>(lane == 0 ? gt : 0, t, sc.warp_sums, gt_total, sync), 0);
+  const int eq_before = __shfl_sync(
+      0xffffffffu, group_excl_scan<THREADS>(lane == 0 ? eq : 0, t, sc.warp_sums, eq_total, sync), 0);
   if (gt > 0 || (eq > 0 && eq_before < take_eq)) {
-    for (int j = j0; j < j1; ++j) {
-      const uint32_t key = key_at(j);
-      if (key > tau) {
-        out[pos++] = j;
-      } else if (key == tau) {
-        if (eq_seen < take_eq) out[pos++] = j;
-        ++eq_seen;
+    const uint32_t lt = (1u << lane) - 1u;
+    int pos_run = gt_before + min(eq_before, take_eq);  // output slots before this chunk
+    int eq_run = eq_before;                             // tau-entries before this chunk
+    for (int c0 = w0; c0 < w1; c0 += 32 * kU) {
+      uint32_t kk[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) kk[u] = c0 + u * 32 + lane < w1 ? key_at(c0 + u * 32 + lane) : 0u;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int j = c0 + u * 32 + lane;
+        const bool valid = j < w1;
+        const bool e = valid && kk[u] == tau;
+        const uint32_t be = __ballot_sync(0xffffffffu, e);
+        const bool keep = (valid && kk[u] > tau) || (e && eq_run + __popc(be & lt) < take_eq);
+        const uint32_t bk = __ballot_sync(0xffffffffu, keep);
+        // pos < k always holds for a consistent selection; the bound keeps a
+        // selection whose group barrier gave up (kernel aborting) inside out[]
+        const int pos = pos_run + __popc(bk & lt);
+        if (keep && pos < k) out[pos] = j;
+        pos_run += __popc(bk);
+        eq_run += __popc(be);
       }
     }
   }
-  const int out_base = gt_total + min(eq_total, take_eq);
-  for (int j = out_base + threadIdx.x; j < k; j += THREADS) out[j] = -1;
-  if (threadIdx.x == 0) p.cnt[row] = out_base;
+  const int out_base = min(k, gt_total + min(eq_total, take_eq));
+  for (int j = max(0, out_base) + t; j < k; j += THREADS) out[j] = -1;
+  if (t == 0) *cnt_out = out_base;
+}
+
+// Candidates of selection tile `tile`: blocks b with b * B <= the tile's last
+// query position (window-exclusive reading: <= last - w).
+__device__ __forceinline__ int n_candidates(const TileInfo& ti, int nblk, int B, int w, int exclusive) {
+  const int last_pos = ti.pos0 + ti.n - 1;
+  const int lim = exclusive ? last_pos - w : last_pos;
+  return lim < 0 ? 0 : min(nblk, lim / B + 1);
+}
+
+template <int THREADS, bool STAGED>
+__global__ void __launch_bounds__(THREADS)
+    topk_kernel(const Params p, const __grid_constant__ SeqTable st) {
+  __shared__ SelScratch<THREADS> sc;
+  __shared__ uint32_t staged[STAGED ? kStageMax : 1];
+  const int row = blockIdx.x;  // tile * Hkv + g
+  const TileInfo ti = tile_info(st, row / p.Hkv);
+  const int n = n_candidates(ti, p.nblk, p.B, p.w, p.exclusive);
+  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(p.scores + size_t(row) * p.nblk);
+  if constexpr (STAGED) {
+    if (n > p.k && p.k > 0) {
+      for (int j = threadIdx.x; j < n; j += THREADS) staged[j] = __ldg(gkeys + j);
+      __syncthreads();
+    }
+  }
+  auto key_at = [&](int j) -> uint32_t {
+    if constexpr (STAGED) return staged[j];
+    else return __ldg(gkeys + j);
+  };
+  select_row<THREADS>(n, p.k, int(threadIdx.x), key_at, [] { __syncthreads(); }, sc, p.idx + size_t(row) * p.k,
+                      p.cnt + row);
 }
 
 }  // namespace topk

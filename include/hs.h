@@ -178,6 +178,32 @@ HS_API hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const fl
                          void* ws, size_t ws_bytes, hs_stream_t stream);
 
 /*
+ * hs_full_attn_select_topk -- hs_full_attn_select followed by hs_topk_select,
+ * with the top-k taken inside the score pass where the selection is token
+ * level (HySparse2 release note on airebao.com: the top-k choice comes free
+ * with the full layer).
+ *
+ * Outputs o, lse, idx and cnt are exactly those of the two calls in sequence
+ * (same selection rule, ties and -1 padding). Token-level prefill (B = 1,
+ * not the one-query decode shape): each (tile, KV head)'s top-k is selected
+ * by the CTA that finishes its last score range, from the scores still in
+ * L2, and those cache lines are then dropped without write-back, so the
+ * scores make no HBM round trip and no separate top-k launch runs; `scores`
+ * is scratch of the usual [n_tiles, H_kv, n_blk] shape and its content on
+ * return is undefined. Other shapes (block-level selection, decode) run the
+ * two calls back to back and `scores` holds the scores as documented there.
+ * In: as hs_full_attn_select (lse required at token level). Out: o, lse,
+ * idx [n_tiles,H_kv,k], cnt [n_tiles,H_kv] (both required).
+ * Workspace: hs_workspace_size(HS_OP_FULL_ATTN_SELECT, ...).
+ * Errors: as hs_full_attn_select; HS_ERR_INVALID_ARG for null idx / cnt.
+ */
+HS_API hs_status hs_full_attn_select_topk(const hs_varlen* vl, const hs_sel* sel,
+                                   const void* q, const void* k, const void* v,
+                                   void* o, float* lse, float* scores,
+                                   int32_t* idx, int32_t* cnt,
+                                   void* ws, size_t ws_bytes, hs_stream_t stream);
+
+/*
  * hs_sparse_attn_prefill -- one sparse layer of a hybrid block.
  *
  * This layer's own queries attend over the full layer's K/V (KV Reuse) at

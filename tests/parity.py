@@ -93,9 +93,13 @@ def assert_indices_match(idx_g, cnt_g, scores_o, idx_o, cnt_o, tiles, k):
 
 
 class GpuBlock:
-    """Runs one hybrid block through the library's public block runner."""
+    """Runs one hybrid block through the library's public block runner.
 
-    def __init__(self, w, inp, device="cuda", fused=True):
+    By default the top-k runs as its own call on stored scores (fuse_topk=False)
+    so the scores can be checked against the oracle; the fused top-k is checked
+    bit for bit against that path."""
+
+    def __init__(self, w, inp, device="cuda", fused=True, fuse_topk=False):
         import hybrid_sparse_attention_tma_b200 as hs
         from hybrid_sparse_attention_tma_b200.block import HybridBlock, SparseLayerIn
         self.w = w
@@ -103,7 +107,7 @@ class GpuBlock:
         self.vl = hs.Varlen(w.cu_q(), w.cu_kv(), w.n_q_heads, w.n_kv_heads, w.head_dim, device=device)
         self.sel = hs.Sel(w.q_tile, w.block, w.topk, w.window, w.exclusive)
         self.block = HybridBlock(self.vl, w.q_tile, w.block, w.topk, w.window, w.swa_window, device=device,
-                                 fused=fused, exclusive=w.exclusive)
+                                 fused=fused, exclusive=w.exclusive, fuse_topk=fuse_topk)
         if self.block.decode and w.swa_window > 0:
             # decode reads each layer's own window cache as a ring of swa_window slots
             self.layers = [SparseLayerIn(L.q, *self.block.swa_rings(L.k_swa, L.v_swa), L.gamma) for L in inp.layers]

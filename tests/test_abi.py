@@ -127,6 +127,17 @@ def test_host_validation_errors(lib):
     assert swad(dec, 256, 256, 16) == L.HS_ERR_UNSUPPORTED
     assert swad(dec, 128, 128, None) == L.HS_ERR_INVALID_ARG
     assert swad(dec, 128, 128, 18) == L.HS_ERR_INVALID_ARG      # misaligned gate
+    # full layer + fused top-k: idx and cnt are required; the full layer's checks apply
+    ftk = lambda vl_, s_, idx, cnt, ptr=16, ws_bytes=1 << 30: lib.hs_full_attn_select_topk(
+        ctypes.byref(vl_) if vl_ is not None else None, ctypes.byref(s_), ptr, ptr, ptr, ptr, ptr, ptr, idx, cnt, 16,
+        ws_bytes, None)
+    assert ftk(vl, tok, None, 16) == L.HS_ERR_INVALID_ARG
+    assert ftk(vl, tok, 16, None) == L.HS_ERR_INVALID_ARG
+    assert ftk(None, tok, 16, 16) == L.HS_ERR_INVALID_ARG
+    assert ftk(vl, tok, 16, 16, ptr=None) == L.HS_ERR_INVALID_ARG
+    assert ftk(vl, tok, 16, 16, ptr=18) == L.HS_ERR_INVALID_ARG          # misaligned
+    assert ftk(vl, tok, 16, 16, ws_bytes=8) == L.HS_ERR_WORKSPACE
+    assert ftk(vl, L.HsSel(16, 1, 5000, 32), 16, 16) == L.HS_ERR_UNSUPPORTED
     # unknown selection flags are rejected
     bad = L.HsSel(16, 16, 8, 32, 2)
     assert _call_full(lib, vl, bad) == L.HS_ERR_INVALID_ARG
@@ -147,6 +158,9 @@ def test_batch_without_new_tokens_returns_before_touching_pointers(lib):
     n = None
     assert lib.hs_full_attn_select(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, n, n, 0, n) == L.HS_OK
     assert lib.hs_topk_select(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, 0, n) == L.HS_OK
+    for s_ in (blk, L.HsSel(64, 1, 1024, 128)):
+        assert lib.hs_full_attn_select_topk(ctypes.byref(vl), ctypes.byref(s_), n, n, n, n, n, n, n, n, n, 0,
+                                            n) == L.HS_OK
     assert lib.hs_sparse_attn_prefill(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, n, n, n, 0, n) == L.HS_OK
     assert lib.hs_sparse_swa_gated_prefill(ctypes.byref(vl), ctypes.byref(blk), n, n, n, n, n, 128, n, n, n, n, n,
                                            n, n, 0, n) == L.HS_OK

@@ -127,16 +127,38 @@ def check_block(w, inp, res, tile_ids=None, fp8=False):
             assert_close_out(o_l, O.gated_merge(gamma, o_sp, o_swa), what=f"layer {li} chain o")
 
 
+def check_fused_topk(w, blk, inp, res, fp8=False):
+    """Token-level prefill: hs_full_attn_select_topk (the top-k taken inside the
+    score pass) returns exactly the o, lse, idx and cnt of the two calls the
+    block ran (full layer, then hs_topk_select on the stored scores), whole
+    arrays including the -1 padding."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    if w.block != 1 or blk.block.decode:
+        return
+    k, v = inp.k, inp.v
+    if fp8:  # the block expanded the FP8 cache once; the full layer read that
+        k, v = blk.block._bufs["k_deq"], blk.block._bufs["v_deq"]
+    ws = hs.Workspace("cuda")
+    o, lse, idx, cnt = hs.full_attn_select_topk(blk.vl, blk.sel, inp.q, k, v, ws=ws)
+    hs.check_error(ws)
+    assert torch.equal(cnt, res["cnt"]), "fused top-k: cnt differs from the two-call path"
+    assert torch.equal(idx, res["idx"]), "fused top-k: idx differs from the two-call path"
+    assert torch.equal(o.view(torch.int16), res["o_full"].view(torch.int16))
+    assert torch.equal(lse.view(torch.int32), res["lse_full"].view(torch.int32))
+
+
 def run_and_check(w, seed=None, tile_ids=None, fp8=False, fused=True):
     import sys, time
     t0 = time.time()
     inp = W.make_block_inputs(w, device="cuda", seed=seed)
     torch.cuda.synchronize()
     t1 = time.time()
-    res = GpuBlock(w, inp, fused=fused).run(fp8=fp8)
+    blk = GpuBlock(w, inp, fused=fused)
+    res = blk.run(fp8=fp8)
     torch.cuda.synchronize()
     t2 = time.time()
     check_block(w, inp, res, tile_ids, fp8=fp8)
+    check_fused_topk(w, blk, inp, res, fp8=fp8)
     print(f"[{w.name}] inputs {t1 - t0:.1f}s gpu {t2 - t1:.2f}s oracle check {time.time() - t2:.1f}s",
           file=sys.stderr, flush=True)
     return inp, res
@@ -284,6 +306,78 @@ def test_forward_from_host_equals_forward(name):
         assert torch.equal(ref["o_full"], b["o_full"]) and torch.equal(ref["idx"], b["idx"])
         assert torch.equal(ref["o"][-1], b["layers"][-1]["o"])
         assert torch.equal(ref["o"][-2], b["layers"][-2]["o"])
+
+
+FUSED_TOPK_CASES = ["random", "dup_rows", "all_equal", "exclusive", "k_over_n", "k0", "d64_gqa", "block16",
+                    "decode"]
+
+
+@pytest.mark.parametrize("case", FUSED_TOPK_CASES)
+def test_fused_topk_equals_two_calls_on_ties_and_edges(case):
+    """hs_full_attn_select_topk against hs_full_attn_select + hs_topk_select on
+    inputs built for the selection's hard cases: K rows repeating with period
+    37 (equal scores for every key the same queries see: ties broken toward
+    the lower index), all-zero K (every visible key tied), the
+    window-exclusive reading, k above every tile's candidates, k = 0, d = 64
+    with GQA, plus the shapes that run the two calls inside (block level,
+    decode). o, lse, cnt and the kept indices must match exactly."""
+    import hybrid_sparse_attention_tma_b200 as hs
+    g = torch.Generator().manual_seed(5)
+    Hq, Hkv, d, T, B = 16, 1, 128, 16, 1
+    cu_q, cu_kv = [0, 300, 480, 481], [0, 1000, 1180, 1700]  # chunked, fresh, one query
+    if case == "d64_gqa":
+        Hq, Hkv, d = 8, 2, 64
+    if case == "block16":
+        B = 16
+    if case == "decode":
+        T, cu_q = 1, [0, 1, 2, 3]
+    Tq, Tkv = cu_q[-1], cu_kv[-1]
+    q = torch.randn(Tq, Hq, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(Tkv, Hkv, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(Tkv, Hkv, d, generator=g).to(torch.bfloat16)
+    if case == "dup_rows":
+        k = k[torch.arange(Tkv) % 37]
+    if case == "all_equal":
+        k = torch.zeros_like(k)
+    topk = {"k_over_n": 2000, "k0": 0}.get(case, 96)
+    window = 32
+    vl = hs.Varlen(cu_q, cu_kv, Hq, Hkv, d, device="cuda")
+    sel = hs.Sel(T, B, topk, window, case == "exclusive")
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    ws = hs.Workspace("cuda")
+    o1, lse1, sc = hs.full_attn_select(vl, sel, q, k, v, ws=ws)
+    idx1, cnt1 = hs.topk_select(vl, sel, sc, ws=ws)
+    o2, lse2, idx2, cnt2 = hs.full_attn_select_topk(vl, sel, q, k, v, ws=ws)
+    hs.check_error(ws)
+    assert torch.equal(cnt1, cnt2)
+    if topk > 0:
+        assert torch.equal(idx1, idx2)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    assert torch.equal(lse1.view(torch.int32), lse2.view(torch.int32))
+    if case == "all_equal" and B == 1:
+        # every candidate of a plane whose first query sees it is tied: the kept
+        # set of each tile starts at index 0
+        c = cnt2.cpu()
+        assert (idx2.cpu()[:, 0, 0][c[:, 0] > 0] == 0).all()
+
+
+@pytest.mark.parametrize("name", ["tok_mqa32", "swa_tok"])
+def test_block_with_fused_topk_equals_two_call_block(name):
+    """The block runner's token-level default (top-k inside the score pass)
+    writes exactly what the two-call block writes, every layer."""
+    from hybrid_sparse_attention_tma_b200.block import HybridBlock
+    w = VARIANTS[name].with_(n_sparse=2)
+    inp = W.make_block_inputs(w, device="cuda", seed=17)
+    a = GpuBlock(w, inp).run()
+    ref = {"idx": a["idx"].clone(), "cnt": a["cnt"].clone(), "o": [L["o"].clone() for L in a["layers"]]}
+    fb = GpuBlock(w, inp, fuse_topk=True)
+    assert fb.block.fuse_topk
+    b = fb.run()
+    torch.cuda.synchronize()
+    assert b["scores"] is None
+    assert torch.equal(ref["cnt"], b["cnt"]) and torch.equal(ref["idx"], b["idx"])
+    for x, y in zip(ref["o"], b["layers"]):
+        assert torch.equal(x.view(torch.int16), y["o"].view(torch.int16))
 
 
 def test_swa_gate_two_call_path():
