@@ -92,7 +92,8 @@ struct Ctl {
   uint64_t acc_full[kBlocks], acc_free[kBlocks];
   uint64_t teardown;
   uint64_t sel_bar;
-  int sel_slot;  // queue slot taken by the selector group
+  int sel_plane;  // plane handed from the polling selector thread to the group (-1: stop)
+  int sel_round;  // hand-overs so far
   uint32_t tmem_base;
   int abort;
 };
@@ -241,29 +242,32 @@ __device__ __forceinline__ void discard_lines(const void* base, size_t bytes, in
     asm volatile("discard.global.L2 [%0], 128;" ::"l"(a) : "memory");
 }
 
-// A selector's wait for queue slot h to be filled may last as long as the
-// whole pass: it gives up only when no plane at all was completed (the filled
-// count stood still) for the time limit. Returns the plane, or -1.
-__device__ __noinline__ int wait_for_slot(const int* slot, const int* filled, volatile int* abort_flag,
-                                          const WaitCtl& wc, int site, int ctx) {
+// A selector's wait for a word to reach `want` (a queue slot to be filled,
+// want = 0; the group's hand-over count) may last as long as the whole pass:
+// it gives up only when no plane at all was completed (the queue's filled
+// count stood still) for the time limit. Returns the word's value, or -1.
+__device__ __noinline__ int wait_at_least(const volatile int* word, int want, const int* filled,
+                                          volatile int* abort_flag, const WaitCtl& wc, int site, int ctx) {
   unsigned long long t0 = global_ns();
   long long c0 = clock64();
   int seen = -1;
-  while (true) {
-    const int v = *reinterpret_cast<const volatile int*>(slot);
-    if (v >= 0) return v;
+  for (int it = 0;; ++it) {
+    const int v = *word;
+    if (v >= want) return v;
     if (*abort_flag) return -1;
-    const int now = *reinterpret_cast<const volatile int*>(filled);
-    if (now != seen) {
-      seen = now;
-      t0 = global_ns();
-      c0 = clock64();
-    } else if (wait_expired(t0, c0, wc.timeout_ns)) {
-      *abort_flag = 1;
-      record_failure(wc, site, ctx);
-      return -1;
+    if ((it & 15) == 0) {  // the progress signal is a global read: not on every poll
+      const int now = *reinterpret_cast<const volatile int*>(filled);
+      if (now != seen) {
+        seen = now;
+        t0 = global_ns();
+        c0 = clock64();
+      } else if (wait_expired(t0, c0, wc.timeout_ns)) {
+        *abort_flag = 1;
+        record_failure(wc, site, ctx);
+        return -1;
+      }
     }
-    __nanosleep(1024);
+    __nanosleep(2048);
   }
 }
 
@@ -298,6 +302,7 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
     mbar_init(&c.teardown, 1);
     if constexpr (SELECT) mbar_init(&c.sel_bar, kSelThreads / 32);  // selector group barrier
     c.abort = 0;
+    c.sel_round = 0;
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -529,15 +534,23 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
       ph ^= 1;
     };
     const int n_planes = st.n_tiles * p.Hkv;
-    while (ok) {
-      // take the next queue slot (one thread), share it with the group
-      if (t == 0) c.sel_slot = atomicAdd(p.qctr, 1);
-      gsync();
-      const int h = *reinterpret_cast<volatile int*>(&c.sel_slot);
-      gsync();  // both warps have read it before it is overwritten
-      if (!ok || h >= n_planes) break;
+    for (int round = 1; ok; ++round) {
+      // one thread takes the next queue slot and waits (sleeping between
+      // polls of one word) for it to be filled; the other warp sleeps on the
+      // hand-over count in shared memory
       int plane = -1;
-      if (lane == 0) plane = wait_for_slot(p.queue + h, p.qctr + 1, abort_flag, p.wc, 141, h);
+      if (t == 0) {
+        const int h = atomicAdd(p.qctr, 1);
+        if (h < n_planes) plane = wait_at_least(p.queue + h, 0, p.qctr + 1, abort_flag, p.wc, 141, h);
+        *reinterpret_cast<volatile int*>(&c.sel_plane) = plane;
+        __threadfence_block();
+        *reinterpret_cast<volatile int*>(&c.sel_round) = round;
+      } else if (t == 32) {
+        if (wait_at_least(&c.sel_round, round, p.qctr + 1, abort_flag, p.wc, 142, round) >= round) {
+          __threadfence_block();  // the plane is read after the count that announced it
+          plane = *reinterpret_cast<volatile int*>(&c.sel_plane);
+        }
+      }
       plane = __shfl_sync(0xffffffffu, plane, 0);
       if (plane < 0 || plane >= n_planes) break;
       __threadfence();
