@@ -51,6 +51,11 @@ METRIC = "hybrid-block attn tokens/s; TFLOP/s & HBM GB/s as % of roofline (1×B2
 L2_BYTES = 126 * 1024 * 1024  # B200 L2; the per-kernel timing flushes twice this before each call
 KERNEL_SOURCES = ["hybrid_sparse_attention_tma_b200/csrc/attn_fwd.cuh",
                   "hybrid_sparse_attention_tma_b200/csrc/hs_common.cuh"]
+# the token-level full layer: the forward, then the score pass with the top-k fused
+TOKEN_LAYER_SOURCES = KERNEL_SOURCES + ["hybrid_sparse_attention_tma_b200/csrc/token_scores.cuh",
+                                        "hybrid_sparse_attention_tma_b200/csrc/topk.cuh",
+                                        "hybrid_sparse_attention_tma_b200/csrc/seqtable.cuh"]
+TRAFFIC_SOURCES = {"attn_fwd_full": KERNEL_SOURCES, "full_layer_token": TOKEN_LAYER_SOURCES}
 
 
 def parse():
@@ -107,9 +112,9 @@ def full_flops(w: W.Workload) -> float:
     return 4.0 * w.head_dim * w.n_q_heads * causal_pairs(w)
 
 
-def src_hash() -> str:
+def src_hash(kernel: str = "attn_fwd_full") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in TRAFFIC_SOURCES[kernel]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -124,7 +129,7 @@ def traffic_for(kernel: str, workload: str):
     with open(path) as f:
         d = json.load(f)
     e = d.get(f"{kernel}:{workload}")
-    if not e or e.get("src_hash") != src_hash():
+    if not e or e.get("src_hash") != src_hash(kernel):
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -563,7 +568,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     dom = dict(kernels["full"])
     dom["kernel"] = ("full_decode_tc_kernel (both exact passes, one persistent launch)" if blk.decode
                      else "attn_fwd_kernel<d, full, B> (+ token-score pass with the top-k fused when B = 1)")
-    dom["traffic"] = traffic_for("attn_fwd_full", workload_name)
+    token_full = w.block == 1 and not blk.decode  # forward + score pass (top-k fused) per launch
+    dom["traffic"] = traffic_for("full_layer_token" if token_full else "attn_fwd_full", workload_name)
     dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
 
     # ---- e2e through the public API with host buffers ----
