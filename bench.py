@@ -6,8 +6,8 @@ chunked prefill -- 4 sequences with cached contexts {262144, 131072, 65536,
 16384} and new chunks {8192, 4096, 8192, 2048} queries, 64 query heads / 1 KV
 head, d = 128, token-level top-1024 + forced recent 128, tile 64, 1 full layer
 feeding 11 sparse layers; seeded synthetic bf16 N(0,1) inputs with 0.5 %
-planted keys. A "step" is one pass of the whole block: hs_full_attn_select_topk
-(forward + token-score pass with the top-k inside it) -> hs_gather_selected_kv
+planted keys. A "step" is one pass of the whole block: hs_full_attn_select
+(forward + token-score pass) -> hs_topk_select -> hs_gather_selected_kv
 -> 11 x hs_sparse_attn_prefill.
 The per-step working set (~5 GB) is larger than the 126 MB L2. On one GPU the
 same line also carries a shorter measurement of every other configuration
@@ -404,7 +404,7 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
     recall = needle_recall(w, inp, blk._bufs["idx"], blk._bufs["cnt"]) if world == 1 else None
 
     swa_dec = blk.decode and blk.swa_window > 0
-    # token-level prefill takes the top-k inside the score pass: no top-k launch
+    # with the block's fuse_topk the top-k runs inside the score pass: no top-k launch
     kinds = (["full"] + ([] if blk.fuse_topk else ["topk"]) + ["sparse"] + (["gather"] if blk.gathered else [])
              + (["swa"] if swa_dec else []))
     L0 = layers[0]
@@ -567,8 +567,8 @@ def bench_ours(args, world, rank, local, w=None, steps=None, with_e2e=True, fp8=
         e["share_of_step"] = round(e["ms_per_launch"] * per_step[kd] / ms_step, 4)
     dom = dict(kernels["full"])
     dom["kernel"] = ("full_decode_tc_kernel (both exact passes, one persistent launch)" if blk.decode
-                     else "attn_fwd_kernel<d, full, B> (+ token-score pass with the top-k fused when B = 1)")
-    token_full = w.block == 1 and not blk.decode  # forward + score pass (top-k fused) per launch
+                     else "attn_fwd_kernel<d, full, B> (+ token-score pass when B = 1)")
+    token_full = w.block == 1 and not blk.decode  # forward + score pass per launch
     dom["traffic"] = traffic_for("full_layer_token" if token_full else "attn_fwd_full", workload_name)
     dom["peak_kind"] = f"{src} {'HBM copy' if blk.decode else 'bf16 burst'}"
 

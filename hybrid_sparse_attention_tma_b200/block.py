@@ -29,7 +29,7 @@ class SparseLayerIn:
 
 class HybridBlock:
     def __init__(self, vl: Varlen, q_tile: int, block: int, topk: int, window: int, swa_window: int = 0,
-                 device="cuda", fused: bool = True, exclusive: bool = False, fuse_topk: bool = True):
+                 device="cuda", fused: bool = True, exclusive: bool = False, fuse_topk: bool = False):
         self.vl = vl
         self.sel = Sel(q_tile, block, topk, window, exclusive)
         self.swa_window = swa_window
@@ -46,9 +46,11 @@ class HybridBlock:
         # token-level prefill: the selected rows are gathered once per block
         # (hs_gather_selected_kv) and every plain sparse layer reads them
         self.gathered = (not self.decode and block == 1 and topk > 0 and not (swa_window > 0 and fused))
-        # token-level prefill: the top-k is taken inside the score pass
-        # (hs_full_attn_select_topk; the scores then stay scratch) unless
-        # fuse_topk=False (full layer, then hs_topk_select on the stored scores)
+        # token-level prefill with fuse_topk=True: the top-k is taken inside the
+        # score pass (hs_full_attn_select_topk; the scores then stay scratch).
+        # The default runs the full layer, then hs_topk_select on the stored
+        # scores, which measures faster on B200 (the selection competes with
+        # the score pass for its SMs more than the separate launch costs).
         self.fuse_topk = fuse_topk and block == 1 and not self.decode
 
     def swa_rings(self, k_swa, v_swa, stream=None):

@@ -477,8 +477,12 @@ struct FusedTopk {
 // The token-level score pass: a second QK pass reduces max(s - lse) per key
 // (see token_scores.cuh); with `top`, each plane's top-k is selected in the
 // same kernel and the scores are left as scratch.
-hs_status token_pass(const hs_varlen* vl, const Shape& sh, int T, const Maps& m, const float* lse, float* scores,
-                     int nblk, float scale_log2, void* ws, cudaStream_t s, const FusedTopk* top) {
+hs_status token_pass(const hs_varlen* vl, const Shape& sh, int T, const void* q, const Maps& fwd_maps,
+                     const float* lse, float* scores, int nblk, float scale_log2, void* ws, cudaStream_t s,
+                     const FusedTopk* top) {
+  // Q chunks of tscore::kRows rows (query * G + head): a box of kRows / G queries
+  Maps m = fwd_maps;
+  if (!make_map_3d(&m.q, q, sh.d, sh.Hq, sh.Tq, sh.G, tscore::kRows / sh.G)) return HS_ERR_CUDA;
   SeqTable table;
   if (!fill_seqtable(vl, T, &table)) return HS_ERR_UNSUPPORTED;
   const long long items = token_score_items(vl, T, sh.Hkv);
@@ -738,7 +742,7 @@ static hs_status full_attn_select_impl(const hs_varlen* vl, const hs_sel* sel, c
   if (rc != HS_OK || B > 1) return rc;
   // token level: the second QK pass (see token_scores.cuh), with the top-k fused when asked
   if (!lse) return HS_ERR_INVALID_ARG;
-  return token_pass(vl, sh, T, m, lse, scores, nblk, p.scale_log2, ws, s, top);
+  return token_pass(vl, sh, T, q, m, lse, scores, nblk, p.scale_log2, ws, s, top);
 }
 
 hs_status hs_full_attn_select(const hs_varlen* vl, const hs_sel* sel, const void* q, const void* k,

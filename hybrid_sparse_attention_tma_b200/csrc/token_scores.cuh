@@ -12,10 +12,13 @@
 // single exp2 per (tile, key) at the end.
 //
 // CTA: warp 0-3 reducers (thread = key), warp 4 TMA producer, warp 5 UMMA
-// issuer. A work item is (tile, KV head, 512 keys): its 4 key blocks (128
+// issuer. A work item is (tile, KV head, 256 keys): its 2 key blocks (128
 // keys each) stay in shared memory while the tile's T*G query rows stream
-// through a 3-stage ring of 128-row chunks (with their lse). TMEM holds one
-// 128 x 128 fp32 accumulator per key block (4 x 128 columns).
+// through a ring of 256-row chunks (with their lse), each block taking one
+// M = 128, N = 256 MMA per K step: per FLOP that reads a quarter fewer
+// operand bytes from shared memory than N = 128, whose port the operand
+// reads alone would fill. TMEM holds one 128 x 256 fp32 accumulator per key
+// block (2 x 256 columns).
 //
 // Fused top-k (SELECT): the top-k of a (tile, KV head) plane is taken inside
 // this kernel (HySparse2 release note: the selection is a free by-product of
@@ -43,11 +46,13 @@ constexpr int kThreads = 192;     // reducers (4 warps), producer, issuer
 constexpr int kSelThreads = 64;   // selector warps of the fused top-k (8 warps in all: no register cap below 255)
 template <bool SELECT>
 constexpr int threads() { return SELECT ? kThreads + kSelThreads : kThreads; }
-constexpr int kBlocks = 4;   // key blocks per item
+constexpr int kBlocks = 2;   // key blocks per item
+constexpr int kRows = 256;   // query rows per chunk (the MMA's N)
 constexpr int kQStagesMax = 3;
 template <int D>
 constexpr int q_stages() { return D == 128 ? 2 : 3; }  // 2 at d = 128 to fit the augmentation tiles
-constexpr int kSlabBytes = 128 * 128;
+constexpr int kSlabBytes = 128 * 128;     // a 128-row x 64-column swizzled slab (K block)
+constexpr int kQSlabBytes = kRows * 128;  // a kRows-row x 64-column slab (Q chunk)
 
 struct Params {
   const float* lse;  // [Hq, Tq] natural log (from the forward pass)
@@ -75,13 +80,15 @@ struct Params {
 // core matrices, the two K halves 128 bytes apart, 8-row groups 256 apart.
 template <int D>
 struct Layout {
-  static constexpr int kTile = (D / 64) * kSlabBytes;  // 128 rows x D bf16
+  static constexpr int kTile = (D / 64) * kSlabBytes;    // K block: 128 rows x D bf16
+  static constexpr int kQTile = (D / 64) * kQSlabBytes;  // Q chunk: kRows rows x D bf16
   static constexpr int kQStages = q_stages<D>();
-  static constexpr int kAug = 128 * 16 * 2;            // 128 rows x 16 bf16
+  static constexpr int kAug = 128 * 16 * 2;              // K augmentation: 128 rows x 16 bf16
+  static constexpr int kQAug = kRows * 16 * 2;           // Q augmentation: kRows rows x 16 bf16
   static constexpr int kOffK = 0;
   static constexpr int kOffQ = kBlocks * kTile;
-  static constexpr int kOffQa = kOffQ + kQStages * kTile;
-  static constexpr int kOffKa = kOffQa + kQStages * kAug;
+  static constexpr int kOffQa = kOffQ + kQStages * kQTile;
+  static constexpr int kOffKa = kOffQa + kQStages * kQAug;
   static constexpr int kOffCtl = kOffKa + kAug;
   static constexpr int kOffSel = kOffCtl + 512;  // selector scratch (fused top-k)
 };
@@ -124,7 +131,7 @@ __device__ __forceinline__ uint32_t aug_off(int r, int half) {
 struct Item {
   int tile, g, key0, nkeys;  // keys [key0, key0 + nkeys)
   TileInfo ti;
-  int nchunks;               // 128-row chunks of the tile (rows = n * G)
+  int nchunks;               // kRows-row chunks of the tile (rows = n * G)
 };
 
 __device__ __forceinline__ int ranges_of(const TileInfo& ti) {
@@ -191,7 +198,7 @@ __device__ __forceinline__ Item get_item(const SeqTable& st, const Params& p, co
   it.key0 = r * kBlocks * 128;
   const int last = it.ti.pos0 + it.ti.n - 1;  // candidate keys are <= last
   it.nkeys = min(kBlocks * 128, last + 1 - it.key0);
-  it.nchunks = (it.ti.n * p.G + 127) / 128;
+  it.nchunks = (it.ti.n * p.G + kRows - 1) / kRows;
   return it;
 }
 
@@ -338,34 +345,35 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
       ++items;
       // the chunk's lse values (rows lane + 32 k, row = query * G + head-in-group)
       // are loaded one chunk ahead, so their latency overlaps the ring wait
-      const int qpc = 128 / p.G;
+      constexpr int kRowsPerLane = kRows / 32;
+      const int qpc = kRows / p.G;
       const float inv_c = 1.f / p.scale_log2;
-      auto load_lse = [&](int qc, float (&x)[4]) {
+      auto load_lse = [&](int qc, float (&x)[kRowsPerLane]) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kRowsPerLane; ++k) {
           const int rr = lane + 32 * k;
           const int ql = qc * qpc + rr / p.G;
           const int h = it.g * p.G + rr % p.G;
           x[k] = ql < it.ti.n ? __ldg(p.lse + size_t(h) * p.Tq + it.ti.qrow0 + ql) : 0.f;
         }
       };
-      float lse_nx[4];
+      float lse_nx[kRowsPerLane];
       load_lse(0, lse_nx);
       for (int qc = 0; qc < it.nchunks && ok; ++qc) {
         const int s = qctr % kQStages;
-        float lse_cur[4];
+        float lse_cur[kRowsPerLane];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) lse_cur[k] = lse_nx[k];
+        for (int k = 0; k < kRowsPerLane; ++k) lse_cur[k] = lse_nx[k];
         if (qc + 1 < it.nchunks) load_lse(qc + 1, lse_nx);
         int okw = 1;
         if (lane == 0) okw = mbar_wait(&c.q_empty[s], ((qctr / kQStages) & 1) ^ 1, abort_flag, p.wc, 102, (wi << 12) | qc);
         okw = __shfl_sync(0xffffffffu, okw, 0);
         if (!okw) { ok = false; break; }
-        // augmentation of the chunk's 128 rows: [hi, lo] = -lse2 / c as a bf16
+        // augmentation of the chunk's kRows rows: [hi, lo] = -lse2 / c as a bf16
         // pair; rows past the tile get a huge negative hi so they never win a maximum
-        uint8_t* qa = smem + L::kOffQa + s * L::kAug;
+        uint8_t* qa = smem + L::kOffQa + s * L::kQAug;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < kRowsPerLane; ++k) {
           const int rr = lane + 32 * k;
           const int ql = qc * qpc + rr / p.G;
           uint32_t hl = pack_bf16(-3.0e38f, 0.f);
@@ -380,10 +388,10 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          mbar_expect_tx(&c.q_full[s], L::kTile);
+          mbar_expect_tx(&c.q_full[s], L::kQTile);
           for (int sl = 0; sl < D / 64; ++sl)
-            tma_load_3d(smem + L::kOffQ + s * L::kTile + sl * kSlabBytes, &map_q, &c.q_full[s], sl * 64, it.g * p.G,
-                        it.ti.qrow0 + qc * qpc);
+            tma_load_3d(smem + L::kOffQ + s * L::kQTile + sl * kQSlabBytes, &map_q, &c.q_full[s], sl * 64,
+                        it.g * p.G, it.ti.qrow0 + qc * qpc);
           last_q[s] = qctr;
         }
         ++qctr;
@@ -397,9 +405,9 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
   } else if (warp == 5) {
     // ===================== UMMA issuer: S^T[key, row] = K_blk . Q_chunk^T =====================
     if (lane == 0) {
-      constexpr uint32_t kId = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t kId = idesc_bf16_f32(128, kRows, false, false);
       int qctr = 0, items = 0;
-      int acc_cnt[kBlocks] = {0, 0, 0, 0};
+      int acc_cnt[kBlocks] = {};
       bool ok = true;
       // descriptors built once; a K step adds its offset / 16 to the start field
       const uint64_t k_desc0 = sdesc_sw128(smem_u32(smem + L::kOffK), 16, 1024);
@@ -421,14 +429,15 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
             ++acc_cnt[b];
             tc_fence_after();
             const uint64_t ka = k_desc0 + uint64_t((b * L::kTile) >> 4);
-            const uint64_t qb = q_desc0 + uint64_t((s * L::kTile) >> 4);
+            const uint64_t qb = q_desc0 + uint64_t((s * L::kQTile) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t off = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
-              umma_bf16(tmem + b * 128, ka + off, qb + off, kId, kk > 0 ? 1u : 0u);
+              const uint64_t koff = uint64_t(((kk >> 2) * kSlabBytes + (kk & 3) * 32) >> 4);
+              const uint64_t qoff = uint64_t(((kk >> 2) * kQSlabBytes + (kk & 3) * 32) >> 4);
+              umma_bf16(tmem + b * kRows, ka + koff, qb + qoff, kId, kk > 0 ? 1u : 0u);
             }
             // + 1 * hi + 1 * lo = -lse2 / c per row
-            umma_bf16(tmem + b * 128, ka_desc, qa_desc0 + uint64_t((s * L::kAug) >> 4), kId, 1u);
+            umma_bf16(tmem + b * kRows, ka_desc, qa_desc0 + uint64_t((s * L::kQAug) >> 4), kId, 1u);
             umma_commit(&c.acc_full[b]);
           }
           if (!ok) break;
@@ -444,19 +453,19 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
   } else if (warp < 4) {
     // ===================== reducers: thread = key lane =====================
     const int kl = warp * 32 + lane;  // key within each 128-key block
-    int acc_cnt[kBlocks] = {0, 0, 0, 0};
+    int acc_cnt[kBlocks] = {};
     bool ok = true;
     const float cs = p.scale_log2;
     for (int wi = blockIdx.x; wi < p.n_items; wi += gridDim.x) {
       const Item it = get_item(st, p, tile_items_prefix, wi);
       const int nb = (it.nkeys + 127) / 128;
-      const int qpc = 128 / p.G;
+      const int qpc = kRows / p.G;
       float best[kBlocks];
 #pragma unroll
       for (int b = 0; b < kBlocks; ++b) best[b] = -INFINITY;
       for (int qc = 0; qc < it.nchunks && ok; ++qc) {
         // valid columns of this chunk: rows of queries inside the tile
-        const int c_max = min(128, (it.ti.n - qc * qpc) * p.G);
+        const int c_max = min(kRows, (it.ti.n - qc * qpc) * p.G);
         const int pos_first = it.ti.pos0 + qc * qpc;  // position of the chunk's first query
 #pragma unroll
         for (int b = 0; b < kBlocks; ++b) {
@@ -467,24 +476,27 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
           const int key = it.key0 + b * 128 + kl;
           // causal: column c (query pos_first + c / G) sees key iff c >= G * (key - pos_first)
           const int c_min = max(0, (key - pos_first) * p.G);
-          const bool full = (c_min == 0) && (c_max == 128);
-          const uint32_t taddr = tmem + b * 128 + (uint32_t(warp * 32) << 16);
+          const bool full = (c_min == 0) && (c_max == kRows);
+          const uint32_t taddr = tmem + b * kRows + (uint32_t(warp * 32) << 16);
           float m = best[b];  // max over rows of s - lse2 / c
-          // the accumulator's 128 columns in four loads, one wait
-          uint32_t v[4][32];
+          // the accumulator's kRows columns, 128 at a time: four loads, one wait
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) tmem_ld32(taddr + ch * 32, v[ch]);
-          tmem_ld_wait();
+          for (int h = 0; h < kRows / 128; ++h) {
+            uint32_t v[4][32];
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            if (full) {
+            for (int ch = 0; ch < 4; ++ch) tmem_ld32(taddr + h * 128 + ch * 32, v[ch]);
+            tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; e += 2) m = max3f(m, __uint_as_float(v[ch][e]), __uint_as_float(v[ch][e + 1]));
-            } else {
+            for (int ch = 0; ch < 4; ++ch) {
+              if (full) {
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int col = ch * 32 + e;
-                if (col >= c_min && col < c_max) m = fmaxf(m, __uint_as_float(v[ch][e]));
+                for (int e = 0; e < 32; e += 2) m = max3f(m, __uint_as_float(v[ch][e]), __uint_as_float(v[ch][e + 1]));
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const int col = h * 128 + ch * 32 + e;
+                  if (col >= c_min && col < c_max) m = fmaxf(m, __uint_as_float(v[ch][e]));
+                }
               }
             }
           }
@@ -505,13 +517,15 @@ __global__ void __launch_bounds__(threads<SELECT>(), 1)
       }
       if constexpr (SELECT) {
         // Count the item on its plane once all four warps' scores are visible
-        // device-wide; the CTA that brings the count to the plane's item total
-        // appends the plane to the queue of completed planes. Every reducer
-        // thread takes this barrier once per item, whatever its `ok`.
-        __threadfence();
+        // device-wide: the barrier orders the four warps' stores before
+        // thread 0's gpu-scope fence, which is cumulative, so one fence
+        // publishes them all. The CTA that brings the count to the plane's
+        // item total appends the plane to the queue of completed planes.
+        // Every reducer thread takes this barrier once per item, whatever its `ok`.
         named_bar_sync(1, 128);
         if (threadIdx.x == 0 && ok && !*abort_flag) {
           const int plane = it.tile * p.Hkv + it.g;
+          __threadfence();
           if (atomicAdd(p.arrive + plane, 1) == ranges_of(it.ti) - 1) {
             __threadfence();  // the other CTAs' scores of the plane are seen before the slot is
             const int slot = atomicAdd(p.qctr + 1, 1);

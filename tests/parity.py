@@ -95,9 +95,9 @@ def assert_indices_match(idx_g, cnt_g, scores_o, idx_o, cnt_o, tiles, k):
 class GpuBlock:
     """Runs one hybrid block through the library's public block runner.
 
-    By default the top-k runs as its own call on stored scores (fuse_topk=False)
-    so the scores can be checked against the oracle; the fused top-k is checked
-    bit for bit against that path."""
+    The top-k runs as its own call on stored scores (the runner's default) so
+    the scores can be checked against the oracle; the fused top-k
+    (fuse_topk=True) is checked bit for bit against that path."""
 
     def __init__(self, w, inp, device="cuda", fused=True, fuse_topk=False):
         import hybrid_sparse_attention_tma_b200 as hs

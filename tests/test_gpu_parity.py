@@ -363,8 +363,8 @@ def test_fused_topk_equals_two_calls_on_ties_and_edges(case):
 
 @pytest.mark.parametrize("name", ["tok_mqa32", "swa_tok"])
 def test_block_with_fused_topk_equals_two_call_block(name):
-    """The block runner's token-level default (top-k inside the score pass)
-    writes exactly what the two-call block writes, every layer."""
+    """The block runner with fuse_topk (top-k inside the score pass) writes
+    exactly what the two-call block writes, every layer."""
     from hybrid_sparse_attention_tma_b200.block import HybridBlock
     w = VARIANTS[name].with_(n_sparse=2)
     inp = W.make_block_inputs(w, device="cuda", seed=17)
