@@ -205,6 +205,12 @@ VARIANTS = {
     # window-exclusive top-k at block level, GQA
     "blk_exclusive": W.Workload("v13", ctx=(64, 0), new=(260, 200), n_q_heads=8, n_kv_heads=2, head_dim=64,
                                 q_tile=32, block=16, topk=4, window=24, n_sparse=1, exclusive=True),
+    # token level with G = 128 (two queries per 256-row score chunk) and with G = 1 (MHA, d = 64: a
+    # 64-query tile fills a quarter of a score chunk)
+    "tok_g128": W.Workload("v14", ctx=(37,), new=(50,), n_q_heads=128, n_kv_heads=1, head_dim=128, q_tile=4,
+                           block=1, topk=24, window=8, n_sparse=1),
+    "tok_mha_d64": W.Workload("v15", ctx=(0, 130), new=(300, 45), n_q_heads=2, n_kv_heads=2, head_dim=64,
+                              q_tile=64, block=1, topk=40, window=16, n_sparse=1),
     # token-level selection with the window branch and gate fused in (one launch per layer)
     "swa_tok": W.Workload("v11", ctx=(0, 300), new=(260, 90), n_q_heads=16, n_kv_heads=1, head_dim=128,
                           q_tile=16, block=1, topk=64, window=8, n_sparse=1, swa_window=32, needle_rate=0.02),
