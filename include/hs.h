@@ -185,12 +185,17 @@ HS_API hs_status hs_topk_select(const hs_varlen* vl, const hs_sel* sel, const fl
  *
  * Outputs o, lse, idx and cnt are exactly those of the two calls in sequence
  * (same selection rule, ties and -1 padding). Token-level prefill (B = 1,
- * not the one-query decode shape): each (tile, KV head)'s top-k is selected
- * by the CTA that finishes its last score range, from the scores still in
- * L2, and those cache lines are then dropped without write-back, so the
- * scores make no HBM round trip and no separate top-k launch runs; `scores`
- * is scratch of the usual [n_tiles, H_kv, n_blk] shape and its content on
- * return is undefined. Other shapes (block-level selection, decode) run the
+ * not the one-query decode shape): the CTA that finishes a (tile, KV head)'s
+ * last score range queues it, and two selector warps of whichever CTA is
+ * free select it while its scores are in L2, then drop those cache lines
+ * without write-back; no separate top-k launch runs, and the scores reach
+ * HBM only where a long context's K stream evicted them first. `scores` is
+ * scratch of the usual [n_tiles, H_kv, n_blk] shape and
+ * its content on return is undefined. The kernels wait across CTAs for
+ * queued planes (bounded: an error, not a hang, if a plane never comes), so
+ * they assume all CTAs of the launch are resident, as they are on an idle
+ * GPU. HybridBlock keeps the two calls by default: on B200 the selection
+ * beside the score pass costs more than the separate launch. Other shapes (block-level selection, decode) run the
  * two calls back to back and `scores` holds the scores as documented there.
  * In: as hs_full_attn_select (lse required at token level). Out: o, lse,
  * idx [n_tiles,H_kv,k], cnt [n_tiles,H_kv] (both required).
