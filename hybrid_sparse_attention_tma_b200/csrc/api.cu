@@ -388,7 +388,7 @@ SparseDecodePlan sparse_decode_plan(const Shape& sh, const hs_sel* sel, int spli
 // Workspace: the header only (the ranges of a unit merge in shared memory).
 size_t sparse_decode_ws_bytes(const Shape&, const hs_sel*) { return kHeaderBytes; }
 
-// Token-level scores: items are (tile, KV head, 512-key range) up to the
+// Token-level scores: items are (tile, KV head, 256-key range) up to the
 // tile's last query position.
 long long token_score_items(const hs_varlen* vl, int T, int Hkv) {
   long long n = 0;

@@ -127,7 +127,7 @@ __device__ __forceinline__ uint32_t aug_off(int r, int half) {
 }
 
 // item -> (tile, g, first key); items are enumerated tile by tile, KV head by
-// KV head, in 512-key ranges up to the tile's last query position.
+// KV head, in 256-key ranges (kBlocks x 128) up to the tile's last query position.
 struct Item {
   int tile, g, key0, nkeys;  // keys [key0, key0 + nkeys)
   TileInfo ti;
@@ -202,7 +202,7 @@ __device__ __forceinline__ Item get_item(const SeqTable& st, const Params& p, co
   return it;
 }
 
-// Prefix sums of items per tile in item order (Hkv * 512-key ranges), one CTA
+// Prefix sums of items per tile in item order (Hkv * 256-key ranges), one CTA
 // of 1024 threads. With `order` (fused top-k) the item order is longest tile
 // first, written to order[], and the top-k's per-plane arrival counters, its
 // queue of completed planes and the queue's two counters are reset.
